@@ -1,0 +1,110 @@
+// C ABI of the library: argument validation on the host, then one kernel launch per call.
+// Declarations, argument meaning, layouts and error behaviour are in include/puro_fp8.h.
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/puro_fp8.h"
+#include "quant.h"
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The kernels are built for sm_100a only: refuse any other device up front.
+int check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PURO_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  return (major == 10 && minor == 0) ? PURO_OK : PURO_ERR_DEVICE;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? PURO_OK : PURO_ERR_LAUNCH; }
+
+}  // namespace
+
+extern "C" {
+
+int puro_fp8_quantize_1x128(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                            int64_t ldq, float *S, puro_stream_t stream) {
+  if (X == nullptr || Xq == nullptr || S == nullptr) return PURO_ERR_NULL;
+  if (R < 1 || C < 128 || C % 128 != 0 || ldx < C || ldq < C) return PURO_ERR_SHAPE;
+  if (R > (1ll << 31) - 1 || C / 128 > 65535) return PURO_ERR_SHAPE;
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(S, 4) || ldx % 8 != 0 || ldq % 16 != 0)
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return from_cuda(puro::launch_quant_rows(X, R, C, ldx, Xq, ldq, S, stream));
+}
+
+int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, int64_t C, int64_t ldx,
+                                       uint8_t *XqT, float *ST, uint8_t *Xq, float *S,
+                                       puro_stream_t stream) {
+  if (X == nullptr || XqT == nullptr || ST == nullptr) return PURO_ERR_NULL;
+  if ((Xq == nullptr) != (S == nullptr)) return PURO_ERR_NULL;
+  if (T < 128 || T % 128 != 0 || C < 8 || C % 8 != 0 || ldx < C) return PURO_ERR_SHAPE;
+  if (Xq != nullptr && C % 128 != 0) return PURO_ERR_SHAPE;
+  if (T / 128 > 65535 || (C + 127) / 128 > (1ll << 31) - 1) return PURO_ERR_SHAPE;
+  if (!aligned(X, 16) || !aligned(XqT, 16) || !aligned(ST, 4) || ldx % 8 != 0)
+    return PURO_ERR_ALIGN;
+  if (Xq != nullptr && (!aligned(Xq, 16) || !aligned(S, 4))) return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return from_cuda(puro::launch_quant_cols(X, T, C, ldx, XqT, ST, Xq, S, stream));
+}
+
+int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
+                              uint8_t *WqT, float *S, puro_stream_t stream) {
+  if (W == nullptr || Wq == nullptr || S == nullptr) return PURO_ERR_NULL;
+  if (R < 1 || C < 128 || C % 128 != 0 || ldw < C) return PURO_ERR_SHAPE;
+  if ((R + 127) / 128 > 65535 || C / 128 > (1ll << 31) - 1) return PURO_ERR_SHAPE;
+  if (WqT != nullptr && R % 16 != 0) return PURO_ERR_SHAPE;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(S, 4) || ldw % 8 != 0)
+    return PURO_ERR_ALIGN;
+  if (WqT != nullptr && !aligned(WqT, 16)) return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return from_cuda(puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, S, stream));
+}
+
+int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                            const float *Bs, uint16_t *C, int64_t M, int64_t N, int64_t K,
+                            int layout, void *workspace, size_t ws_bytes, puro_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  if (Aq == nullptr || As == nullptr || Bq == nullptr || Bs == nullptr || C == nullptr)
+    return PURO_ERR_NULL;
+  if (layout != PURO_FPROP && layout != PURO_DGRAD && layout != PURO_WGRAD)
+    return PURO_ERR_LAYOUT;
+  if (M < 1 || N < 8 || N % 8 != 0 || K < 128 || K % 128 != 0) return PURO_ERR_SHAPE;
+  // 32-bit tensor-map coordinates and kernel indices
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
+  if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16) || !aligned(As, 4) ||
+      !aligned(Bs, layout == PURO_WGRAD ? 16 : 4))
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_gemm_blockwise(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
+}
+
+int puro_fp8_sync_status(puro_stream_t stream) {
+  int status = 0;
+  if (int e = puro::read_and_clear_device_status(stream, &status)) return e;
+  return status != 0 ? PURO_ERR_TIMEOUT : PURO_OK;
+}
+
+const char *puro_strerror(int status) {
+  switch (status) {
+    case PURO_OK: return "ok";
+    case PURO_ERR_NULL: return "a required pointer is NULL";
+    case PURO_ERR_SHAPE: return "invalid size (non-positive, not a multiple of 128 where required, or too large)";
+    case PURO_ERR_ALIGN: return "pointer or leading dimension not aligned as required";
+    case PURO_ERR_LAYOUT: return "unknown GEMM layout";
+    case PURO_ERR_LAUNCH: return "kernel launch failed";
+    case PURO_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case PURO_ERR_WORKSPACE: return "workspace too small";
+    case PURO_ERR_CUDA: return "CUDA runtime or driver call failed (is there a GPU?)";
+    case PURO_ERR_DEVICE: return "the current device is not sm_100 (B200-class)";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,514 @@
+// Blockwise-FP8 GEMM for sm_100a: TMA -> swizzled shared memory -> tcgen05 MMA (E4M3,
+// FP32 accumulate in TMEM) -> FP32 scale promotion on CUDA cores -> BF16.
+//
+// "Paper walkthrough: Puro-2B ...", section "Lever 2: use blockwise FP8 from step zero":
+// the linear-layer GEMMs run in FP8 with local scales, one per 128 elements along the
+// reduction dimension for activations and gradients and one per 128x128 block for
+// weights. The scales change every 128 elements of K, so each 128-wide K block is
+// accumulated on its own by the tensor cores (FP32 partial in TMEM) and added into the
+// running FP32 sum with its two scales:
+//     C[m, n] = sum_kb  sA(kb, m) * sB(kb, n) * P_kb[m, n],   P_kb = Aq[m, kb] . Bq[n, kb]
+//
+// One persistent CTA per SM, tiles of 128 x 256, warp-specialised:
+//   warp 0      TMA producer: A and B tiles of one K block per ring stage (4 stages);
+//               for wgrad also the 256 column scales of B per K block (8-stage ring)
+//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one of two
+//               256-column TMEM buffers, committed to the stage's "empty" barrier and
+//               the buffer's "full" barrier; also owns the TMEM allocation
+//   warps 2-3   idle (they complete warpgroup 0, which hands its registers over)
+//   warps 4..11 promotion + epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 and
+//               columns 128*((w-4)/4) .. +127, i.e. one output row and 128 columns per
+//               thread; partial * (sA * sB) is added into 128 FP32 registers with
+//               packed FP32x2 FMAs; at the end of the tile the sums are rounded to
+//               BF16 and stored.
+// Every mbarrier wait is bounded (wall-clock limit plus an iteration cap). A wait that
+// gives up raises a CTA-wide abort flag and the device status word; all warps then
+// leave their loops, in-flight copies and MMAs are waited for (bounded), and TMEM is
+// freed before the CTA exits.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+
+#include "../../include/puro_fp8.h"
+#include "ptx.cuh"
+#include "quant.h"
+
+namespace puro {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;                  // one scale block of K per stage
+constexpr int STAGES = 4;
+constexpr int SC_STAGES = 8;
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_FIRST_WARP = 4;               // warps 0-3 form warpgroup 0
+constexpr int THREADS = 32 * (EPI_FIRST_WARP + EPI_WARPS);  // 384: three warpgroups
+// Register split. The CTA is launched with LAUNCH_REGS per thread (what ptxas gets for
+// 384 threads and one CTA per SM); warpgroup 0 (TMA, MMA, two idle warps) then gives
+// registers back and the two promotion warpgroups take them:
+//   128 * PRODUCER_REGS + 256 * CONSUMER_REGS == 384 * LAUNCH_REGS  (64512)
+// and per SM sub-partition (one warp of each warpgroup) 32 * (40 + 2 * 232) <= 16384.
+constexpr int LAUNCH_REGS = 168;
+constexpr int PRODUCER_REGS = 40;
+constexpr int CONSUMER_REGS = 232;
+static_assert(128 * PRODUCER_REGS + 256 * CONSUMER_REGS == THREADS * LAUNCH_REGS,
+              "register split must add up to the launch allocation");
+constexpr int A_BYTES = BM * BK;          // 16 KB
+constexpr int B_BYTES = BN * BK;          // 32 KB
+constexpr int SC_BYTES = BN * 4;          // 1 KB
+constexpr uint32_t TMEM_COLS = 2 * BN;    // two FP32 partial buffers
+constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_SC = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_BAR = OFF_SC + SC_STAGES * SC_BYTES;
+constexpr int N_BARS = 2 * STAGES + 4 + 2 * SC_STAGES + 1;
+constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
+constexpr int SMEM_USED = OFF_MISC + 16;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024 bytes
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+struct GemmArgs {
+  const float *As;
+  const float *Bs;
+  uint16_t *C;
+  int M, N, K;
+  int num_m, num_n, kblocks, m_fastest;
+  unsigned long long timeout_ns;
+  int *status;
+};
+
+__device__ int g_status;  // non-zero: a bounded wait gave up since the last read
+
+__device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mt, int &nt) {
+  if (a.m_fastest) {
+    mt = tile % a.num_m;
+    nt = tile / a.num_m;
+  } else {
+    nt = tile % a.num_n;
+    mt = tile / a.num_n;
+  }
+}
+
+__device__ __forceinline__ void raise_abort(volatile int *abort, int *status) {
+  *abort = 1;
+  atomicOr(status, 1);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmS, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + s); };
+  auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + SC_STAGES + s); };
+  const uint32_t drain_bar = bar0 + 8u * (N_BARS - 1);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  const float *sc_smem = reinterpret_cast<const float *>(smem + OFF_SC);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), EPI_WARPS);
+    }
+    for (int s = 0; s < SC_STAGES; ++s) {
+      mbar_init(sfull_bar(s), 1);
+      mbar_init(sempty_bar(s), EPI_WARPS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    if (LAYOUT == PURO_WGRAD) prefetch_tensormap(&tmS);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  const int tiles = args.num_m * args.num_n;
+  const int kblocks = args.kblocks;
+  const uint64_t tmo = args.timeout_ns;
+
+  if (warp < EPI_FIRST_WARP) {
+    // Each role's code sits inside the branch that set its register limit, so ptxas
+    // allocates the promotion path with CONSUMER_REGS and this one with PRODUCER_REGS.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PRODUCER_REGS));
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0, ss = 0;
+      uint32_t ph = 0, sph = 0;
+      uint32_t issued = 0, issued_parity = 0;  // per-stage bit masks
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        int mt, nt;
+        tile_coords(tile, args, mt, nt);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty_bar(s), ph ^ 1u, tmo, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+          tma_load_2d(sbase + OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
+          tma_load_2d(sbase + OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
+          issued |= 1u << s;
+          issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
+          if (LAYOUT == PURO_WGRAD) {
+            if (!mbar_wait(sempty_bar(ss), sph ^ 1u, tmo, abort)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(sfull_bar(ss), SC_BYTES);
+            tma_load_2d(sbase + OFF_SC + ss * SC_BYTES, &tmS, sfull_bar(ss), nt * BN, kb);
+            if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
+          }
+          if (++s == STAGES) s = 0, ph ^= 1u;
+        }
+      }
+      if (!ok) {
+        raise_abort(abort, args.status);
+        // Let every issued tensor load land before the CTA can exit.
+        for (int i = 0; i < STAGES; ++i)
+          if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, use = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        for (int kb = 0; kb < kblocks; ++kb, ++use) {
+          const uint32_t b = use & 1u;
+          if (!mbar_wait(tempty_bar(b), ((use >> 1) & 1u) ^ 1u, tmo, abort) ||
+              !mbar_wait(full_bar(s), ph, tmo, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t d = tmem + b * BN;
+          const uint32_t a_addr = sbase + OFF_A + s * A_BYTES;
+          const uint32_t b_addr = sbase + OFF_B + s * B_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_e4m3(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), IDESC,
+                     k > 0 ? 1u : 0u);
+          mma_commit(empty_bar(s));
+          mma_commit(tfull_bar(b));
+          if (++s == STAGES) s = 0, ph ^= 1u;
+        }
+      }
+      if (!ok) {
+        raise_abort(abort, args.status);
+        mma_commit(drain_bar);  // arrives once every MMA issued above has finished
+        mbar_wait(drain_bar, 0, tmo, nullptr);
+      }
+    }
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(CONSUMER_REGS));
+    // ------------------------------------------------------------ promotion + epilogue
+    const int quad = warp & 3;
+    const int half = (warp - EPI_FIRST_WARP) >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int nb_total = (args.N + 127) / 128;
+    uint32_t use = 0;
+    int ss = 0;
+    uint32_t sph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      int mt, nt;
+      tile_coords(tile, args, mt, nt);
+      const int m = mt * BM + row;
+      const bool m_ok = m < args.M;
+      const int nb = nt * 2 + half;  // 128-wide block of N this warp covers
+      const int n_base = nb * 128;
+      const bool nb_ok = nb < nb_total;
+      uint64_t acc[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] = 0;
+
+      auto load_sa = [&](int kb) -> float {
+        return m_ok ? __ldg(args.As + static_cast<int64_t>(kb) * args.M + m) : 0.0f;
+      };
+      auto load_sb = [&](int kb) -> float {
+        if (LAYOUT == PURO_WGRAD || !nb_ok) return 0.0f;
+        return LAYOUT == PURO_FPROP ? __ldg(args.Bs + static_cast<int64_t>(nb) * kblocks + kb)
+                                    : __ldg(args.Bs + static_cast<int64_t>(kb) * nb_total + nb);
+      };
+      float sa_next = load_sa(0);
+      float sb_next = load_sb(0);
+      for (int kb = 0; kb < kblocks; ++kb, ++use) {
+        const float sa = sa_next;
+        const float sb = sb_next;
+        if (kb + 1 < kblocks) {
+          sa_next = load_sa(kb + 1);
+          sb_next = load_sb(kb + 1);
+        }
+        const uint32_t b = use & 1u;
+        if (!mbar_wait(tfull_bar(b), (use >> 1) & 1u, tmo, abort)) {
+          ok = false;
+          break;
+        }
+        const float *sbv = nullptr;
+        if (LAYOUT == PURO_WGRAD) {
+          if (!mbar_wait(sfull_bar(ss), sph, tmo, abort)) {
+            ok = false;
+            break;
+          }
+          sbv = sc_smem + ss * BN + half * 128;
+        }
+        tc_fence_after_sync();
+        const uint32_t taddr = tmem + lane_base + b * BN + half * 128;
+        const uint64_t s2 = LAYOUT == PURO_WGRAD ? pack2(sa, sa) : pack2(sa * sb, sa * sb);
+        // 16 columns per TMEM load keeps one chunk of partials (and, for wgrad, its column
+        // scales) in registers next to the 128 accumulators.
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[16];
+          tmem_ld_16cols(taddr + 16 * c, r);
+          tmem_wait_ld();
+          if (c == 7) {  // the buffer is fully in registers: hand it back to the MMA warp
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(b));
+          }
+          if (LAYOUT == PURO_WGRAD) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 sb4 = *reinterpret_cast<const float4 *>(sbv + 16 * c + 4 * j);
+              const uint64_t p0 =
+                  fmul2(pack2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s2);
+              const uint64_t p1 =
+                  fmul2(pack2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s2);
+              acc[8 * c + 2 * j] = ffma2(p0, pack2(sb4.x, sb4.y), acc[8 * c + 2 * j]);
+              acc[8 * c + 2 * j + 1] = ffma2(p1, pack2(sb4.z, sb4.w), acc[8 * c + 2 * j + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              acc[8 * c + i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                                     s2, acc[8 * c + i]);
+          }
+        }
+        if (LAYOUT == PURO_WGRAD) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sempty_bar(ss));
+          if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (m_ok) {
+        uint16_t *crow = args.C + static_cast<int64_t>(m) * args.N;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = n_base + 8 * j;
+          if (n < args.N) {
+            float v[8];
+            unpack2(acc[4 * j], v[0], v[1]);
+            unpack2(acc[4 * j + 1], v[2], v[3]);
+            unpack2(acc[4 * j + 2], v[4], v[5]);
+            unpack2(acc[4 * j + 3], v[6], v[7]);
+            const uint4 o = make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]),
+                                       bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
+            *reinterpret_cast<uint4 *>(crow + n) = o;
+          }
+        }
+      }
+    }
+    if (!ok) raise_abort(abort, args.status);
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// Row-major [rows, cols] matrix of `elem` bytes per element, box [box_rows, box_cols].
+bool make_map(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem,
+              uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+              CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long ns = [] {
+    const char *e = std::getenv("PURO_WAIT_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 2000;
+    if (ms < 1) ms = 1;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return ns;
+}
+
+int *device_status_ptr() {
+  int *p = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_status) != cudaSuccess) return nullptr;
+  return p;
+}
+
+template <int LAYOUT>
+int launch_layout(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ts,
+                  const GemmArgs &args, int grid, cudaStream_t stream) {
+  auto kern = k_gemm_blockwise<LAYOUT>;
+  // The register split inside the kernel assumes exactly LAUNCH_REGS per thread at launch;
+  // with any other count the promotion warps' setmaxnreg.inc could wait forever.
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PURO_ERR_CUDA;
+  if (fa.numRegs != LAUNCH_REGS || fa.maxThreadsPerBlock < THREADS) {
+    std::fprintf(stderr, "puro_fp8: GEMM kernel built with %d registers (expected %d); not launched\n",
+                 fa.numRegs, LAUNCH_REGS);
+    return PURO_ERR_LAUNCH;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "puro_fp8: cudaFuncSetAttribute: %s\n", cudaGetErrorString(e));
+    return PURO_ERR_CUDA;
+  }
+  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, ts, args);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr,
+                 "puro_fp8: GEMM launch (grid %d, %d threads, %d B smem): %s "
+                 "[kernel: %d regs, max %d threads/block, max dyn smem %d]\n",
+                 grid, THREADS, SMEM_BYTES, cudaGetErrorString(e), fa.numRegs,
+                 fa.maxThreadsPerBlock, fa.maxDynamicSharedSizeBytes);
+    return PURO_ERR_LAUNCH;
+  }
+  return PURO_OK;
+}
+
+}  // namespace
+
+int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs,
+                          uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
+                          cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  int *status = device_status_ptr();
+  if (status == nullptr) return PURO_ERR_CUDA;
+
+  CUtensorMap ta, tb, ts;
+  if (!make_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, BN, BK,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return PURO_ERR_CUDA;
+  if (layout == PURO_WGRAD) {
+    if (!make_map(&ts, Bs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K / 128, N, 1, BN,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return PURO_ERR_CUDA;
+  } else {
+    ts = tb;  // unused
+  }
+
+  GemmArgs args;
+  args.As = As;
+  args.Bs = Bs;
+  args.C = C;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.num_m = static_cast<int>((M + BM - 1) / BM);
+  args.num_n = static_cast<int>((N + BN - 1) / BN);
+  args.kblocks = static_cast<int>(K / BK);
+  // Walk the smaller operand fastest so that it stays resident in L2 while the larger
+  // one streams through once.
+  args.m_fastest = M <= N ? 1 : 0;
+  args.timeout_ns = wait_timeout_ns();
+  args.status = status;
+  const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+
+  switch (layout) {
+    case PURO_FPROP: return launch_layout<PURO_FPROP>(ta, tb, ts, args, grid, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(ta, tb, ts, args, grid, stream);
+    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(ta, tb, ts, args, grid, stream);
+    default: return PURO_ERR_LAYOUT;
+  }
+}
+
+int read_and_clear_device_status(cudaStream_t stream, int *status_out) {
+  int host = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&host, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  *status_out = host;
+  return PURO_OK;
+}
+
+}  // namespace puro

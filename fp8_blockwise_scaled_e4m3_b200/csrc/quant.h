@@ -1,0 +1,26 @@
+// Internal launchers of the quantiser and GEMM kernels (host side). Arguments are
+// validated by the C-ABI layer before these are called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace puro {
+
+cudaError_t launch_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                              int64_t ldq, float *S, cudaStream_t stream);
+cudaError_t launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint8_t *XqT,
+                              float *ST, uint8_t *Xq, float *S, cudaStream_t stream);
+cudaError_t launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
+                                uint8_t *WqT, float *S, cudaStream_t stream);
+
+// Returns 0 on success, a negative puro_status on failure.
+int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs,
+                          uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
+                          cudaStream_t stream);
+
+// Reads and clears the device status word of the GEMM kernels (after a stream sync).
+int read_and_clear_device_status(cudaStream_t stream, int *status_out);
+
+}  // namespace puro

@@ -1,0 +1,188 @@
+"""Python binding of libpuro_fp8.so: argument marshalling only.
+
+Every function with a ``puro_`` name mirrors the C entry point of the same name in
+``include/puro_fp8.h``: it takes torch tensors that already live on the GPU, passes
+their device pointers, sizes and the current CUDA stream, and raises ``PuroError`` on a
+non-zero status. The convenience functions below them allocate the outputs with torch
+and call the same entry points. Nothing here computes: every step runs in the CUDA
+kernels, and importing this module fails if the library has not been built.
+"""
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+PURO_FPROP, PURO_DGRAD, PURO_WGRAD = 0, 1, 2
+LAYOUTS = {"fprop": PURO_FPROP, "dgrad": PURO_DGRAD, "wgrad": PURO_WGRAD}
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+class PuroError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status} ({strerror(status)})")
+
+
+def _load():
+    if not os.path.exists(LIB):
+        raise ImportError(
+            f"{LIB} is missing: build it with `python -m fp8_blockwise_scaled_e4m3_b200.build`")
+    lib = ctypes.CDLL(LIB)
+    sig = {
+        "puro_fp8_quantize_1x128": [_p, _i64, _i64, _i64, _p, _i64, _p, _p],
+        "puro_fp8_quantize_1x128_transposed": [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+        "puro_fp8_quantize_128x128": [_p, _i64, _i64, _i64, _p, _p, _p, _p],
+        "puro_fp8_gemm_blockwise": [_p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p,
+                                    ctypes.c_size_t, _p],
+        "puro_fp8_sync_status": [_p],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.puro_strerror.argtypes = [ctypes.c_int]
+    lib.puro_strerror.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    """The loaded ctypes.CDLL (for ABI tests)."""
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return _lib.puro_strerror(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise PuroError(status, where)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, dtype, name, rows_contig=True):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if rows_contig and t.dim() == 2 and t.stride(1) != 1:
+        raise ValueError(f"{name} must have unit column stride")
+
+
+def _dense(t, name):
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ------------------------------------------------------------------ C-ABI mirrors
+
+def puro_fp8_quantize_1x128(X, Xq, S, stream=None):
+    _need(X, torch.bfloat16, "X"); _need(Xq, torch.uint8, "Xq"); _need(S, torch.float32, "S")
+    _dense(S, "S")
+    R, C = X.shape
+    with torch.cuda.device(X.device):
+        _check(_lib.puro_fp8_quantize_1x128(_ptr(X), R, C, X.stride(0), _ptr(Xq), Xq.stride(0),
+                                            _ptr(S), _stream(stream)), "puro_fp8_quantize_1x128")
+
+
+def puro_fp8_quantize_1x128_transposed(X, XqT, ST, Xq=None, S=None, stream=None):
+    _need(X, torch.bfloat16, "X"); _need(XqT, torch.uint8, "XqT"); _need(ST, torch.float32, "ST")
+    _need(Xq, torch.uint8, "Xq"); _need(S, torch.float32, "S")
+    for t, n in ((XqT, "XqT"), (ST, "ST"), (Xq, "Xq"), (S, "S")):
+        _dense(t, n)
+    T, C = X.shape
+    with torch.cuda.device(X.device):
+        _check(_lib.puro_fp8_quantize_1x128_transposed(_ptr(X), T, C, X.stride(0), _ptr(XqT), _ptr(ST),
+                                                       _ptr(Xq), _ptr(S), _stream(stream)),
+               "puro_fp8_quantize_1x128_transposed")
+
+
+def puro_fp8_quantize_128x128(W, Wq, WqT, S, stream=None):
+    _need(W, torch.bfloat16, "W"); _need(Wq, torch.uint8, "Wq"); _need(WqT, torch.uint8, "WqT")
+    _need(S, torch.float32, "S")
+    for t, n in ((Wq, "Wq"), (WqT, "WqT"), (S, "S")):
+        _dense(t, n)
+    R, C = W.shape
+    with torch.cuda.device(W.device):
+        _check(_lib.puro_fp8_quantize_128x128(_ptr(W), R, C, W.stride(0), _ptr(Wq), _ptr(WqT), _ptr(S),
+                                              _stream(stream)), "puro_fp8_quantize_128x128")
+
+
+def puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, workspace=None, stream=None):
+    layout = LAYOUTS.get(layout, layout)
+    _need(Aq, torch.uint8, "Aq"); _need(Bq, torch.uint8, "Bq"); _need(C, torch.bfloat16, "C")
+    _need(As, torch.float32, "As"); _need(Bs, torch.float32, "Bs")
+    for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C")):
+        _dense(t, n)
+    M, K = Aq.shape
+    N = Bq.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(Aq.device):
+        _check(_lib.puro_fp8_gemm_blockwise(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
+                                            int(layout), _ptr(workspace), ws_bytes, _stream(stream)),
+               "puro_fp8_gemm_blockwise")
+
+
+def puro_fp8_sync_status(stream=None):
+    _check(_lib.puro_fp8_sync_status(_stream(stream)), "puro_fp8_sync_status")
+
+
+# ------------------------------------------------------------------ allocating helpers
+
+def quantize_1x128(X, stream=None):
+    """X [R, C] bf16 -> (Xq uint8 [R, C], S float32 [C/128, R])."""
+    R, C = X.shape
+    Xq = torch.empty((R, C), dtype=torch.uint8, device=X.device)
+    S = torch.empty((C // 128, R), dtype=torch.float32, device=X.device)
+    puro_fp8_quantize_1x128(X, Xq, S, stream)
+    return Xq, S
+
+
+def quantize_1x128_transposed(X, dual=False, stream=None):
+    """X [T, C] bf16 -> (XqT [C, T], ST [T/128, C]) and, if dual, also (Xq, S) row-wise."""
+    T, C = X.shape
+    XqT = torch.empty((C, T), dtype=torch.uint8, device=X.device)
+    ST = torch.empty((T // 128, C), dtype=torch.float32, device=X.device)
+    Xq = S = None
+    if dual:
+        Xq = torch.empty((T, C), dtype=torch.uint8, device=X.device)
+        S = torch.empty((C // 128, T), dtype=torch.float32, device=X.device)
+    puro_fp8_quantize_1x128_transposed(X, XqT, ST, Xq, S, stream)
+    return (XqT, ST, Xq, S) if dual else (XqT, ST)
+
+
+def quantize_128x128(W, transposed=True, stream=None):
+    """W [R, C] bf16 -> (Wq [R, C], WqT [C, R] or None, S [ceil(R/128), C/128])."""
+    R, C = W.shape
+    Wq = torch.empty((R, C), dtype=torch.uint8, device=W.device)
+    WqT = torch.empty((C, R), dtype=torch.uint8, device=W.device) if transposed else None
+    S = torch.empty(((R + 127) // 128, C // 128), dtype=torch.float32, device=W.device)
+    puro_fp8_quantize_128x128(W, Wq, WqT, S, stream)
+    return Wq, WqT, S
+
+
+def gemm(Aq, As, Bq, Bs, layout, out=None, stream=None):
+    """C [M, N] bf16 = blockwise GEMM of the given operands (see puro_fp8_gemm_blockwise)."""
+    M, N = Aq.shape[0], Bq.shape[0]
+    C = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=Aq.device)
+    puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, None, stream)
+    return C

@@ -1,0 +1,156 @@
+/*
+ * puro_fp8.h -- C ABI of the blockwise-FP8 (E4M3) linear-layer library for B200 (sm_100a).
+ *
+ * The method ("Paper walkthrough: Puro-2B -- pretraining a 2B model from scratch for
+ * $6.9K on consumer GPUs", section "Lever 2: use blockwise FP8 from step zero"): only
+ * the linear-layer GEMMs run in FP8, FP8 is a compute format and not a storage format,
+ * and scales are local -- activations and their gradients get one scale per 128
+ * consecutive elements along the reduction dimension, weights one scale per 128x128
+ * block. Readings this library takes where the page is silent: the FP8 format is E4M3
+ * (bias 7, max 448, no infinities, 0x7F/0xFF NaN); a block's scale is s = amax / 448,
+ * a correctly rounded FP32 division, computed from the tensor being quantised (no
+ * amax history); a code is E4M3(x / s) with a correctly rounded FP32 division, then
+ * round-to-nearest-even saturating to +-448; an all-zero block has s = 0 and signed
+ * zero codes. GEMM partial sums are FP32 per 128-wide K block, promoted with the two
+ * scales in FP32, output BF16 (round to nearest even).
+ *
+ * Conventions for every entry point:
+ *  - Every pointer is a DEVICE pointer to memory the caller owns and allocated; the
+ *    library allocates nothing and keeps no reference after the call is enqueued.
+ *  - BF16 data is passed as uint16_t bit patterns; FP8 codes as uint8_t; scales float.
+ *  - Matrices are row-major. Leading dimensions are in elements.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default stream).
+ *  - Arguments are checked on the host before anything is launched; a failed check
+ *    returns a negative puro_status and enqueues nothing.
+ *  - Inputs must be finite (no NaN / Inf); this is not checked.
+ *  - Calls are stateless and thread-safe; the only global state is the device status
+ *    word read by puro_fp8_sync_status().
+ */
+#ifndef PURO_FP8_H
+#define PURO_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PURO_API __attribute__((visibility("default")))
+#else
+#define PURO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (ABI-identical to cudaStream_t / CUstream). */
+typedef struct CUstream_st *puro_stream_t;
+
+typedef enum {
+  PURO_OK = 0,
+  PURO_ERR_NULL = -1,      /* a required pointer is NULL                               */
+  PURO_ERR_SHAPE = -2,     /* a size is <= 0, a reduction dim is not a multiple of 128,
+                              or a leading dimension is smaller than the row length     */
+  PURO_ERR_ALIGN = -3,     /* a pointer or leading dimension breaks the 16-byte rule    */
+  PURO_ERR_LAYOUT = -4,    /* unknown GEMM layout                                       */
+  PURO_ERR_LAUNCH = -5,    /* the CUDA launch failed (cudaGetLastError after launch)    */
+  PURO_ERR_TIMEOUT = -6,   /* a bounded device-side wait gave up (see sync_status)      */
+  PURO_ERR_WORKSPACE = -7, /* workspace too small for the requested split               */
+  PURO_ERR_CUDA = -8,      /* another CUDA runtime / driver call failed                 */
+  PURO_ERR_DEVICE = -9     /* the current device is not sm_100 (B200-class)             */
+} puro_status;
+
+/* Operand layouts of puro_fp8_gemm_blockwise (see there). */
+enum { PURO_FPROP = 0, PURO_DGRAD = 1, PURO_WGRAD = 2 };
+
+/*
+ * 1x128 quantisation along the columns (the reduction dimension) of X [R, C].
+ * Source: "Lever 2: use blockwise FP8 from step zero" -- activations and their
+ * gradients in groups of 128 along the reduction dimension. Used for the forward
+ * activation (fprop A operand) and for dY (dgrad A operand).
+ *
+ *   X   [R, C] BF16, row stride ldx (>= C)         input
+ *   Xq  [R, C] E4M3 codes, row stride ldq (>= C)   output
+ *   S   [C/128, R] float, dense                   output; S[j*R + r] is the scale of
+ *                                                  X[r, 128j .. 128j+127]
+ * Requires R >= 1, C >= 128, C % 128 == 0; X, Xq 16-byte aligned, ldx % 8 == 0,
+ * ldq % 16 == 0; S 4-byte aligned.
+ */
+PURO_API int puro_fp8_quantize_1x128(const uint16_t *X, int64_t R, int64_t C, int64_t ldx,
+                            uint8_t *Xq, int64_t ldq, float *S, puro_stream_t stream);
+
+/*
+ * 1x128 quantisation along the rows (tokens) of X [T, C], written transposed.
+ * Source: "Lever 2: use blockwise FP8 from step zero" -- gradients (and activations)
+ * in groups of 128 along the reduction dimension; for the weight-gradient GEMM
+ * dW = dY^T X that dimension is the token dimension, so both of its operands are
+ * re-quantised from BF16 in 128-token groups.
+ *
+ *   X    [T, C] BF16, row stride ldx (>= C)   input (tokens are rows)
+ *   XqT  [C, T] E4M3 codes, dense              output; XqT[c, t] is the code of X[t, c]
+ *   ST   [T/128, C] float, dense               output; ST[b*C + c] is the scale of
+ *                                              X[128b .. 128b+127, c]
+ *   Xq, S  optional (both NULL or both set): the row-wise 1x128 quantisation of the
+ *          same X (exactly what puro_fp8_quantize_1x128 writes with ldq = C), made
+ *          from the same read of X. Requires C % 128 == 0 when set.
+ * Requires T >= 128, T % 128 == 0, C >= 8, C % 8 == 0; X 16-byte aligned, ldx % 8 == 0;
+ * XqT, Xq 16-byte aligned.
+ */
+PURO_API int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, int64_t C, int64_t ldx,
+                                       uint8_t *XqT, float *ST, uint8_t *Xq, float *S,
+                                       puro_stream_t stream);
+
+/*
+ * 128x128 block quantisation of a weight W [R, C] (R = output features, C = input
+ * features, the forward reduction dimension).
+ * Source: "Lever 2: use blockwise FP8 from step zero" -- weights in 128x128 blocks.
+ *
+ *   W    [R, C] BF16, row stride ldw (>= C)   input
+ *   Wq   [R, C] E4M3 codes, dense             output (fprop B operand)
+ *   WqT  [C, R] E4M3 codes, dense, optional   output: the same codes transposed (dgrad
+ *                                             B operand); NULL to skip. Needs R % 16 == 0.
+ *   S    [ceil(R/128), C/128] float, dense    output; S[i*(C/128) + j] is the scale of
+ *                                             block (i, j). A partial last row block
+ *                                             takes its amax over the rows that exist.
+ * Requires R >= 1, C % 128 == 0; W, Wq, WqT 16-byte aligned, ldw % 8 == 0.
+ */
+PURO_API int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t ldw,
+                              uint8_t *Wq, uint8_t *WqT, float *S, puro_stream_t stream);
+
+/*
+ * Blockwise-FP8 GEMM  C[m, n] = sum_kb sA(kb, m) * sB(kb, n) * sum_{k in kb} A[m, k] B[n, k]
+ * with an FP32 tensor-core partial per 128-wide K block, FP32 promotion and BF16 output.
+ * Source: "Lever 2: use blockwise FP8 from step zero" (the linear-layer GEMMs in FP8
+ * with local scales); forward, dgrad and wgrad of one linear layer are the three
+ * layouts below.
+ *
+ *   Aq  [M, K] E4M3 codes, dense      As [K/128, M] float    (1x128 along K)
+ *   Bq  [N, K] E4M3 codes, dense      Bs depends on layout:
+ *     PURO_FPROP  Y  = X W^T:   Bq = Wq,  Bs = S of W  [ceil(N/128), K/128]
+ *     PURO_DGRAD  dX = dY W:    Bq = WqT, Bs = S of W  [K/128, ceil(N/128)]
+ *     PURO_WGRAD  dW = dY^T X:  Bq = XqT, Bs = ST of X [K/128, N]
+ *   C   [M, N] BF16, dense            output
+ *   workspace, ws_bytes   reserved for split-K; may be NULL / 0.
+ * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, Bq, C 16-byte aligned;
+ * As, Bs 4-byte aligned (Bs 16-byte aligned for PURO_WGRAD). M and N need not be
+ * multiples of the tile size.
+ */
+PURO_API int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                            const float *Bs, uint16_t *C, int64_t M, int64_t N, int64_t K,
+                            int layout, void *workspace, size_t ws_bytes,
+                            puro_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that kernels
+ * set when a bounded wait gives up. Returns PURO_OK, PURO_ERR_TIMEOUT, or
+ * PURO_ERR_CUDA if the synchronisation itself reported an error.
+ */
+PURO_API int puro_fp8_sync_status(puro_stream_t stream);
+
+/* Human-readable text of a puro_status value (static storage, never NULL). */
+PURO_API const char *puro_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PURO_FP8_H */

@@ -1,0 +1,108 @@
+"""The C-ABI library builds, loads and exports every entry point include/puro_fp8.h declares,
+and rejects bad arguments on the host with the documented status codes.
+
+No call here carries arguments that pass validation, so nothing is ever launched: these
+tests are safe with or without a GPU (the fake pointers never reach a kernel).
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "puro_fp8.h")
+
+OK, ENULL, ESHAPE, EALIGN, ELAYOUT, ECUDA = 0, -1, -2, -3, -4, -8
+A16 = 0x10000  # a 16-byte-aligned fake address (never dereferenced)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_blockwise_scaled_e4m3_b200 import build
+    build.build()
+    from fp8_blockwise_scaled_e4m3_b200 import puro_fp8
+    return puro_fp8.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"PURO_API\s+[\w\s\*]+?\b(puro_\w+)\s*\(", text)))
+
+
+def exported_symbols(path):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    return sorted({line.split()[-1] for line in out.splitlines() if line.split()[-1].startswith("puro_")})
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert names == sorted([
+        "puro_fp8_quantize_1x128", "puro_fp8_quantize_1x128_transposed", "puro_fp8_quantize_128x128",
+        "puro_fp8_gemm_blockwise", "puro_fp8_sync_status", "puro_strerror"]) or set(names) >= {
+        "puro_fp8_quantize_1x128", "puro_fp8_quantize_1x128_transposed", "puro_fp8_quantize_128x128",
+        "puro_fp8_gemm_blockwise", "puro_fp8_sync_status", "puro_strerror"}
+
+
+def test_library_exports_exactly_the_declared_symbols(lib):
+    from fp8_blockwise_scaled_e4m3_b200.build import LIB
+    assert exported_symbols(LIB) == declared_functions()
+    for name in declared_functions():
+        assert hasattr(lib, name)
+
+
+def test_strerror_covers_every_status(lib):
+    for s in range(-9, 1):
+        assert lib.puro_strerror(s) and lib.puro_strerror(s) != b"unknown status"
+    assert lib.puro_strerror(-1234) == b"unknown status"
+
+
+def test_quantize_1x128_validation(lib):
+    f = lib.puro_fp8_quantize_1x128
+    assert f(None, 4, 128, 128, A16, 128, A16, None) == ENULL
+    assert f(A16, 0, 128, 128, A16, 128, A16, None) == ESHAPE
+    assert f(A16, 4, 100, 128, A16, 128, A16, None) == ESHAPE      # C % 128
+    assert f(A16, 4, 256, 128, A16, 256, A16, None) == ESHAPE      # ldx < C
+    assert f(A16 + 2, 4, 128, 128, A16, 128, A16, None) == EALIGN  # X not 16-byte aligned
+    assert f(A16, 4, 128, 132, A16, 128, A16, None) == EALIGN      # ldx % 8
+    assert f(A16, 4, 128, 128, A16, 136, A16, None) == EALIGN      # ldq % 16
+
+
+def test_quantize_transposed_validation(lib):
+    f = lib.puro_fp8_quantize_1x128_transposed
+    assert f(A16, 256, 64, 64, None, A16, None, None, None) == ENULL
+    assert f(A16, 256, 64, 64, A16, A16, A16, None, None) == ENULL   # Xq without S
+    assert f(A16, 200, 64, 64, A16, A16, None, None, None) == ESHAPE  # T % 128
+    assert f(A16, 256, 60, 64, A16, A16, None, None, None) == ESHAPE  # C % 8
+    assert f(A16, 256, 64, 64, A16, A16, A16, A16, None) == ESHAPE    # dual needs C % 128
+    assert f(A16, 256, 64, 64, A16 + 8, A16, None, None, None) == EALIGN
+
+
+def test_quantize_128x128_validation(lib):
+    f = lib.puro_fp8_quantize_128x128
+    assert f(A16, 300, 256, 256, None, None, A16, None) == ENULL
+    assert f(A16, 300, 200, 256, A16, None, A16, None) == ESHAPE
+    assert f(A16, 300, 256, 256, A16, A16, A16, None) == ESHAPE      # WqT needs R % 16
+    assert f(A16, 304, 256, 256, A16, A16 + 4, A16, None) == EALIGN
+
+
+def test_gemm_validation(lib):
+    f = lib.puro_fp8_gemm_blockwise
+    args = [A16, A16, A16, A16, A16]
+    assert f(None, *args[1:], 128, 256, 256, 0, None, 0, None) == ENULL
+    assert f(*args, 128, 256, 256, 7, None, 0, None) == ELAYOUT
+    assert f(*args, 0, 256, 256, 0, None, 0, None) == ESHAPE
+    assert f(*args, 128, 250, 256, 0, None, 0, None) == ESHAPE       # N % 8
+    assert f(*args, 128, 256, 200, 0, None, 0, None) == ESHAPE       # K % 128
+    assert f(A16 + 1, *args[1:], 128, 256, 256, 0, None, 0, None) == EALIGN
+    assert f(*args[:3], A16 + 4, A16, 128, 256, 256, 2, None, 0, None) == EALIGN  # wgrad Bs
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_without_gpu_calls_report_cuda_error(lib):
+    assert lib.puro_fp8_sync_status(None) == ECUDA
