@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the blockwise-FP8 (E4M3) linear path on B200.
+
+One step = every quantise and GEMM call of one training micro-step of a
+Qwen3-1.7B-shaped model with an untied LM head (28 blocks of QKV, O, gate/up and down
+linears plus the 151936-wide head) over one micro-batch of 2 x 4096 = 8192 tokens:
+  forward sweep  (blocks 0..27, head):  quantise X (1x128), quantise W (128x128, with
+                                        the transposed codes), fprop GEMM
+  backward sweep (head, blocks 27..0):  quantise dY (1x128 along tokens + row-wise, one
+                                        read), quantise X along tokens, dgrad and wgrad
+That is 7 launches per linear, 791 per step, 84.56 TFLOP of GEMM work (2MNK, i.e.
+6 x linear parameters x tokens) and ~40 GB of quantiser traffic. Inputs are seeded
+synthetic BF16 tensors resident in HBM (about 21 GB, distinct per block, so every step
+reads far more than the 126 MB L2).
+
+Printed (rank 0): one JSON line. `value` is GEMM TFLOP/s of the whole step (quantisers
+included in the time), summed over ranks; `roofline` is the GEMM kernel alone (CUDA
+events around every launch in the timed region) against the tensor peak; `roofline_quant`
+the quantisers against HBM bandwidth; `cpu_baseline` the CPU oracle on a bounded
+sample; `e2e` the same step through the public API with the inputs copied from pinned
+host memory and the weight gradients copied back, inside the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: launch with torchrun; each rank runs its own micro-batch (weak scaling, no
+collective in the data path; the timing is the max over ranks).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 blockwise GEMM TFLOP/s (fwd+dgrad+wgrad, Qwen3-1.7B shapes) and % FP8 peak"
+FP8_DENSE_PEAK_TFLOPS = 4500.0  # nominal B200 dense FP8
+WORKLOAD = "qwen3-1.7b-linear-stack-28L+lm_head fwd+dgrad+wgrad, 8192 tokens (2x4096)"
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--tokens", type=int, default=8192)
+    p.add_argument("--layers", type=int, default=28)
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks sampler
+
+class Clocks:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        self.proc = None
+        self.gpu_index = gpu_index
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self, t_begin, t_end):
+        """Stops sampling; summarises the samples taken between host times t_begin and t_end."""
+        import datetime
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(c[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    clk, clk_max = float(c[1]), float(c[2])
+                except ValueError:
+                    continue
+                if not (t_begin <= ts <= t_end):
+                    continue
+                sm.append(clk)
+                mx.append(clk_max)
+                for name, v in zip(names, c[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ the GPU step
+
+class Step:
+    """All buffers of one micro-step and the sequence of library calls over them."""
+
+    def __init__(self, pf, wl, tokens, layers, device, seed):
+        import torch
+        self.pf, self.torch = pf, torch
+        T = tokens
+        self.tokens = T
+        self.linears = []  # (tag, X, W, dY, wq, wqt, ws) in forward order
+        for l in range(layers):
+            fwd = wl.layer_forward(seed, T, device, layer=l)
+            grads = wl.layer_grads(seed, T, device, layer=l)
+            for (name, x, w), (_, dy) in zip(fwd, grads):
+                self.linears.append([f"L{l}.{name}", x, w, dy])
+        h, w_head, dl = wl.lm_head(seed, T, device)
+        self.linears.append(["lm_head", h, w_head, dl])
+        torch.cuda.synchronize()
+        self.scratch = {}
+        u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
+        for lin in self.linears:
+            _, x, w, dy = lin
+            n, k = w.shape
+            lin += [torch.empty((n, k), dtype=u8, device=device),           # Wq
+                    torch.empty((k, n), dtype=u8, device=device),           # WqT
+                    torch.empty(((n + 127) // 128, k // 128), dtype=f32, device=device)]  # Ws
+            if (n, k) not in self.scratch:
+                e = lambda *s, dt=u8: torch.empty(s, dtype=dt, device=device)
+                self.scratch[(n, k)] = dict(
+                    xq=e(T, k), xs=e(k // 128, T, dt=f32),
+                    dyq=e(T, n), dys=e(n // 128, T, dt=f32),
+                    dyqt=e(n, T), dyst=e(T // 128, n, dt=f32),
+                    xqt=e(k, T), xst=e(T // 128, k, dt=f32),
+                    y=e(T, n, dt=bf), dx=e(T, k, dt=bf), dw=e(n, k, dt=bf))
+        self.gemm_flops = sum(3 * 2 * T * lin[2].shape[0] * lin[2].shape[1] for lin in self.linears)
+        # algorithmic quantiser bytes: BF16 read + code writes + FP32 scale writes
+        qb = 0
+        for _, x, w, dy, *_ in self.linears:
+            n, k = w.shape
+            qb += T * k * (2 + 1) + 4 * T * (k // 128)                  # X row-wise
+            qb += n * k * (2 + 2) + 4 * (n // 128) * (k // 128)         # W + WqT
+            qb += T * n * (2 + 2) + 4 * (T * (n // 128) + (T // 128) * n)  # dY dual
+            qb += T * k * (2 + 1) + 4 * (T // 128) * k                  # X along tokens
+        self.quant_bytes = qb
+        self.launches_per_step = 7 * len(self.linears)
+
+    def run(self, ev=None, stream=None, after_wgrad=None):
+        """Enqueue one step. ev: list to which (kind, event) pairs are appended after
+        each launch (an initial event must already be recorded). after_wgrad(i, dW) is
+        called right after linear i's wgrad is enqueued (its dW buffer is reused by the
+        next linear of the same shape)."""
+        pf = self.pf
+        rec = (lambda kind: ev.append((kind, _record(self.torch)))) if ev is not None else (lambda kind: None)
+        for tag, x, w, dy, wq, wqt, ws in self.linears:
+            s = self.scratch[tuple(w.shape)]
+            pf.puro_fp8_quantize_1x128(x, s["xq"], s["xs"], stream); rec("q")
+            pf.puro_fp8_quantize_128x128(w, wq, wqt, ws, stream); rec("q")
+            pf.puro_fp8_gemm_blockwise(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, None, stream); rec("g")
+        for i in range(len(self.linears) - 1, -1, -1):
+            tag, x, w, dy, wq, wqt, ws = self.linears[i]
+            s = self.scratch[tuple(w.shape)]
+            pf.puro_fp8_quantize_1x128_transposed(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], stream); rec("q")
+            pf.puro_fp8_quantize_1x128_transposed(x, s["xqt"], s["xst"], None, None, stream); rec("q")
+            pf.puro_fp8_gemm_blockwise(s["dyq"], s["dys"], wqt, ws, s["dx"], pf.PURO_DGRAD, None, stream); rec("g")
+            pf.puro_fp8_gemm_blockwise(s["dyqt"], s["dyst"], s["xqt"], s["xst"], s["dw"], pf.PURO_WGRAD, None,
+                                       stream); rec("g")
+            if after_wgrad is not None:
+                after_wgrad(i, s["dw"])
+
+
+def _record(torch):
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()
+    return e
+
+
+def _dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def _barrier_sync(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def _max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def oracle_linear_sample(tokens, seed=0):
+    """The oracle on one O-projection linear (2048 -> 2048) over `tokens` tokens: all its
+    quantise calls plus fprop, dgrad and wgrad. Returns (GEMM FLOPs, seconds)."""
+    from fp8_blockwise_scaled_e4m3_b200 import workloads as wl
+    from oracle import gemm as og
+    from oracle import quant as oq
+    g = wl.generator(seed, 0, "cpu")
+    x = wl.bf16_bits(wl.bf16(wl.heavy_tailed((tokens, 2048), 1.0, g, "cpu")))
+    w = wl.bf16_bits(wl.bf16(wl.normal((2048, 2048), wl.WEIGHT_STD, g, "cpu")))
+    dy = wl.bf16_bits(wl.bf16(wl.heavy_tailed((tokens, 2048), wl.GRAD_STD, g, "cpu")))
+    t0 = time.perf_counter()
+    xq, xs = oq.quant_1x128(x)
+    wq, wqt, ws = oq.quant_128x128(w)
+    og.gemm_ref(xq, xs, wq, ws, "fprop")
+    dyq, dys = oq.quant_1x128(dy)
+    dyt, dyst = oq.quant_1x128_transposed(dy)
+    xt, xst = oq.quant_1x128_transposed(x)
+    og.gemm_ref(dyq, dys, wqt, ws, "dgrad")
+    og.gemm_ref(dyt, dyst, xt, xst, "wgrad")
+    dt = time.perf_counter() - t0
+    return 3 * 2 * tokens * 2048 * 2048, dt
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(tokens):
+    flops, dt = oracle_linear_sample(tokens)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _cpu_threads(),
+            "kind": "oracle",
+            "sample": f"CPU oracle (NumPy; FP32 quantisers single-threaded, FP64 GEMMs on the BLAS "
+                      f"threads) on one O-projection linear 2048->2048 at {tokens} tokens: its quantise "
+                      f"calls + fprop/dgrad/wgrad, {flops / 1e9:.1f} GFLOP in {dt:.2f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = _dist_setup(args.gpus)
+    if rank != 0:
+        return
+    tokens = 2048
+    for _ in range(args.warmup):
+        oracle_linear_sample(tokens)
+    flops = dt = 0.0
+    for _ in range(args.steps):
+        f, t = oracle_linear_sample(tokens)
+        flops, dt = flops + f, dt + t
+    v = flops / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "reference_sample": f"O-projection linear at {tokens} tokens per step"},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": _cpu_threads(), "kind": "oracle",
+                             "sample": f"one O-projection linear 2048->2048 at {tokens} tokens per step"},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def run_ours(args):
+    import torch
+    from fp8_blockwise_scaled_e4m3_b200 import puro_fp8 as pf
+    from fp8_blockwise_scaled_e4m3_b200 import workloads as wl
+
+    rank, world, local = _dist_setup(args.gpus)
+    device = torch.device("cuda", torch.cuda.current_device())
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
+
+    step = Step(pf, wl, args.tokens, args.layers, device, seed=4 + 1000 * rank)
+    stream = torch.cuda.current_stream()
+
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()  # sampling starts before the warm-up; only the timed region is kept
+    for _ in range(args.warmup):
+        step.run(stream=stream)
+    pf.puro_fp8_sync_status()
+    _barrier_sync(world)
+
+    t_begin = time.time()
+    events = []
+    start = _record(torch)
+    events.append(("start", start))
+    for _ in range(args.steps):
+        step.run(ev=events, stream=stream)
+    end = events[-1][1]
+    end.synchronize()
+    _barrier_sync(world)
+    clk = clocks.stop(t_begin, time.time())
+    pf.puro_fp8_sync_status()
+
+    ms_total = start.elapsed_time(end)
+    ms_total = _max_over_ranks(ms_total, world)
+    t_gemm = t_quant = 0.0
+    n_gemm = n_quant = 0
+    for (_, e0), (kind, e1) in zip(events[:-1], events[1:]):
+        dt = e0.elapsed_time(e1)
+        if kind == "g":
+            t_gemm, n_gemm = t_gemm + dt, n_gemm + 1
+        else:
+            t_quant, n_quant = t_quant + dt, n_quant + 1
+
+    ms_step = ms_total / args.steps
+    value = world * step.gemm_flops / (ms_step * 1e-3) / 1e12
+    gemm_tflops = step.gemm_flops * args.steps / (t_gemm * 1e-3) / 1e12
+    quant_gbs = step.quant_bytes * args.steps / (t_quant * 1e-3) / 1e9
+    fp8_peak_measured = 2.0 * bf16_tf_sus  # FP8 dense = 2 x BF16 dense (nominal ratio)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_gpu": args.tokens, "layers": args.layers,
+                   "lm_head": True, "gemm_tflop_per_step": round(step.gemm_flops / 1e12, 4),
+                   "quant_gb_per_step": round(step.quant_bytes / 1e9, 3),
+                   "l2": "inputs larger than L2: %.1f GB of distinct BF16 inputs read per step" % (
+                       sum(t.numel() * 2 for lin in step.linears for t in lin[1:4]) / 1e9),
+                   "parallelism": f"dp{world} (independent micro-batches, no collective)"},
+        "frac_of_fp8_peak": round(value / world / FP8_DENSE_PEAK_TFLOPS, 4),
+        "roofline": {"bound": "tensor", "kernel": "k_gemm_blockwise (all fprop/dgrad/wgrad launches)",
+                     "achieved": round(gemm_tflops, 2), "peak": round(fp8_peak_measured, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / fp8_peak_measured, 4),
+                     "peak_note": f"2 x {peak_src} sustained BF16 ({bf16_tf_sus}); "
+                                  f"frac of nominal 4.5 PF = {gemm_tflops / FP8_DENSE_PEAK_TFLOPS:.4f}",
+                     "traffic": None,
+                     "launches_timed": n_gemm, "avg_launch_ms": round(t_gemm / max(n_gemm, 1), 4)},
+        "roofline_quant": {"bound": "hbm", "kernel": "quantisers (k_quant_rows/cols/weight)",
+                           "achieved": round(quant_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
+                           "frac": round(quant_gbs / hbm_gbs, 4),
+                           "peak_note": f"{peak_src} copy bandwidth; frac of nominal 8 TB/s = "
+                                        f"{quant_gbs / 8000:.4f}",
+                           "launches_timed": n_quant, "avg_launch_ms": round(t_quant / max(n_quant, 1), 4)},
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clk,
+    }
+
+    # ---------------------------------------------------------------- e2e (host buffers)
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(step, torch, pf, args, world)
+
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(args.tokens)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(step, torch, pf, args, world):
+    """The same step through the public API with host buffers: every step copies the BF16
+    inputs (X, W, dY of every linear) from pinned host memory and reads the weight
+    gradients back into pinned host memory, inside the timed region."""
+    try:
+        host_in = []
+        for lin in step.linears:
+            host_in.append([torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in lin[1:4]])
+            for h, t in zip(host_in[-1], lin[1:4]):
+                h.copy_(t)
+        host_dw = [torch.empty(lin[2].shape, dtype=torch.bfloat16, pin_memory=True) for lin in step.linears]
+    except RuntimeError as e:  # pinned host memory exhausted
+        return {"unavailable": f"pinned host buffers could not be allocated: {e}"[:200]}
+    h2d = sum(t.numel() * t.element_size() for ts in host_in for t in ts)
+    d2h = sum(t.numel() * t.element_size() for t in host_dw)
+
+    def one_step():
+        for lin, hs in zip(step.linears, host_in):
+            for dev_t, h in zip(lin[1:4], hs):
+                dev_t.copy_(h, non_blocking=True)
+        step.run(after_wgrad=lambda i, dw: host_dw[i].copy_(dw, non_blocking=True))
+
+    one_step()
+    _barrier_sync(world)
+    steps = max(1, args.e2e_steps)
+    t0 = _record(torch)
+    for _ in range(steps):
+        one_step()
+    t1 = _record(torch)
+    t1.synchronize()
+    _barrier_sync(world)
+    ms = _max_over_ranks(t0.elapsed_time(t1), world) / steps
+    return {"value": round(world * step.gemm_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

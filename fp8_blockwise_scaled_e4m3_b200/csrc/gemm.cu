@@ -298,34 +298,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after_sync();
         const uint32_t taddr = tmem + lane_base + b * BN + half * 128;
         const uint64_t s2 = LAYOUT == PURO_WGRAD ? pack2(sa, sa) : pack2(sa * sb, sa * sb);
-        // 16 columns per TMEM load keeps one chunk of partials (and, for wgrad, its column
-        // scales) in registers next to the 128 accumulators.
+        // Two TMEM loads of 64 columns each, one wait per load: the load latency is
+        // paid twice per K block, and 64 partials fit next to the 128 accumulators.
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t r[16];
-          tmem_ld_16cols(taddr + 16 * c, r);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[64];
+          tmem_ld_64cols(taddr + 64 * c, r);
           tmem_wait_ld();
-          if (c == 7) {  // the buffer is fully in registers: hand it back to the MMA warp
+          if (c == 1) {  // the buffer is fully in registers: hand it back to the MMA warp
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(b));
           }
           if (LAYOUT == PURO_WGRAD) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float4 sb4 = *reinterpret_cast<const float4 *>(sbv + 16 * c + 4 * j);
+            for (int j = 0; j < 16; ++j) {
+              const float4 sb4 = *reinterpret_cast<const float4 *>(sbv + 64 * c + 4 * j);
               const uint64_t p0 =
                   fmul2(pack2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s2);
               const uint64_t p1 =
                   fmul2(pack2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s2);
-              acc[8 * c + 2 * j] = ffma2(p0, pack2(sb4.x, sb4.y), acc[8 * c + 2 * j]);
-              acc[8 * c + 2 * j + 1] = ffma2(p1, pack2(sb4.z, sb4.w), acc[8 * c + 2 * j + 1]);
+              acc[32 * c + 2 * j] = ffma2(p0, pack2(sb4.x, sb4.y), acc[32 * c + 2 * j]);
+              acc[32 * c + 2 * j + 1] = ffma2(p1, pack2(sb4.z, sb4.w), acc[32 * c + 2 * j + 1]);
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              acc[8 * c + i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
-                                     s2, acc[8 * c + i]);
+            for (int i = 0; i < 32; ++i)
+              acc[32 * c + i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                                      s2, acc[32 * c + i]);
           }
         }
         if (LAYOUT == PURO_WGRAD) {

@@ -21,6 +21,7 @@
 #include <cstdint>
 
 #include "quant.h"
+#include "quant_math.cuh"
 
 namespace puro {
 namespace {
@@ -40,11 +41,12 @@ __device__ __forceinline__ uint4 load_stream(const uint16_t *p) {
 }
 
 // Four quotients -> four E4M3 codes, first argument in the lowest byte.
-__device__ __forceinline__ uint32_t codes4(float a, float b, float c, float d, float div) {
-  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(a, div), __fdiv_rn(b, div)),
-                                               __NV_SATFINITE, __NV_E4M3);
-  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(c, div), __fdiv_rn(d, div)),
-                                               __NV_SATFINITE, __NV_E4M3);
+__device__ __forceinline__ uint32_t codes4(float a, float b, float c, float d,
+                                           const BlockDivider &div) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+      make_float2(block_divide(div, a), block_divide(div, b)), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+      make_float2(block_divide(div, c), block_divide(div, d)), __NV_SATFINITE, __NV_E4M3);
   return lo | (hi << 16);
 }
 
@@ -56,15 +58,15 @@ __device__ __forceinline__ float absmax8(const uint4 &v) {
   return m;
 }
 
-__device__ __forceinline__ uint2 codes8(const uint4 &v, float div) {
+__device__ __forceinline__ uint2 codes8(const uint4 &v, const BlockDivider &div) {
   return make_uint2(codes4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), div),
                     codes4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w), div));
 }
 
-// Scale of a block with absolute maximum `amax`, and the divisor to use for its codes.
-__device__ __forceinline__ void block_scale(float amax, float &s, float &div) {
+// Scale of a block with absolute maximum `amax`, and the divider for its codes.
+__device__ __forceinline__ void block_scale(float amax, float &s, BlockDivider &div) {
   s = __fdiv_rn(amax, 448.0f);
-  div = amax > 0.0f ? s : 1.0f;
+  div = amax > 0.0f ? make_divider(s) : zero_block_divider();
 }
 
 // Max over the 16 lanes of a half-warp (lanes 0-15 and 16-31 reduce separately).
@@ -96,7 +98,8 @@ __global__ void __launch_bounds__(kThreads) k_quant_rows(const uint16_t *__restr
   for (int u = 0; u < kRowsPerHalfWarp; ++u) {
     const int64_t r = r_first + 16 * u;
     const float amax = halfwarp_max(absmax8(v[u]));
-    float s, div;
+    float s;
+    BlockDivider div;
     block_scale(amax, s, div);
     const uint2 q = codes8(v[u], div);
     if (r < R) {
@@ -149,8 +152,9 @@ __device__ __forceinline__ void read_column_pairs(const uint8_t *tile, uint32_t 
 
 // Codes of the held column pair with divisors div0 (column 2cp) and div1 (column 2cp+1)
 // into the code tile: code tile row = tile column, 128 bytes = the 128 tile rows.
-__device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[32], float div0,
-                                                     float div1, uint8_t *codes) {
+__device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[32],
+                                                     const BlockDivider &div0,
+                                                     const BlockDivider &div1, uint8_t *codes) {
   const int cp = threadIdx.x & 63;
   const int g = threadIdx.x >> 6;
   uint32_t q0[8], q1[8];
@@ -210,7 +214,8 @@ __global__ void __launch_bounds__(kThreads) k_quant_cols(const uint16_t *__restr
     for (int p = 0; p < 8; ++p) {
       const int64_t tok = tok0 + hw + 16 * p;
       const float amax = halfwarp_max(absmax8(t.v[p]));
-      float s, div;
+      float s;
+      BlockDivider div;
       block_scale(amax, s, div);
       *reinterpret_cast<uint2 *>(Xq + tok * C + col0 + l * 8) = codes8(t.v[p], div);
       if (l == 0) S[blockIdx.x * T + tok] = s;
@@ -234,7 +239,8 @@ __global__ void __launch_bounds__(kThreads) k_quant_cols(const uint16_t *__restr
   a0 = fmaxf(fmaxf(part[0][2 * cp], part[1][2 * cp]), fmaxf(part[2][2 * cp], part[3][2 * cp]));
   a1 = fmaxf(fmaxf(part[0][2 * cp + 1], part[1][2 * cp + 1]),
              fmaxf(part[2][2 * cp + 1], part[3][2 * cp + 1]));
-  float s0, d0, s1, d1;
+  float s0, s1;
+  BlockDivider d0, d1;
   block_scale(a0, s0, d0);
   block_scale(a1, s1, d1);
   uint8_t *codes = tile;  // reuse: 128 x kCodePitch bytes fit in the BF16 tile
@@ -273,7 +279,8 @@ __global__ void __launch_bounds__(kThreads) k_quant_weight(const uint16_t *__res
   float amax = warp_max[0];
 #pragma unroll
   for (int i = 1; i < kThreads / 32; ++i) amax = fmaxf(amax, warp_max[i]);
-  float s, div;
+  float s;
+  BlockDivider div;
   block_scale(amax, s, div);
   if (threadIdx.x == 0) S[blockIdx.y * (C / kTile) + blockIdx.x] = s;
 

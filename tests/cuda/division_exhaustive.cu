@@ -1,0 +1,74 @@
+// Test-only kernel: the quantisers' per-block quotient (Markstein's correction with a
+// correctly rounded reciprocal, IEEE division for tiny scales) against CUDA's
+// correctly rounded division, for every pair the quantisers can meet: every positive
+// finite BF16 amax, its scale s = RN(amax / 448), and every BF16 x with |x| <= amax.
+// Counts: [0] E4M3 code mismatches (satfinite RNE of the two quotients), [1] pairs
+// checked, [2] quotient bit mismatches where |x/s| >= 2^-11 (the range in which E4M3
+// rounding decisions are taken), [3] quotient bit mismatches anywhere.
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../fp8_blockwise_scaled_e4m3_b200/csrc/quant_math.cuh"
+
+namespace {
+
+__device__ __forceinline__ unsigned code_of(float q) {
+  return __nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3);
+}
+
+__global__ void k_check(unsigned long long *counts, unsigned int *first_bad) {
+  const uint32_t amax_bits = blockIdx.x + 1;  // 0x0001 .. 0x7F7F
+  const float amax = __uint_as_float(amax_bits << 16);
+  const float s = __fdiv_rn(amax, 448.0f);
+  const puro::BlockDivider d = puro::make_divider(s);
+  unsigned long long bad = 0, n = 0, qbad_big = 0, qbad = 0;
+  for (uint32_t xb = threadIdx.x + blockIdx.y * blockDim.x; xb < 65536u;
+       xb += blockDim.x * gridDim.y) {
+    const float x = __uint_as_float(xb << 16);
+    if (!(fabsf(x) <= amax)) continue;  // also skips NaN patterns
+    ++n;
+    const float fast = puro::block_divide(d, x);
+    const float ref = __fdiv_rn(x, s);
+    if (code_of(fast) != code_of(ref)) {
+      ++bad;
+      atomicCAS(first_bad, 0u, (amax_bits << 16) | xb);
+    }
+    if (__float_as_uint(fast) != __float_as_uint(ref)) {
+      ++qbad;
+      if (fabsf(ref) >= 0x1p-11f) ++qbad_big;
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    n += __shfl_xor_sync(0xffffffffu, n, o);
+    qbad_big += __shfl_xor_sync(0xffffffffu, qbad_big, o);
+    qbad += __shfl_xor_sync(0xffffffffu, qbad, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(counts + 0, bad);
+    atomicAdd(counts + 1, n);
+    atomicAdd(counts + 2, qbad_big);
+    atomicAdd(counts + 3, qbad);
+  }
+}
+
+}  // namespace
+
+extern "C" int run_division_check(unsigned long long *host_counts, unsigned int *host_first_bad) {
+  unsigned long long *counts = nullptr;
+  unsigned int *first = nullptr;
+  if (cudaMalloc(&counts, 4 * sizeof(unsigned long long)) != cudaSuccess) return 1;
+  if (cudaMalloc(&first, sizeof(unsigned int)) != cudaSuccess) return 2;
+  cudaMemset(counts, 0, 4 * sizeof(unsigned long long));
+  cudaMemset(first, 0, sizeof(unsigned int));
+  k_check<<<dim3(0x7F7F, 16), 256>>>(counts, first);
+  if (cudaGetLastError() != cudaSuccess) return 3;
+  if (cudaMemcpy(host_counts, counts, 4 * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return 4;
+  cudaMemcpy(host_first_bad, first, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+  cudaFree(counts);
+  cudaFree(first);
+  return 0;
+}
