@@ -10,7 +10,7 @@
 //     C[m, n] = sum_kb  sA(kb, m) * sB(kb, n) * P_kb[m, n],   P_kb = Aq[m, kb] . Bq[n, kb]
 //
 // One persistent CTA per SM, tiles of 128 x 256, warp-specialised:
-//   warp 0      TMA producer: A and B tiles of one K block per ring stage (4 stages);
+//   warp 0      TMA producer: A and B tiles of one K block per ring stage (3 stages);
 //               for wgrad also the 256 column scales of B per K block (8-stage ring)
 //   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one of two
 //               256-column TMEM buffers, committed to the stage's "empty" barrier and
@@ -19,8 +19,10 @@
 //   warps 4..11 promotion + epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 and
 //               columns 128*((w-4)/4) .. +127, i.e. one output row and 128 columns per
 //               thread; partial * (sA * sB) is added into 128 FP32 registers with
-//               packed FP32x2 FMAs; at the end of the tile the sums are rounded to
-//               BF16 and stored.
+//               packed FP32x2 FMAs; at the end of the tile each warp rounds its 32 x 128
+//               sums to BF16 into a 128B-swizzled staging buffer and hands it to two TMA
+//               tensor stores, so the warps go straight back to the next tile (stores
+//               outside M x N are clipped by the TMA unit).
 // Every mbarrier wait is bounded (wall-clock limit plus an iteration cap). A wait that
 // gives up raises a CTA-wide abort flag and the device status word; all warps then
 // leave their loops, in-flight copies and MMAs are waited for (bounded), and TMEM is
@@ -43,7 +45,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;                  // one scale block of K per stage
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int SC_STAGES = 8;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_FIRST_WARP = 4;               // warps 0-3 form warpgroup 0
@@ -67,7 +69,11 @@ constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
 constexpr int OFF_SC = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_BAR = OFF_SC + SC_STAGES * SC_BYTES;
+constexpr int STG_BOX_BYTES = 32 * 128;   // 32 rows x 64 BF16 columns, 128B-swizzled
+constexpr int STG_WARP_BYTES = 2 * STG_BOX_BYTES;
+constexpr int OFF_STG = OFF_SC + SC_STAGES * SC_BYTES;  // output staging, one per warp
+constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
+static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
 constexpr int N_BARS = 2 * STAGES + 4 + 2 * SC_STAGES + 1;
 constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
 constexpr int SMEM_USED = OFF_MISC + 16;
@@ -109,7 +115,8 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 template <int LAYOUT>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmS, const GemmArgs args) {
+                     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmC,
+                     const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -149,6 +156,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmC);
     if (LAYOUT == PURO_WGRAD) prefetch_tensormap(&tmS);
   }
   if (warp == 1) {
@@ -335,24 +343,36 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (!ok) break;
-      if (m_ok) {
-        uint16_t *crow = args.C + static_cast<int64_t>(m) * args.N;
+      // Stage this warp's 32 rows x 128 columns as BF16 (two 64-column boxes, 16-byte
+      // chunk c of row r at chunk position c ^ (r % 8)) and store them with the TMA unit.
+      const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST_WARP) * STG_WARP_BYTES;
+      if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores left the buffer
+      __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int n = n_base + 8 * j;
-          if (n < args.N) {
-            float v[8];
-            unpack2(acc[4 * j], v[0], v[1]);
-            unpack2(acc[4 * j + 1], v[2], v[3]);
-            unpack2(acc[4 * j + 2], v[4], v[5]);
-            unpack2(acc[4 * j + 3], v[6], v[7]);
-            const uint4 o = make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]),
-                                       bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
-            *reinterpret_cast<uint4 *>(crow + n) = o;
-          }
+      for (int j = 0; j < 16; ++j) {
+        float v[8];
+        unpack2(acc[4 * j], v[0], v[1]);
+        unpack2(acc[4 * j + 1], v[2], v[3]);
+        unpack2(acc[4 * j + 2], v[4], v[5]);
+        unpack2(acc[4 * j + 3], v[6], v[7]);
+        const uint32_t addr = stg + (j >> 3) * STG_BOX_BYTES + lane * 128 + (((j & 7) ^ (lane & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                     "r"(bf16x2_bits(v[0], v[1])), "r"(bf16x2_bits(v[2], v[3])),
+                     "r"(bf16x2_bits(v[4], v[5])), "r"(bf16x2_bits(v[6], v[7]))
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int row0 = mt * BM + quad * 32;
+        if (row0 < args.M) {
+          if (n_base < args.N) tma_store_2d(&tmC, stg, n_base, row0);
+          if (n_base + 64 < args.N) tma_store_2d(&tmC, stg + STG_BOX_BYTES, n_base + 64, row0);
         }
+        bulk_commit_group();
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // stores complete before the CTA exits
     if (!ok) raise_abort(abort, args.status);
   }
 
@@ -417,7 +437,7 @@ int *device_status_ptr() {
 
 template <int LAYOUT>
 int launch_layout(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ts,
-                  const GemmArgs &args, int grid, cudaStream_t stream) {
+                  const CUtensorMap &tc, const GemmArgs &args, int grid, cudaStream_t stream) {
   auto kern = k_gemm_blockwise<LAYOUT>;
   // The register split inside the kernel assumes exactly LAUNCH_REGS per thread at launch;
   // with any other count the promotion warps' setmaxnreg.inc could wait forever.
@@ -433,7 +453,7 @@ int launch_layout(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMa
     std::fprintf(stderr, "puro_fp8: cudaFuncSetAttribute: %s\n", cudaGetErrorString(e));
     return PURO_ERR_CUDA;
   }
-  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, ts, args);
+  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, ts, tc, args);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     std::fprintf(stderr,
@@ -458,10 +478,12 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
   int *status = device_status_ptr();
   if (status == nullptr) return PURO_ERR_CUDA;
 
-  CUtensorMap ta, tb, ts;
+  CUtensorMap ta, tb, ts, tc;
   if (!make_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, BN, BK,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tc, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return PURO_ERR_CUDA;
   if (layout == PURO_WGRAD) {
@@ -491,9 +513,9 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
 
   switch (layout) {
-    case PURO_FPROP: return launch_layout<PURO_FPROP>(ta, tb, ts, args, grid, stream);
-    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(ta, tb, ts, args, grid, stream);
-    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(ta, tb, ts, args, grid, stream);
+    case PURO_FPROP: return launch_layout<PURO_FPROP>(ta, tb, ts, tc, args, grid, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(ta, tb, ts, tc, args, grid, stream);
+    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(ta, tb, ts, tc, args, grid, stream);
     default: return PURO_ERR_LAYOUT;
   }
 }
