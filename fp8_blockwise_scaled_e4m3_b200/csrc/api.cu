@@ -21,8 +21,6 @@ int check_device() {
   return (major == 10 && minor == 0) ? PURO_OK : PURO_ERR_DEVICE;
 }
 
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? PURO_OK : PURO_ERR_LAUNCH; }
-
 }  // namespace
 
 extern "C" {
@@ -35,7 +33,7 @@ int puro_fp8_quantize_1x128(const uint16_t *X, int64_t R, int64_t C, int64_t ldx
   if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(S, 4) || ldx % 8 != 0 || ldq % 16 != 0)
     return PURO_ERR_ALIGN;
   if (int d = check_device()) return d;
-  return from_cuda(puro::launch_quant_rows(X, R, C, ldx, Xq, ldq, S, stream));
+  return puro::launch_quant_rows(X, R, C, ldx, Xq, ldq, S, stream);
 }
 
 int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, int64_t C, int64_t ldx,
@@ -50,7 +48,7 @@ int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, int64_t C, 
     return PURO_ERR_ALIGN;
   if (Xq != nullptr && (!aligned(Xq, 16) || !aligned(S, 4))) return PURO_ERR_ALIGN;
   if (int d = check_device()) return d;
-  return from_cuda(puro::launch_quant_cols(X, T, C, ldx, XqT, ST, Xq, S, stream));
+  return puro::launch_quant_cols(X, T, C, ldx, XqT, ST, Xq, S, stream);
 }
 
 int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
@@ -63,7 +61,7 @@ int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t l
     return PURO_ERR_ALIGN;
   if (WqT != nullptr && !aligned(WqT, 16)) return PURO_ERR_ALIGN;
   if (int d = check_device()) return d;
-  return from_cuda(puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, S, stream));
+  return puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, S, stream);
 }
 
 int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
@@ -86,9 +84,10 @@ int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *B
 }
 
 int puro_fp8_sync_status(puro_stream_t stream) {
-  int status = 0;
-  if (int e = puro::read_and_clear_device_status(stream, &status)) return e;
-  return status != 0 ? PURO_ERR_TIMEOUT : PURO_OK;
+  int gemm = 0, quant = 0;
+  if (int e = puro::read_and_clear_device_status(stream, &gemm)) return e;
+  if (int e = puro::read_and_clear_quant_status(stream, &quant)) return e;
+  return (gemm | quant) != 0 ? PURO_ERR_TIMEOUT : PURO_OK;
 }
 
 const char *puro_strerror(int status) {

@@ -43,9 +43,7 @@ namespace puro {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 128;                  // one scale block of K per stage
-constexpr int STAGES = 3;
 constexpr int SC_STAGES = 8;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_FIRST_WARP = 4;               // warps 0-3 form warpgroup 0
@@ -61,24 +59,40 @@ constexpr int CONSUMER_REGS = 232;
 static_assert(128 * PRODUCER_REGS + 256 * CONSUMER_REGS == THREADS * LAUNCH_REGS,
               "register split must add up to the launch allocation");
 constexpr int A_BYTES = BM * BK;          // 16 KB
-constexpr int B_BYTES = BN * BK;          // 32 KB
-constexpr int SC_BYTES = BN * 4;          // 1 KB
-constexpr uint32_t TMEM_COLS = 2 * BN;    // two FP32 partial buffers
-constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN);
-
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_SC = OFF_B + STAGES * B_BYTES;
 constexpr int STG_BOX_BYTES = 32 * 128;   // 32 rows x 64 BF16 columns, 128B-swizzled
-constexpr int STG_WARP_BYTES = 2 * STG_BOX_BYTES;
-constexpr int OFF_STG = OFF_SC + SC_STAGES * SC_BYTES;  // output staging, one per warp
-constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
-static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
-constexpr int N_BARS = 2 * STAGES + 4 + 2 * SC_STAGES + 1;
-constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
-constexpr int SMEM_USED = OFF_MISC + 16;
-constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack to align the base to 1024 bytes
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+// Tile width TN (256 or 128) sets the rest. TMEM holds 512 FP32 columns, i.e.
+// 512 / TN partial buffers; each promotion warp owns TN / 2 columns of one lane quadrant.
+template <int TN>
+struct Cfg {
+  static constexpr int BN = TN;
+  static constexpr int NBUF = 512 / TN;            // TMEM partial buffers
+  static constexpr int WCOLS = TN / 2;             // columns per promotion warp
+  static constexpr int CHUNKS = WCOLS / 64;        // 64-column TMEM loads per K block
+  static constexpr int STAGES = TN == 256 ? 3 : 5;
+  static constexpr int B_BYTES = TN * BK;
+  static constexpr int SC_BYTES = TN * 4;          // wgrad column scales per K block
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC = idesc_e4m3_f32(BM, TN);
+  static constexpr int STG_WARP_BYTES = (WCOLS / 64) * STG_BOX_BYTES;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;  // output staging, one per warp
+  static constexpr int OFF_SC = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
+  static constexpr int OFF_BAR = OFF_SC + SC_STAGES * SC_BYTES;
+  static constexpr int N_BARS = 2 * STAGES + 2 * NBUF + 2 * SC_STAGES + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
+  static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+// fprop and dgrad carry one scalar scale per 128-column block and keep the wide tile;
+// wgrad scales every column, and its longer promotion gains more from four buffers.
+template <int LAYOUT>
+struct TileFor {
+  static constexpr int TN = LAYOUT == PURO_WGRAD ? 128 : 256;
+};
 
 struct GemmArgs {
   const float *As;
@@ -112,11 +126,16 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-template <int LAYOUT>
+template <int LAYOUT, int TN>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmC,
                      const GemmArgs args) {
+  using C = Cfg<TN>;
+  constexpr int BN = C::BN, NBUF = C::NBUF, STAGES = C::STAGES;
+  constexpr int B_BYTES = C::B_BYTES, SC_BYTES = C::SC_BYTES;
+  constexpr int OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_STG = C::OFF_STG, OFF_SC = C::OFF_SC;
+  constexpr int OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC, N_BARS = C::N_BARS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -125,9 +144,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
-  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + s); };
-  auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 4 + SC_STAGES + s); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + NBUF + b); };
+  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 * NBUF + s); };
+  auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 * NBUF + SC_STAGES + s); };
   const uint32_t drain_bar = bar0 + 8u * (N_BARS - 1);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
   volatile int *abort = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
@@ -141,7 +160,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(tfull_bar(b), 1);
       mbar_init(tempty_bar(b), EPI_WARPS);
     }
@@ -160,7 +179,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (LAYOUT == PURO_WGRAD) prefetch_tensormap(&tmS);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -223,8 +242,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
         for (int kb = 0; kb < kblocks; ++kb, ++use) {
-          const uint32_t b = use & 1u;
-          if (!mbar_wait(tempty_bar(b), ((use >> 1) & 1u) ^ 1u, tmo, abort) ||
+          const uint32_t b = use % NBUF;
+          if (!mbar_wait(tempty_bar(b), ((use / NBUF) & 1u) ^ 1u, tmo, abort) ||
               !mbar_wait(full_bar(s), ph, tmo, abort)) {
             ok = false;
             break;
@@ -235,7 +254,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t b_addr = sbase + OFF_B + s * B_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)
-            mma_e4m3(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), IDESC,
+            mma_e4m3(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), C::IDESC,
                      k > 0 ? 1u : 0u);
           mma_commit(empty_bar(s));
           mma_commit(tfull_bar(b));
@@ -252,6 +271,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(CONSUMER_REGS));
     // ------------------------------------------------------------ promotion + epilogue
+    constexpr int WCOLS = C::WCOLS;
     const int quad = warp & 3;
     const int half = (warp - EPI_FIRST_WARP) >> 2;
     const int row = quad * 32 + lane;
@@ -266,12 +286,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       tile_coords(tile, args, mt, nt);
       const int m = mt * BM + row;
       const bool m_ok = m < args.M;
-      const int nb = nt * 2 + half;  // 128-wide block of N this warp covers
-      const int n_base = nb * 128;
+      const int n_base = nt * BN + half * WCOLS;  // first column of this warp
+      const int nb = n_base / 128;                // its 128-wide scale block of N
       const bool nb_ok = nb < nb_total;
-      uint64_t acc[64];
+      uint64_t acc[WCOLS / 2];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0;
+      for (int i = 0; i < WCOLS / 2; ++i) acc[i] = 0;
 
       auto load_sa = [&](int kb) -> float {
         return m_ok ? __ldg(args.As + static_cast<int64_t>(kb) * args.M + m) : 0.0f;
@@ -290,66 +310,61 @@ __global__ void __launch_bounds__(THREADS, 1)
           sa_next = load_sa(kb + 1);
           sb_next = load_sb(kb + 1);
         }
-        const uint32_t b = use & 1u;
-        if (!mbar_wait(tfull_bar(b), (use >> 1) & 1u, tmo, abort)) {
-          ok = false;
-          break;
-        }
-        const float *sbv = nullptr;
+        const uint32_t b = use % NBUF;
+        // wgrad: the K block's column scales arrive well ahead of its partials, so the
+        // per-column factors t = sA * sB[n] are formed before the TMEM wait and the
+        // partials then need one FMA each, as in fprop and dgrad.
+        uint64_t t2[LAYOUT == PURO_WGRAD ? WCOLS / 2 : 1];
         if (LAYOUT == PURO_WGRAD) {
           if (!mbar_wait(sfull_bar(ss), sph, tmo, abort)) {
             ok = false;
             break;
           }
-          sbv = sc_smem + ss * BN + half * 128;
-        }
-        tc_fence_after_sync();
-        const uint32_t taddr = tmem + lane_base + b * BN + half * 128;
-        const uint64_t s2 = LAYOUT == PURO_WGRAD ? pack2(sa, sa) : pack2(sa * sb, sa * sb);
-        // Two TMEM loads of 64 columns each, one wait per load: the load latency is
-        // paid twice per K block, and 64 partials fit next to the 128 accumulators.
+          const float *sbv = sc_smem + ss * BN + half * WCOLS;
+          const uint64_t sa2 = pack2(sa, sa);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[64];
-          tmem_ld_64cols(taddr + 64 * c, r);
-          tmem_wait_ld();
-          if (c == 1) {  // the buffer is fully in registers: hand it back to the MMA warp
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(b));
+          for (int j = 0; j < WCOLS / 4; ++j) {
+            const float4 sb4 = *reinterpret_cast<const float4 *>(sbv + 4 * j);
+            t2[2 * j] = fmul2(sa2, pack2(sb4.x, sb4.y));
+            t2[2 * j + 1] = fmul2(sa2, pack2(sb4.z, sb4.w));
           }
-          if (LAYOUT == PURO_WGRAD) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float4 sb4 = *reinterpret_cast<const float4 *>(sbv + 64 * c + 4 * j);
-              const uint64_t p0 =
-                  fmul2(pack2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s2);
-              const uint64_t p1 =
-                  fmul2(pack2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s2);
-              acc[32 * c + 2 * j] = ffma2(p0, pack2(sb4.x, sb4.y), acc[32 * c + 2 * j]);
-              acc[32 * c + 2 * j + 1] = ffma2(p1, pack2(sb4.z, sb4.w), acc[32 * c + 2 * j + 1]);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              acc[32 * c + i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
-                                      s2, acc[32 * c + i]);
-          }
-        }
-        if (LAYOUT == PURO_WGRAD) {
           __syncwarp();
           if (lane == 0) mbar_arrive(sempty_bar(ss));
           if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
         }
+        if (!mbar_wait(tfull_bar(b), (use / NBUF) & 1u, tmo, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t taddr = tmem + lane_base + b * BN + half * WCOLS;
+        const uint64_t s2 = pack2(sa * sb, sa * sb);
+        // 64-column TMEM loads, one wait each; the buffer goes back to the MMA warp as
+        // soon as the last one has landed in registers.
+#pragma unroll
+        for (int c = 0; c < C::CHUNKS; ++c) {
+          uint32_t r[64];
+          tmem_ld_64cols(taddr + 64 * c, r);
+          tmem_wait_ld();
+          if (c == C::CHUNKS - 1) {
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(b));
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            acc[32 * c + i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                                    LAYOUT == PURO_WGRAD ? t2[32 * c + i] : s2, acc[32 * c + i]);
+        }
       }
       if (!ok) break;
-      // Stage this warp's 32 rows x 128 columns as BF16 (two 64-column boxes, 16-byte
+      // Stage this warp's 32 rows x WCOLS columns as BF16 (64-column boxes, 16-byte
       // chunk c of row r at chunk position c ^ (r % 8)) and store them with the TMA unit.
-      const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST_WARP) * STG_WARP_BYTES;
+      const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST_WARP) * C::STG_WARP_BYTES;
       if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores left the buffer
       __syncwarp();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < WCOLS / 8; ++j) {
         float v[8];
         unpack2(acc[4 * j], v[0], v[1]);
         unpack2(acc[4 * j + 1], v[2], v[3]);
@@ -366,8 +381,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) {
         const int row0 = mt * BM + quad * 32;
         if (row0 < args.M) {
-          if (n_base < args.N) tma_store_2d(&tmC, stg, n_base, row0);
-          if (n_base + 64 < args.N) tma_store_2d(&tmC, stg + STG_BOX_BYTES, n_base + 64, row0);
+#pragma unroll
+          for (int box = 0; box < WCOLS / 64; ++box)
+            if (n_base + 64 * box < args.N)
+              tma_store_2d(&tmC, stg + box * STG_BOX_BYTES, n_base + 64 * box, row0);
         }
         bulk_commit_group();
       }
@@ -380,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -436,9 +453,31 @@ int *device_status_ptr() {
 }
 
 template <int LAYOUT>
-int launch_layout(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ts,
-                  const CUtensorMap &tc, const GemmArgs &args, int grid, cudaStream_t stream) {
-  auto kern = k_gemm_blockwise<LAYOUT>;
+int launch_layout(const uint8_t *Aq, const uint8_t *Bq, const float *Bs, uint16_t *Cout,
+                  GemmArgs args, int sms, cudaStream_t stream) {
+  constexpr int TN = TileFor<LAYOUT>::TN;
+  constexpr int SMEM_BYTES = Cfg<TN>::SMEM_BYTES;
+  const int64_t M = args.M, N = args.N, K = args.K;
+  CUtensorMap ta, tb, ts, tc;
+  if (!make_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, TN, BK,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return PURO_ERR_CUDA;
+  if (LAYOUT == PURO_WGRAD) {
+    if (!make_map(&ts, Bs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K / 128, N, 1, TN,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return PURO_ERR_CUDA;
+  } else {
+    ts = tb;  // unused
+  }
+  args.num_m = static_cast<int>((M + BM - 1) / BM);
+  args.num_n = static_cast<int>((N + TN - 1) / TN);
+  const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  auto kern = k_gemm_blockwise<LAYOUT, TN>;
   // The register split inside the kernel assumes exactly LAUNCH_REGS per thread at launch;
   // with any other count the promotion warps' setmaxnreg.inc could wait forever.
   cudaFuncAttributes fa{};
@@ -478,22 +517,6 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
   int *status = device_status_ptr();
   if (status == nullptr) return PURO_ERR_CUDA;
 
-  CUtensorMap ta, tb, ts, tc;
-  if (!make_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK,
-                CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, BN, BK,
-                CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tc, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
-                CU_TENSOR_MAP_SWIZZLE_128B))
-    return PURO_ERR_CUDA;
-  if (layout == PURO_WGRAD) {
-    if (!make_map(&ts, Bs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K / 128, N, 1, BN,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
-      return PURO_ERR_CUDA;
-  } else {
-    ts = tb;  // unused
-  }
-
   GemmArgs args;
   args.As = As;
   args.Bs = Bs;
@@ -501,21 +524,17 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
   args.M = static_cast<int>(M);
   args.N = static_cast<int>(N);
   args.K = static_cast<int>(K);
-  args.num_m = static_cast<int>((M + BM - 1) / BM);
-  args.num_n = static_cast<int>((N + BN - 1) / BN);
   args.kblocks = static_cast<int>(K / BK);
   // Walk the smaller operand fastest so that it stays resident in L2 while the larger
   // one streams through once.
   args.m_fastest = M <= N ? 1 : 0;
   args.timeout_ns = wait_timeout_ns();
   args.status = status;
-  const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
 
   switch (layout) {
-    case PURO_FPROP: return launch_layout<PURO_FPROP>(ta, tb, ts, tc, args, grid, stream);
-    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(ta, tb, ts, tc, args, grid, stream);
-    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(ta, tb, ts, tc, args, grid, stream);
+    case PURO_FPROP: return launch_layout<PURO_FPROP>(Aq, Bq, Bs, C, args, sms, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(Aq, Bq, Bs, C, args, sms, stream);
+    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(Aq, Bq, Bs, C, args, sms, stream);
     default: return PURO_ERR_LAYOUT;
   }
 }

@@ -6,49 +6,70 @@
 //   amax = max|x|;  s = amax / 448 (IEEE division);  q = E4M3_rn_satfinite(x / s)
 // and an all-zero block stores s = 0 with signed-zero codes (x / 1 keeps the sign).
 //
-// Kernels:
-//   k_quant_rows      1x128 along the columns of X [R, C]     (fprop A, dgrad A)
-//   k_quant_cols      1x128 along the rows (tokens), output transposed, optionally also
-//                     the row-wise codes from the same read   (wgrad A and B)
-//   k_quant_weight    128x128 blocks, optionally the transposed codes (fprop / dgrad B)
-// All read BF16 with 16-byte vector loads, several in flight per thread, and reduce
-// amax with warp shuffles; the transposed outputs go through a shared-memory tile so
-// every global store is a full 16-byte vector of a contiguous 128-byte row.
+// One persistent kernel serves every quantiser; it walks 128 x 128 BF16 tiles of the
+// input X [R, C] (row stride ldx):
+//   Q_ROWS    1x128 groups along the columns:   Xq [R, C] (row stride ldq), S [C/128][R]
+//   Q_COLS    1x128 groups along the rows, transposed: XqT [C, R], ST [R/128][C]
+//   Q_DUAL    both of the above from one read of X
+//   Q_WEIGHT  one group per 128x128 tile:        Wq [R, C], S [ceil(R/128)][C/128],
+//             and optionally the same codes transposed, WqT [C, R]
+// Tiles arrive by TMA (two 64-column boxes with the 128-byte swizzle) into a 5-stage
+// mbarrier ring of shared memory, so the next tiles are in flight while the current
+// one is computed and nothing in flight occupies registers. Row-wise codes leave with
+// coalesced 8-byte stores; transposed codes are assembled in a swizzled shared tile
+// and written by one TMA tensor store. TMA zero-fills reads past the edge (no effect
+// on amax) and clips writes past it. Every wait is bounded.
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 
+#include "../../include/puro_fp8.h"
+#include "ptx.cuh"
 #include "quant.h"
 #include "quant_math.cuh"
 
 namespace puro {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRowsPerHalfWarp = 4;            // k_quant_rows: rows per 16-lane group
-constexpr int kRowsPerCta = 16 * kRowsPerHalfWarp;
-constexpr int kTile = 128;                      // transposed kernels: 128 x 128 tile
-constexpr int kPitch = kTile * 2 + 16;          // BF16 tile row pitch in bytes (272)
-constexpr int kCodePitch = kTile + 16;          // code tile row pitch in bytes (144)
+enum QMode { Q_ROWS = 1, Q_COLS = 2, Q_DUAL = 3, Q_WEIGHT = 4 };
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+constexpr int kTile = 128;
+// Threads per CTA: many warps hide the shared-memory and conversion latencies of the
+// per-tile work; the register budget (64K per SM) sets the count per mode.
+template <int MODE>
+struct Threads {
+  static constexpr int value = MODE == 1 ? 1024 : 512;
+};
+constexpr int kStages = 5;
+constexpr int kBoxBytes = kTile * 128;         // 128 rows x 64 BF16 (128 bytes), swizzled
+constexpr int kStageBytes = 2 * kBoxBytes;     // one 128 x 128 BF16 tile
+constexpr int kOffCodes = kStages * kStageBytes;
+constexpr int kOffPart = kOffCodes + kTile * kTile;  // 128 x 128 code tile, swizzled
+constexpr int kOffWarpMax = kOffPart + 16 * kTile * 4;   // up to 16 token groups
+constexpr int kOffBar = kOffWarpMax + 32 * 4;
+constexpr int kOffMisc = kOffBar + 8 * kStages;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-__device__ __forceinline__ uint4 load_stream(const uint16_t *p) {
-  return __ldcs(reinterpret_cast<const uint4 *>(p));
-}
+struct QArgs {
+  int64_t R, C;
+  uint8_t *q;        // row-wise codes (Q_ROWS, Q_DUAL) or Wq (Q_WEIGHT)
+  int64_t ldq;
+  float *s;          // S of the row-wise groups, or of the weight blocks
+  float *st;         // ST of the transposed groups (Q_COLS, Q_DUAL)
+  int write_t;       // Q_WEIGHT: also write WqT through the transposed store
+  int tiles_r, tiles_c;
+  unsigned long long timeout_ns;
+  int *status;
+};
 
-// Four quotients -> four E4M3 codes, first argument in the lowest byte.
-__device__ __forceinline__ uint32_t codes4(float a, float b, float c, float d,
-                                           const BlockDivider &div) {
-  const uint32_t lo = __nv_cvt_float2_to_fp8x2(
-      make_float2(block_divide(div, a), block_divide(div, b)), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t hi = __nv_cvt_float2_to_fp8x2(
-      make_float2(block_divide(div, c), block_divide(div, d)), __NV_SATFINITE, __NV_E4M3);
-  return lo | (hi << 16);
-}
+__device__ int g_quant_status;  // non-zero: a bounded wait gave up since the last read
+
 
 __device__ __forceinline__ float absmax8(const uint4 &v) {
   float m = fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x)));
@@ -59,8 +80,7 @@ __device__ __forceinline__ float absmax8(const uint4 &v) {
 }
 
 __device__ __forceinline__ uint2 codes8(const uint4 &v, const BlockDivider &div) {
-  return make_uint2(codes4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), div),
-                    codes4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w), div));
+  return make_uint2(block_codes4(v.x, v.y, div), block_codes4(v.z, v.w, div));
 }
 
 // Scale of a block with absolute maximum `amax`, and the divider for its codes.
@@ -69,262 +89,372 @@ __device__ __forceinline__ void block_scale(float amax, float &s, BlockDivider &
   div = amax > 0.0f ? make_divider(s) : zero_block_divider();
 }
 
-// Max over the 16 lanes of a half-warp (lanes 0-15 and 16-31 reduce separately).
-__device__ __forceinline__ float halfwarp_max(float v) {
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+// Max over each group of 8 consecutive lanes.
+__device__ __forceinline__ float lane8_max(float v) {
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
   return v;
 }
 
-// ------------------------------------------------------------------ 1x128 along columns
-// CTA = 64 rows x one 128-column block. Half-warp h handles rows base + h + 16u, lane l
-// of the half-warp columns 8l .. 8l+7. All four loads are issued before any arithmetic.
-__global__ void __launch_bounds__(kThreads) k_quant_rows(const uint16_t *__restrict__ X, int64_t R,
-                                                         int64_t ldx, uint8_t *__restrict__ Xq,
-                                                         int64_t ldq, float *__restrict__ S) {
-  const int hw = threadIdx.x >> 4;
-  const int l = threadIdx.x & 15;
-  const int64_t j = blockIdx.y;
-  const int64_t r_first = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + hw;
-  uint4 v[kRowsPerHalfWarp];
-#pragma unroll
-  for (int u = 0; u < kRowsPerHalfWarp; ++u) {
-    const int64_t r = r_first + 16 * u;
-    v[u] = r < R ? load_stream(X + r * ldx + j * kTile + l * 8) : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int u = 0; u < kRowsPerHalfWarp; ++u) {
-    const int64_t r = r_first + 16 * u;
-    const float amax = halfwarp_max(absmax8(v[u]));
-    float s;
-    BlockDivider div;
-    block_scale(amax, s, div);
-    const uint2 q = codes8(v[u], div);
-    if (r < R) {
-      *reinterpret_cast<uint2 *>(Xq + r * ldq + j * kTile + l * 8) = q;
-      if (l == 0) S[j * R + r] = s;
-    }
-  }
+// The tile in a stage: box b = columns 64b .. 64b+63; row r of a box is 128 bytes with
+// its 16-byte chunk k stored at chunk position k ^ (r % 8).
+// Row phase: 8 lanes per tile row; lane j of the group holds columns 8j .. 8j+7 (box 0)
+// and 64+8j .. 64+8j+7 (box 1), so each load of the group covers one whole swizzled row.
+__device__ __forceinline__ uint4 row_chunk(const uint8_t *stage, int r, int box, int j) {
+  return *reinterpret_cast<const uint4 *>(stage + box * kBoxBytes + r * 128 +
+                                          ((j ^ (r & 7)) << 4));
 }
-
-// ------------------------------------------------------------------ shared tile helpers
-// The transposed kernels stage a 128-row x 128-column BF16 tile (rows = tokens for the
-// activation quantiser, output features for the weight quantiser) in shared memory.
-// Loading: half-warp h, lane l reads row h + 16p (p = 0..7), columns 8l .. 8l+7.
-
-struct TileLoad {
-  uint4 v[8];
-};
-
-__device__ __forceinline__ void load_tile(TileLoad &t, const uint16_t *__restrict__ X,
-                                          int64_t row0, int64_t rows_valid, int64_t col0,
-                                          int64_t cols, int64_t ldx) {
-  const int hw = threadIdx.x >> 4;
-  const int l = threadIdx.x & 15;
-  const int64_t col = col0 + l * 8;
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int64_t r = hw + 16 * p;
-    t.v[p] = (r < rows_valid && col < cols) ? load_stream(X + (row0 + r) * ldx + col)
-                                            : make_uint4(0, 0, 0, 0);
-  }
-}
-
-__device__ __forceinline__ void store_tile_smem(const TileLoad &t, uint8_t *tile) {
-  const int hw = threadIdx.x >> 4;
-  const int l = threadIdx.x & 15;
-#pragma unroll
-  for (int p = 0; p < 8; ++p)
-    *reinterpret_cast<uint4 *>(tile + (hw + 16 * p) * kPitch + l * 16) = t.v[p];
-}
-
-// Column phase. Thread (cp = tid % 64, g = tid / 64) holds columns 2cp, 2cp+1 of tile
-// rows 32g .. 32g+31 as BF16 pairs.
-__device__ __forceinline__ void read_column_pairs(const uint8_t *tile, uint32_t (&w)[32]) {
+// Column phase: thread (cp, g) holds columns 2cp, 2cp+1 of tile rows TG*g .. TG*g+TG-1
+// as BF16 pairs (TG = 8192 / NT); a warp reads one 128-byte row of one box per load,
+// conflict free.
+template <int TG>
+__device__ __forceinline__ void read_column_pairs(const uint8_t *stage, uint32_t (&w)[TG]) {
   const int cp = threadIdx.x & 63;
   const int g = threadIdx.x >> 6;
+  const uint8_t *box = stage + (cp >> 5) * kBoxBytes;
+  const int chunk = (cp & 31) >> 2;
+  const int byte = (cp & 3) * 4;
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
-    w[i] = *reinterpret_cast<const uint32_t *>(tile + (32 * g + i) * kPitch + cp * 4);
+  for (int i = 0; i < TG; ++i) {
+    const int t = TG * g + i;
+    w[i] = *reinterpret_cast<const uint32_t *>(box + t * 128 + ((chunk ^ (t & 7)) << 4) + byte);
+  }
 }
 
-// Codes of the held column pair with divisors div0 (column 2cp) and div1 (column 2cp+1)
-// into the code tile: code tile row = tile column, 128 bytes = the 128 tile rows.
-__device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[32],
+// Codes of the held column pair into the code tile: code-tile row = tile column (128
+// bytes = the 128 tile rows), 16-byte chunk k at position k ^ (row % 8). TG = 16 gives
+// one chunk per column, TG = 32 two.
+template <int TG>
+__device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[TG],
                                                      const BlockDivider &div0,
                                                      const BlockDivider &div1, uint8_t *codes) {
+  static_assert(TG == 16 || TG == 32, "16 or 32 tile rows per thread");
   const int cp = threadIdx.x & 63;
   const int g = threadIdx.x >> 6;
-  uint32_t q0[8], q1[8];
+  uint32_t q0[TG / 4], q1[TG / 4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    q0[i] = codes4(bf16_lo(w[4 * i]), bf16_lo(w[4 * i + 1]), bf16_lo(w[4 * i + 2]),
-                   bf16_lo(w[4 * i + 3]), div0);
-    q1[i] = codes4(bf16_hi(w[4 * i]), bf16_hi(w[4 * i + 1]), bf16_hi(w[4 * i + 2]),
-                   bf16_hi(w[4 * i + 3]), div1);
+  for (int i = 0; i < TG / 4; ++i) {
+    // column 2cp is the low half of each word, column 2cp+1 the high half
+    q0[i] = block_codes4(__byte_perm(w[4 * i], w[4 * i + 1], 0x5410),
+                         __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x5410), div0);
+    q1[i] = block_codes4(__byte_perm(w[4 * i], w[4 * i + 1], 0x7632),
+                         __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x7632), div1);
   }
-  uint8_t *row0 = codes + (2 * cp) * kCodePitch + 32 * g;
-  uint8_t *row1 = row0 + kCodePitch;
-  reinterpret_cast<uint4 *>(row0)[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
-  reinterpret_cast<uint4 *>(row0)[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
-  reinterpret_cast<uint4 *>(row1)[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
-  reinterpret_cast<uint4 *>(row1)[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+  const int r0 = 2 * cp, r1 = 2 * cp + 1;
+  uint8_t *row0 = codes + r0 * 128;
+  uint8_t *row1 = codes + r1 * 128;
+#pragma unroll
+  for (int k = 0; k < TG / 16; ++k) {
+    const int chunk = (TG / 16) * g + k;
+    *reinterpret_cast<uint4 *>(row0 + ((chunk ^ (r0 & 7)) << 4)) =
+        make_uint4(q0[4 * k], q0[4 * k + 1], q0[4 * k + 2], q0[4 * k + 3]);
+    *reinterpret_cast<uint4 *>(row1 + ((chunk ^ (r1 & 7)) << 4)) =
+        make_uint4(q1[4 * k], q1[4 * k + 1], q1[4 * k + 2], q1[4 * k + 3]);
+  }
 }
 
-// Code tile -> global: row c of the tile goes to out[(col0 + c) * ld_out + row0 ...],
-// 16 bytes per thread, 8 threads per 128-byte row. Only columns < cols and 16-row
-// chunks < rows_valid are written.
-__device__ __forceinline__ void store_code_tile(const uint8_t *codes, uint8_t *__restrict__ out,
-                                                int64_t ld_out, int64_t row0, int64_t rows_valid,
-                                                int64_t col0, int64_t cols) {
-  const int chunk = threadIdx.x & 7;
+template <int MODE>
+__global__ void __launch_bounds__(Threads<MODE>::value, 1)
+    k_quant_tiles(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
+                  const QArgs args) {
+  constexpr bool kRows = MODE == Q_ROWS || MODE == Q_DUAL;
+  constexpr bool kCols = MODE == Q_COLS || MODE == Q_DUAL;
+  constexpr bool kWeight = MODE == Q_WEIGHT;
+  constexpr int NT = Threads<MODE>::value;
+  constexpr int NG = NT / 64;           // token groups of the column phase
+  constexpr int TG = kTile / NG;        // tile rows per thread in the column phase
+  constexpr int RSTEP = NT / 8;         // tile rows per pass of the row phase
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint8_t *codes = smem + kOffCodes;
+  float (*part)[kTile] = reinterpret_cast<float (*)[kTile]>(smem + kOffPart);
+  float *warp_max = reinterpret_cast<float *>(smem + kOffWarpMax);
+  const uint32_t bar0 = sbase + kOffBar;
+  volatile int *fail = reinterpret_cast<volatile int *>(smem + kOffMisc);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int tiles = args.tiles_r * args.tiles_c;
+  const bool write_t = kCols || (kWeight && args.write_t);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
+    *fail = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmX);
+    if (write_t) prefetch_tensormap(&tmT);
+  }
+  __syncthreads();
+
+  // Tile i of this CTA is global tile blockIdx.x + i * gridDim.x; stage i % kStages.
+  auto issue = [&](int i) {
+    const int tile = blockIdx.x + i * gridDim.x;
+    if (tile >= tiles) return;
+    const int tr = tile / args.tiles_c, tc = tile % args.tiles_c;
+    const int s = i % kStages;
+    const uint32_t bar = bar0 + 8 * s;
+    const uint32_t dst = sbase + s * kStageBytes;
+    mbar_arrive_expect_tx(bar, kStageBytes);
+    tma_load_2d(dst, &tmX, bar, tc * kTile, tr * kTile);
+    tma_load_2d(dst + kBoxBytes, &tmX, bar, tc * kTile + 64, tr * kTile);
+  };
+  if (tid == 0)
+    for (int i = 0; i < kStages; ++i) issue(i);
+
+  const int rg = tid >> 3, j8 = tid & 7;   // row group and its lane in the row phase
+  const int cp = tid & 63, g = tid >> 6;
+  int i = 0;
+  for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
+    const int s = i % kStages;
+    const int tr = tile / args.tiles_c, tc = tile % args.tiles_c;
+    const int64_t r0 = static_cast<int64_t>(tr) * kTile;
+    const int64_t c0 = static_cast<int64_t>(tc) * kTile;
+    const uint8_t *stage = smem + s * kStageBytes;
+    const bool waited = mbar_wait(bar0 + 8 * s, (i / kStages) & 1, args.timeout_ns, fail);
+    if (__syncthreads_or(!waited)) {
+      if (tid == 0) {
+        *fail = 1;
+        atomicOr(args.status, 1);
+      }
+      break;
+    }
+    if (tid == 0 && write_t) bulk_wait_group_read<0>();  // the code tile is free again
+
+    // ---------------------------------------------------------------- weight block
+    BlockDivider wdiv = zero_block_divider();
+    if (kWeight) {
+      float m = 0.0f;
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int c = (threadIdx.x >> 3) + 32 * p;
-    if (col0 + c < cols && 16 * chunk < rows_valid) {
-      const uint4 q = *reinterpret_cast<const uint4 *>(codes + c * kCodePitch + 16 * chunk);
-      *reinterpret_cast<uint4 *>(out + (col0 + c) * ld_out + row0 + 16 * chunk) = q;
+      for (int p = 0; p < kTile / RSTEP; ++p)
+        m = fmaxf(m, fmaxf(absmax8(row_chunk(stage, rg + RSTEP * p, 0, j8)),
+                           absmax8(row_chunk(stage, rg + RSTEP * p, 1, j8))));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) warp_max[warp] = m;
+      __syncthreads();
+      float amax = warp_max[0];
+#pragma unroll
+      for (int k = 1; k < NT / 32; ++k) amax = fmaxf(amax, warp_max[k]);
+      float sblk;
+      block_scale(amax, sblk, wdiv);
+      if (tid == 0) args.s[static_cast<int64_t>(tr) * args.tiles_c + tc] = sblk;
+    }
+
+    // ---------------------------------------------------------------- row-wise codes
+    if (kRows || kWeight) {
+#pragma unroll
+      for (int p = 0; p < kTile / RSTEP; ++p) {
+        const int r = rg + RSTEP * p;
+        const uint4 v0 = row_chunk(stage, r, 0, j8);
+        const uint4 v1 = row_chunk(stage, r, 1, j8);
+        BlockDivider div = wdiv;
+        float srow = 0.0f;
+        if (kRows) block_scale(lane8_max(fmaxf(absmax8(v0), absmax8(v1))), srow, div);
+        const uint2 q0 = codes8(v0, div);
+        const uint2 q1 = codes8(v1, div);
+        const int64_t row = r0 + r;
+        if (row < args.R) {  // C is a multiple of 128 in these modes
+          uint8_t *qrow = args.q + row * args.ldq + c0 + 8 * j8;
+          *reinterpret_cast<uint2 *>(qrow) = q0;
+          *reinterpret_cast<uint2 *>(qrow + 64) = q1;
+          if (kRows && j8 == 0) args.s[(c0 / kTile) * args.R + row] = srow;
+        }
+      }
+    }
+
+    // ---------------------------------------------------------------- transposed codes
+    if constexpr (kCols || kWeight) if (write_t) {
+      uint32_t w[TG];
+      read_column_pairs<TG>(stage, w);
+      BlockDivider d0 = wdiv, d1 = wdiv;
+      if (kCols) {
+        float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+        for (int k = 0; k < TG; ++k) {
+          a0 = fmaxf(a0, fabsf(bf16_lo(w[k])));
+          a1 = fmaxf(a1, fabsf(bf16_hi(w[k])));
+        }
+        part[g][2 * cp] = a0;
+        part[g][2 * cp + 1] = a1;
+      }
+      __syncthreads();  // column partials ready; the code tile is free (thread 0 waited)
+      if (kCols) {
+        float a0 = part[0][2 * cp], a1 = part[0][2 * cp + 1];
+#pragma unroll
+        for (int k = 1; k < NG; ++k) {
+          a0 = fmaxf(a0, part[k][2 * cp]);
+          a1 = fmaxf(a1, part[k][2 * cp + 1]);
+        }
+        float s0, s1;
+        block_scale(a0, s0, d0);
+        block_scale(a1, s1, d1);
+        if (g == 0) {
+          const int64_t c = c0 + 2 * cp;
+          float *strow = args.st + static_cast<int64_t>(tr) * args.C;
+          if (c < args.C) strow[c] = s0;
+          if (c + 1 < args.C) strow[c + 1] = s1;
+        }
+      }
+      column_codes_to_smem<TG>(w, d0, d1, codes);
+      fence_proxy_async_smem();
+    }
+    __syncthreads();  // the stage and (if any) the code tile are complete
+    if (tid == 0) {
+      if (write_t) {
+        tma_store_2d(&tmT, sbase + kOffCodes, static_cast<int32_t>(r0), static_cast<int32_t>(c0));
+        bulk_commit_group();
+      }
+      issue(i + kStages);  // refill the stage just consumed
+    }
+  }
+
+  if (tid == 0) {
+    if (write_t) bulk_wait_group_all();
+    if (*fail) {
+      // Let every load still in flight land before the CTA exits (bounded).
+      for (int k = 0; k < kStages; ++k) {
+        const int ii = i + k;
+        if (blockIdx.x + ii * gridDim.x < tiles)
+          mbar_wait(bar0 + 8 * (ii % kStages), (ii / kStages) & 1, args.timeout_ns, nullptr);
+      }
     }
   }
 }
 
-// ------------------------------------------------------------------ 1x128 along tokens
-// CTA = 128 tokens x 128 columns. Optional dual output: the row-wise 1x128 codes of the
-// same rows, computed from the registers of the load (16 lanes hold one row block).
-__global__ void __launch_bounds__(kThreads) k_quant_cols(const uint16_t *__restrict__ X, int64_t T,
-                                                         int64_t C, int64_t ldx,
-                                                         uint8_t *__restrict__ XqT,
-                                                         float *__restrict__ ST,
-                                                         uint8_t *__restrict__ Xq,
-                                                         float *__restrict__ S) {
-  __shared__ __align__(16) uint8_t tile[kTile * kPitch];
-  __shared__ float part[4][kTile];
-  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kTile;
-  const int64_t tok0 = static_cast<int64_t>(blockIdx.y) * kTile;
+// ------------------------------------------------------------------ host side
 
-  TileLoad t;
-  load_tile(t, X, tok0, kTile, col0, C, ldx);
-  store_tile_smem(t, tile);
-  if (Xq != nullptr) {  // uniform over the grid
-    const int hw = threadIdx.x >> 4;
-    const int l = threadIdx.x & 15;
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      const int64_t tok = tok0 + hw + 16 * p;
-      const float amax = halfwarp_max(absmax8(t.v[p]));
-      float s;
-      BlockDivider div;
-      block_scale(amax, s, div);
-      *reinterpret_cast<uint2 *>(Xq + tok * C + col0 + l * 8) = codes8(t.v[p], div);
-      if (l == 0) S[blockIdx.x * T + tok] = s;
-    }
-  }
-  __syncthreads();
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-  uint32_t w[32];
-  read_column_pairs(tile, w);
-  float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    a0 = fmaxf(a0, fabsf(bf16_lo(w[i])));
-    a1 = fmaxf(a1, fabsf(bf16_hi(w[i])));
-  }
-  const int cp = threadIdx.x & 63;
-  const int g = threadIdx.x >> 6;
-  part[g][2 * cp] = a0;
-  part[g][2 * cp + 1] = a1;
-  __syncthreads();  // every thread has read its tile slice: the tile may be reused
-  a0 = fmaxf(fmaxf(part[0][2 * cp], part[1][2 * cp]), fmaxf(part[2][2 * cp], part[3][2 * cp]));
-  a1 = fmaxf(fmaxf(part[0][2 * cp + 1], part[1][2 * cp + 1]),
-             fmaxf(part[2][2 * cp + 1], part[3][2 * cp + 1]));
-  float s0, s1;
-  BlockDivider d0, d1;
-  block_scale(a0, s0, d0);
-  block_scale(a1, s1, d1);
-  uint8_t *codes = tile;  // reuse: 128 x kCodePitch bytes fit in the BF16 tile
-  column_codes_to_smem(w, d0, d1, codes);
-  if (g == 0) {
-    const int64_t c = col0 + 2 * cp;
-    if (c < C) ST[blockIdx.y * C + c] = s0;
-    if (c + 1 < C) ST[blockIdx.y * C + c + 1] = s1;
-  }
-  __syncthreads();
-  store_code_tile(codes, XqT, T, tok0, kTile, col0, C);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
 }
 
-// ------------------------------------------------------------------ 128x128 weight blocks
-__global__ void __launch_bounds__(kThreads) k_quant_weight(const uint16_t *__restrict__ W,
-                                                           int64_t R, int64_t C, int64_t ldw,
-                                                           uint8_t *__restrict__ Wq,
-                                                           uint8_t *__restrict__ WqT,
-                                                           float *__restrict__ S) {
-  __shared__ __align__(16) uint8_t tile[kTile * kPitch];
-  __shared__ float warp_max[kThreads / 32];
-  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kTile;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kTile;
-  const int64_t rows_valid = R - row0 < kTile ? R - row0 : kTile;
+// [rows, cols] with row stride `ld` elements of `elem` bytes, box [box_rows, box_cols],
+// 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem,
+              uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {ld * static_cast<uint64_t>(elem)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
-  TileLoad t;
-  load_tile(t, W, row0, rows_valid, col0, C, ldw);
-  float m = 0.0f;
-#pragma unroll
-  for (int p = 0; p < 8; ++p) m = fmaxf(m, absmax8(t.v[p]));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
-  if (WqT != nullptr) store_tile_smem(t, tile);
-  __syncthreads();
-  float amax = warp_max[0];
-#pragma unroll
-  for (int i = 1; i < kThreads / 32; ++i) amax = fmaxf(amax, warp_max[i]);
-  float s;
-  BlockDivider div;
-  block_scale(amax, s, div);
-  if (threadIdx.x == 0) S[blockIdx.y * (C / kTile) + blockIdx.x] = s;
+unsigned long long wait_timeout_ns() {
+  static unsigned long long ns = [] {
+    const char *e = std::getenv("PURO_WAIT_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 2000;
+    if (ms < 1) ms = 1;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return ns;
+}
 
-  const int hw = threadIdx.x >> 4;
-  const int l = threadIdx.x & 15;
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int64_t r = hw + 16 * p;
-    if (r < rows_valid)
-      *reinterpret_cast<uint2 *>(Wq + (row0 + r) * C + col0 + l * 8) = codes8(t.v[p], div);
+template <int MODE>
+int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *qt, QArgs args,
+                 cudaStream_t stream) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  if (cudaGetSymbolAddress(reinterpret_cast<void **>(&args.status), g_quant_status) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  CUtensorMap tmX, tmT;
+  if (!make_map(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, C, ldx, kTile, 64))
+    return PURO_ERR_CUDA;
+  if (qt != nullptr) {
+    // the transposed codes [C, R]: one box of 128 rows (tile columns) x 128 bytes
+    if (!make_map(&tmT, qt, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, C, R, R, kTile, kTile))
+      return PURO_ERR_CUDA;
+  } else {
+    tmT = tmX;  // unused
   }
-  if (WqT == nullptr) return;  // uniform over the grid
-
-  uint32_t w[32];
-  read_column_pairs(tile, w);
-  __syncthreads();
-  column_codes_to_smem(w, div, div, tile);
-  __syncthreads();
-  store_code_tile(tile, WqT, R, row0, rows_valid, col0, C);
+  args.R = R;
+  args.C = C;
+  args.tiles_r = static_cast<int>((R + kTile - 1) / kTile);
+  args.tiles_c = static_cast<int>((C + kTile - 1) / kTile);
+  args.timeout_ns = wait_timeout_ns();
+  const int64_t tiles = static_cast<int64_t>(args.tiles_r) * args.tiles_c;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  auto kern = k_quant_tiles<MODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+      cudaSuccess)
+    return PURO_ERR_CUDA;
+  kern<<<grid, Threads<MODE>::value, kSmemBytes, stream>>>(tmX, tmT, args);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "puro_fp8: quantiser launch: %s\n", cudaGetErrorString(e));
+    return PURO_ERR_LAUNCH;
+  }
+  return PURO_OK;
 }
 
 }  // namespace
 
 // ------------------------------------------------------------------ launchers
-cudaError_t launch_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
-                              int64_t ldq, float *S, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>((R + kRowsPerCta - 1) / kRowsPerCta),
-            static_cast<unsigned>(C / kTile));
-  k_quant_rows<<<grid, kThreads, 0, stream>>>(X, R, ldx, Xq, ldq, S);
-  return cudaGetLastError();
+int launch_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                      int64_t ldq, float *S, cudaStream_t stream) {
+  QArgs a{};
+  a.q = Xq;
+  a.ldq = ldq;
+  a.s = S;
+  return launch_tiles<Q_ROWS>(X, R, C, ldx, nullptr, a, stream);
 }
 
-cudaError_t launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint8_t *XqT,
-                              float *ST, uint8_t *Xq, float *S, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>((C + kTile - 1) / kTile), static_cast<unsigned>(T / kTile));
-  k_quant_cols<<<grid, kThreads, 0, stream>>>(X, T, C, ldx, XqT, ST, Xq, S);
-  return cudaGetLastError();
+int launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint8_t *XqT,
+                      float *ST, uint8_t *Xq, float *S, cudaStream_t stream) {
+  QArgs a{};
+  a.st = ST;
+  if (Xq != nullptr) {
+    a.q = Xq;
+    a.ldq = C;
+    a.s = S;
+    return launch_tiles<Q_DUAL>(X, T, C, ldx, XqT, a, stream);
+  }
+  return launch_tiles<Q_COLS>(X, T, C, ldx, XqT, a, stream);
 }
 
-cudaError_t launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
-                                uint8_t *WqT, float *S, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>(C / kTile), static_cast<unsigned>((R + kTile - 1) / kTile));
-  k_quant_weight<<<grid, kThreads, 0, stream>>>(W, R, C, ldw, Wq, WqT, S);
-  return cudaGetLastError();
+int launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
+                        uint8_t *WqT, float *S, cudaStream_t stream) {
+  QArgs a{};
+  a.q = Wq;
+  a.ldq = C;
+  a.s = S;
+  a.write_t = WqT != nullptr;
+  return launch_tiles<Q_WEIGHT>(W, R, C, ldw, WqT, a, stream);
+}
+
+int read_and_clear_quant_status(cudaStream_t stream, int *status_out) {
+  int host = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&host, g_quant_status, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                stream) != cudaSuccess ||
+      cudaMemcpyToSymbolAsync(g_quant_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                              stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  *status_out = host;
+  return PURO_OK;
 }
 
 }  // namespace puro

@@ -8,12 +8,16 @@
 
 namespace puro {
 
-cudaError_t launch_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
-                              int64_t ldq, float *S, cudaStream_t stream);
-cudaError_t launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint8_t *XqT,
-                              float *ST, uint8_t *Xq, float *S, cudaStream_t stream);
-cudaError_t launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
-                                uint8_t *WqT, float *S, cudaStream_t stream);
+// Quantiser launchers; return 0 or a negative puro_status.
+int launch_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                      int64_t ldq, float *S, cudaStream_t stream);
+int launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint8_t *XqT,
+                      float *ST, uint8_t *Xq, float *S, cudaStream_t stream);
+int launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
+                        uint8_t *WqT, float *S, cudaStream_t stream);
+
+// Reads and clears the quantisers' device status word (after a stream sync).
+int read_and_clear_quant_status(cudaStream_t stream, int *status_out);
 
 // Returns 0 on success, a negative puro_status on failure.
 int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs,

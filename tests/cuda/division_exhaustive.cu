@@ -2,9 +2,10 @@
 // correctly rounded reciprocal, IEEE division for tiny scales) against CUDA's
 // correctly rounded division, for every pair the quantisers can meet: every positive
 // finite BF16 amax, its scale s = RN(amax / 448), and every BF16 x with |x| <= amax.
-// Counts: [0] E4M3 code mismatches (satfinite RNE of the two quotients), [1] pairs
-// checked, [2] quotient bit mismatches where |x/s| >= 2^-11 (the range in which E4M3
-// rounding decisions are taken), [3] quotient bit mismatches anywhere.
+// Counts: [0] E4M3 code mismatches (satfinite RNE of the two quotients, and the codes of
+// the packed four-value helper the kernels use), [1] pairs checked, [2] quotient bit
+// mismatches where |x/s| >= 2^-11 (the range in which E4M3 rounding decisions are
+// taken), [3] quotient bit mismatches anywhere.
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -30,7 +31,12 @@ __global__ void k_check(unsigned long long *counts, unsigned int *first_bad) {
     ++n;
     const float fast = puro::block_divide(d, x);
     const float ref = __fdiv_rn(x, s);
-    if (code_of(fast) != code_of(ref)) {
+    const uint32_t w = xb | (xb << 16);  // x in both halves of a BF16 pair
+    const uint32_t packed = puro::block_codes4(w, w, d);
+    const unsigned want = code_of(ref);
+    const bool packed_ok = (packed & 0xFFu) == want && ((packed >> 8) & 0xFFu) == want &&
+                           ((packed >> 16) & 0xFFu) == want && (packed >> 24) == want;
+    if (code_of(fast) != want || !packed_ok) {
       ++bad;
       atomicCAS(first_bad, 0u, (amax_bits << 16) | xb);
     }
