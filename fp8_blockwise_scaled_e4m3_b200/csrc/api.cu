@@ -77,7 +77,7 @@ int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *B
   // 32-bit tensor-map coordinates and kernel indices
   if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
   if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16) || !aligned(As, 4) ||
-      !aligned(Bs, layout == PURO_WGRAD ? 16 : 4))
+      !aligned(Bs, 4))
     return PURO_ERR_ALIGN;
   if (int d = check_device()) return d;
   return puro::launch_gemm_blockwise(Aq, As, Bq, Bs, C, M, N, K, layout, stream);

@@ -9,18 +9,22 @@
 // running FP32 sum with its two scales:
 //     C[m, n] = sum_kb  sA(kb, m) * sB(kb, n) * P_kb[m, n],   P_kb = Aq[m, kb] . Bq[n, kb]
 //
-// One persistent CTA per SM, tiles of 128 x 256, warp-specialised:
-//   warp 0      TMA producer: A and B tiles of one K block per ring stage (3 stages);
-//               for wgrad also the 256 column scales of B per K block (8-stage ring)
-//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one of two
-//               256-column TMEM buffers, committed to the stage's "empty" barrier and
+// One persistent CTA per SM, tiles of 128 x TN (TN = 256 for fprop/dgrad, 128 for
+// wgrad), warp-specialised:
+//   warp 0      TMA producer: A and B tiles of one K block per ring stage
+//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one of the
+//               512 / TN TMEM buffers, committed to the stage's "empty" barrier and
 //               the buffer's "full" barrier; also owns the TMEM allocation
-//   warps 2-3   idle (they complete warpgroup 0, which hands its registers over)
+//   warp 2      scale loader: for every K block, the tile's 128 row scales of A and its
+//               column scales of B (one per 128-column block, or one per column for
+//               wgrad) are copied with cp.async into an 8-slot shared-memory ring, so
+//               the promotion never waits on a global load
+//   warp 3      idle (it completes warpgroup 0, which hands its registers over)
 //   warps 4..11 promotion + epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 and
-//               columns 128*((w-4)/4) .. +127, i.e. one output row and 128 columns per
-//               thread; partial * (sA * sB) is added into 128 FP32 registers with
-//               packed FP32x2 FMAs; at the end of the tile each warp rounds its 32 x 128
-//               sums to BF16 into a 128B-swizzled staging buffer and hands it to two TMA
+//               columns (TN/2)*((w-4)/4) .. +TN/2-1, i.e. one output row and TN/2
+//               columns per thread; partial * (sA * sB) is added into FP32 registers
+//               with packed FP32x2 FMAs; at the end of the tile each warp rounds its
+//               sums to BF16 into a 128B-swizzled staging buffer and hands it to TMA
 //               tensor stores, so the warps go straight back to the next tile (stores
 //               outside M x N are clipped by the TMA unit).
 // Every mbarrier wait is bounded (wall-clock limit plus an iteration cap). A wait that
@@ -44,18 +48,19 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 128;                  // one scale block of K per stage
-constexpr int SC_STAGES = 8;
+constexpr int KPS = 4;        // K blocks of scales per scale-ring slot
+constexpr int SC_STAGES = 4;  // scale-ring slots, i.e. 16 K blocks of look-ahead
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_FIRST_WARP = 4;               // warps 0-3 form warpgroup 0
 constexpr int THREADS = 32 * (EPI_FIRST_WARP + EPI_WARPS);  // 384: three warpgroups
 // Register split. The CTA is launched with LAUNCH_REGS per thread (what ptxas gets for
-// 384 threads and one CTA per SM); warpgroup 0 (TMA, MMA, two idle warps) then gives
+// 384 threads and one CTA per SM); warpgroup 0 (TMA, MMA, scale loader, one idle warp) gives
 // registers back and the two promotion warpgroups take them:
 //   128 * PRODUCER_REGS + 256 * CONSUMER_REGS == 384 * LAUNCH_REGS  (64512)
-// and per SM sub-partition (one warp of each warpgroup) 32 * (40 + 2 * 232) <= 16384.
+// and per SM sub-partition (one warp of each warpgroup) 32 * (56 + 2 * 224) <= 16384.
 constexpr int LAUNCH_REGS = 168;
-constexpr int PRODUCER_REGS = 40;
-constexpr int CONSUMER_REGS = 232;
+constexpr int PRODUCER_REGS = 56;
+constexpr int CONSUMER_REGS = 224;
 static_assert(128 * PRODUCER_REGS + 256 * CONSUMER_REGS == THREADS * LAUNCH_REGS,
               "register split must add up to the launch allocation");
 constexpr int A_BYTES = BM * BK;          // 16 KB
@@ -63,15 +68,18 @@ constexpr int STG_BOX_BYTES = 32 * 128;   // 32 rows x 64 BF16 columns, 128B-swi
 
 // Tile width TN (256 or 128) sets the rest. TMEM holds 512 FP32 columns, i.e.
 // 512 / TN partial buffers; each promotion warp owns TN / 2 columns of one lane quadrant.
-template <int TN>
+template <int LAYOUT, int TN>
 struct Cfg {
   static constexpr int BN = TN;
   static constexpr int NBUF = 512 / TN;            // TMEM partial buffers
   static constexpr int WCOLS = TN / 2;             // columns per promotion warp
-  static constexpr int CHUNKS = WCOLS / 64;        // 64-column TMEM loads per K block
   static constexpr int STAGES = TN == 256 ? 3 : 5;
   static constexpr int B_BYTES = TN * BK;
-  static constexpr int SC_BYTES = TN * 4;          // wgrad column scales per K block
+  // Scale-ring slot, KPS K blocks: KPS x 128 row scales of A, then KPS x SB_STRIDE
+  // scales of B (TN column scales for wgrad, one per 128-column block otherwise).
+  static constexpr int SB_STRIDE = LAYOUT == PURO_WGRAD ? TN : 4;
+  static constexpr int SC_SLOT_FLOATS = KPS * (BM + SB_STRIDE);
+  static constexpr int SC_SLOT_BYTES = SC_SLOT_FLOATS * 4;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC = idesc_e4m3_f32(BM, TN);
   static constexpr int STG_WARP_BYTES = (WCOLS / 64) * STG_BOX_BYTES;
@@ -79,7 +87,7 @@ struct Cfg {
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;  // output staging, one per warp
   static constexpr int OFF_SC = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
-  static constexpr int OFF_BAR = OFF_SC + SC_STAGES * SC_BYTES;
+  static constexpr int OFF_BAR = OFF_SC + SC_STAGES * SC_SLOT_BYTES;
   static constexpr int N_BARS = 2 * STAGES + 2 * NBUF + 2 * SC_STAGES + 1;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
@@ -129,11 +137,10 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 template <int LAYOUT, int TN>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmC,
-                     const GemmArgs args) {
-  using C = Cfg<TN>;
+                     const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+  using C = Cfg<LAYOUT, TN>;
   constexpr int BN = C::BN, NBUF = C::NBUF, STAGES = C::STAGES;
-  constexpr int B_BYTES = C::B_BYTES, SC_BYTES = C::SC_BYTES;
+  constexpr int B_BYTES = C::B_BYTES;
   constexpr int OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_STG = C::OFF_STG, OFF_SC = C::OFF_SC;
   constexpr int OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC, N_BARS = C::N_BARS;
   extern __shared__ uint8_t smem_raw[];
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(tempty_bar(b), EPI_WARPS);
     }
     for (int s = 0; s < SC_STAGES; ++s) {
-      mbar_init(sfull_bar(s), 1);
+      mbar_init(sfull_bar(s), 32);  // one cp.async completion arrival per loader lane
       mbar_init(sempty_bar(s), EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
@@ -176,7 +183,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmC);
-    if (LAYOUT == PURO_WGRAD) prefetch_tensormap(&tmS);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -198,8 +204,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int s = 0, ss = 0;
-      uint32_t ph = 0, sph = 0;
+      int s = 0;
+      uint32_t ph = 0;
       uint32_t issued = 0, issued_parity = 0;  // per-stage bit masks
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
@@ -215,15 +221,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           tma_load_2d(sbase + OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
           issued |= 1u << s;
           issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
-          if (LAYOUT == PURO_WGRAD) {
-            if (!mbar_wait(sempty_bar(ss), sph ^ 1u, tmo, abort)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(sfull_bar(ss), SC_BYTES);
-            tma_load_2d(sbase + OFF_SC + ss * SC_BYTES, &tmS, sfull_bar(ss), nt * BN, kb);
-            if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
-          }
           if (++s == STAGES) s = 0, ph ^= 1u;
         }
       }
@@ -267,6 +264,56 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_wait(drain_bar, 0, tmo, nullptr);
       }
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale loader
+    // Scales outside the matrix are zero-filled, so the promotion needs no bounds checks.
+    const int nb_total = (args.N + 127) / 128;
+    int ss = 0;
+    uint32_t sph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      int mt, nt;
+      tile_coords(tile, args, mt, nt);
+      for (int kb0 = 0; kb0 < kblocks; kb0 += KPS) {
+        if (!mbar_wait(sempty_bar(ss), sph ^ 1u, tmo, abort)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = sbase + OFF_SC + ss * C::SC_SLOT_BYTES;
+        const int nk = kblocks - kb0 < KPS ? kblocks - kb0 : KPS;
+        for (int q = 0; q < nk; ++q) {
+          const int kb = kb0 + q;
+          const float *a_row = args.As + static_cast<int64_t>(kb) * args.M;
+#pragma unroll 1
+          for (int i = lane; i < BM; i += 32) {
+            const int m = mt * BM + i;
+            const bool v = m < args.M;
+            cp_async_4(dst + 4 * (q * BM + i), v ? a_row + m : args.As, v);
+          }
+          const uint32_t dsb = dst + 4 * (KPS * BM + q * C::SB_STRIDE);
+          if (LAYOUT == PURO_WGRAD) {
+            const float *b_row = args.Bs + static_cast<int64_t>(kb) * args.N;
+#pragma unroll 1
+            for (int i = lane; i < BN; i += 32) {
+              const int n = nt * BN + i;
+              const bool v = n < args.N;
+              cp_async_4(dsb + 4 * i, v ? b_row + n : args.Bs, v);
+            }
+          } else if (lane < BN / 128) {
+            const int nb = nt * (BN / 128) + lane;
+            const bool v = nb < nb_total;
+            const float *src = LAYOUT == PURO_FPROP
+                                   ? args.Bs + static_cast<int64_t>(nb) * kblocks + kb
+                                   : args.Bs + static_cast<int64_t>(kb) * nb_total + nb;
+            cp_async_4(dsb + 4 * lane, v ? src : args.Bs, v);
+          }
+        }
+        cp_async_mbar_arrive_noinc(sfull_bar(ss));
+        if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
+      }
+    }
+    if (!ok) raise_abort(abort, args.status);
+    cp_async_wait_all();  // no copy may land after the CTA has exited
   }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(CONSUMER_REGS));
@@ -276,7 +323,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int half = (warp - EPI_FIRST_WARP) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int nb_total = (args.N + 127) / 128;
     uint32_t use = 0;
     int ss = 0;
     uint32_t sph = 0;
@@ -284,77 +330,99 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
       int mt, nt;
       tile_coords(tile, args, mt, nt);
-      const int m = mt * BM + row;
-      const bool m_ok = m < args.M;
       const int n_base = nt * BN + half * WCOLS;  // first column of this warp
-      const int nb = n_base / 128;                // its 128-wide scale block of N
-      const bool nb_ok = nb < nb_total;
       uint64_t acc[WCOLS / 2];
 #pragma unroll
       for (int i = 0; i < WCOLS / 2; ++i) acc[i] = 0;
 
-      auto load_sa = [&](int kb) -> float {
-        return m_ok ? __ldg(args.As + static_cast<int64_t>(kb) * args.M + m) : 0.0f;
-      };
-      auto load_sb = [&](int kb) -> float {
-        if (LAYOUT == PURO_WGRAD || !nb_ok) return 0.0f;
-        return LAYOUT == PURO_FPROP ? __ldg(args.Bs + static_cast<int64_t>(nb) * kblocks + kb)
-                                    : __ldg(args.Bs + static_cast<int64_t>(kb) * nb_total + nb);
-      };
-      float sa_next = load_sa(0);
-      float sb_next = load_sb(0);
       for (int kb = 0; kb < kblocks; ++kb, ++use) {
-        const float sa = sa_next;
-        const float sb = sb_next;
-        if (kb + 1 < kblocks) {
-          sa_next = load_sa(kb + 1);
-          sb_next = load_sb(kb + 1);
-        }
         const uint32_t b = use % NBUF;
-        // wgrad: the K block's column scales arrive well ahead of its partials, so the
-        // per-column factors t = sA * sB[n] are formed before the TMEM wait and the
-        // partials then need one FMA each, as in fprop and dgrad.
-        uint64_t t2[LAYOUT == PURO_WGRAD ? WCOLS / 2 : 1];
-        if (LAYOUT == PURO_WGRAD) {
-          if (!mbar_wait(sfull_bar(ss), sph, tmo, abort)) {
+        // Scales come KPS K blocks per ring slot, well ahead of the partials: one wait at
+        // the slot's first K block, one release after its last.
+        const int kq = kb % KPS;
+        if (kq == 0 && !mbar_wait(sfull_bar(ss), sph, tmo, abort)) {
+          ok = false;
+          break;
+        }
+        const float *slot = sc_smem + ss * C::SC_SLOT_FLOATS;
+        const float sa = slot[kq * BM + row];
+        const float *sbk = slot + KPS * BM + kq * C::SB_STRIDE;
+        const bool slot_done = kq == KPS - 1 || kb == kblocks - 1;
+        auto release_slot = [&]() {
+          if (slot_done) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sempty_bar(ss));
+            if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
+          }
+        };
+        if constexpr (LAYOUT != PURO_WGRAD) {
+          // One scalar factor per thread and K block: partial * (sA * sB).
+          const float sb = sbk[(half * WCOLS) / 128];
+          release_slot();
+          const uint64_t s2 = pack2(sa * sb, sa * sb);
+          if (!mbar_wait(tfull_bar(b), (use / NBUF) & 1u, tmo, abort)) {
             ok = false;
             break;
           }
-          const float *sbv = sc_smem + ss * BN + half * WCOLS;
+          tc_fence_after_sync();
+          const uint32_t taddr = tmem + lane_base + b * BN + half * WCOLS;
+          // 32-column TMEM loads, double-buffered: chunk c + 1 is in flight while chunk
+          // c is added; the buffer goes back to the MMA warp once the last chunk is in.
+          constexpr int NCH = WCOLS / 32;
+          uint32_t ra[32], rb[32];
+          tmem_ld_32cols(taddr, ra);
+          tmem_wait_ld_dep(ra);
+#pragma unroll
+          for (int c = 0; c < NCH; c += 2) {
+            tmem_ld_32cols(taddr + 32 * (c + 1), rb);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              acc[16 * c + i] = ffma2(pack2(__uint_as_float(ra[2 * i]), __uint_as_float(ra[2 * i + 1])),
+                                      s2, acc[16 * c + i]);
+            tmem_wait_ld_dep(rb);
+            if (c + 2 < NCH) {
+              tmem_ld_32cols(taddr + 32 * (c + 2), ra);
+            } else {
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty_bar(b));
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              acc[16 * (c + 1) + i] =
+                  ffma2(pack2(__uint_as_float(rb[2 * i]), __uint_as_float(rb[2 * i + 1])), s2,
+                        acc[16 * (c + 1) + i]);
+            if (c + 2 < NCH) tmem_wait_ld_dep(ra);
+          }
+        } else {
+          // wgrad: a factor per column, t = sA * sB[n], formed while the partials are
+          // on their way from TMEM; then one FMA per partial.
+          static_assert(WCOLS == 64, "wgrad promotion reads 64 columns per warp");
+          if (!mbar_wait(tfull_bar(b), (use / NBUF) & 1u, tmo, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t taddr = tmem + lane_base + b * BN + half * WCOLS;
+          uint32_t r[64];
+          tmem_ld_64cols(taddr, r);
+          uint64_t t2[32];
+          const float *sbv = sbk + half * WCOLS;
           const uint64_t sa2 = pack2(sa, sa);
 #pragma unroll
-          for (int j = 0; j < WCOLS / 4; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const float4 sb4 = *reinterpret_cast<const float4 *>(sbv + 4 * j);
             t2[2 * j] = fmul2(sa2, pack2(sb4.x, sb4.y));
             t2[2 * j + 1] = fmul2(sa2, pack2(sb4.z, sb4.w));
           }
+          release_slot();
+          tmem_wait_ld_dep(r);
+          tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(sempty_bar(ss));
-          if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
-        }
-        if (!mbar_wait(tfull_bar(b), (use / NBUF) & 1u, tmo, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after_sync();
-        const uint32_t taddr = tmem + lane_base + b * BN + half * WCOLS;
-        const uint64_t s2 = pack2(sa * sb, sa * sb);
-        // 64-column TMEM loads, one wait each; the buffer goes back to the MMA warp as
-        // soon as the last one has landed in registers.
-#pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c) {
-          uint32_t r[64];
-          tmem_ld_64cols(taddr + 64 * c, r);
-          tmem_wait_ld();
-          if (c == C::CHUNKS - 1) {
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(b));
-          }
+          if (lane == 0) mbar_arrive(tempty_bar(b));
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            acc[32 * c + i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
-                                    LAYOUT == PURO_WGRAD ? t2[32 * c + i] : s2, acc[32 * c + i]);
+            acc[i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), t2[i], acc[i]);
         }
       }
       if (!ok) break;
@@ -453,12 +521,12 @@ int *device_status_ptr() {
 }
 
 template <int LAYOUT>
-int launch_layout(const uint8_t *Aq, const uint8_t *Bq, const float *Bs, uint16_t *Cout,
+int launch_layout(const uint8_t *Aq, const uint8_t *Bq, uint16_t *Cout,
                   GemmArgs args, int sms, cudaStream_t stream) {
   constexpr int TN = TileFor<LAYOUT>::TN;
-  constexpr int SMEM_BYTES = Cfg<TN>::SMEM_BYTES;
+  constexpr int SMEM_BYTES = Cfg<LAYOUT, TN>::SMEM_BYTES;
   const int64_t M = args.M, N = args.N, K = args.K;
-  CUtensorMap ta, tb, ts, tc;
+  CUtensorMap ta, tb, tc;
   if (!make_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, TN, BK,
@@ -466,13 +534,6 @@ int launch_layout(const uint8_t *Aq, const uint8_t *Bq, const float *Bs, uint16_
       !make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return PURO_ERR_CUDA;
-  if (LAYOUT == PURO_WGRAD) {
-    if (!make_map(&ts, Bs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, K / 128, N, 1, TN,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
-      return PURO_ERR_CUDA;
-  } else {
-    ts = tb;  // unused
-  }
   args.num_m = static_cast<int>((M + BM - 1) / BM);
   args.num_n = static_cast<int>((N + TN - 1) / TN);
   const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
@@ -492,7 +553,7 @@ int launch_layout(const uint8_t *Aq, const uint8_t *Bq, const float *Bs, uint16_
     std::fprintf(stderr, "puro_fp8: cudaFuncSetAttribute: %s\n", cudaGetErrorString(e));
     return PURO_ERR_CUDA;
   }
-  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, ts, tc, args);
+  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, args);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     std::fprintf(stderr,
@@ -532,9 +593,9 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
   args.status = status;
 
   switch (layout) {
-    case PURO_FPROP: return launch_layout<PURO_FPROP>(Aq, Bq, Bs, C, args, sms, stream);
-    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(Aq, Bq, Bs, C, args, sms, stream);
-    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(Aq, Bq, Bs, C, args, sms, stream);
+    case PURO_FPROP: return launch_layout<PURO_FPROP>(Aq, Bq, C, args, sms, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(Aq, Bq, C, args, sms, stream);
+    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(Aq, Bq, C, args, sms, stream);
     default: return PURO_ERR_LAYOUT;
   }
 }

@@ -131,8 +131,7 @@ PURO_API int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, 
  *   C   [M, N] BF16, dense            output
  *   workspace, ws_bytes   reserved for split-K; may be NULL / 0.
  * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, Bq, C 16-byte aligned;
- * As, Bs 4-byte aligned (Bs 16-byte aligned for PURO_WGRAD). M and N need not be
- * multiples of the tile size.
+ * As, Bs 4-byte aligned. M and N need not be multiples of the tile size.
  */
 PURO_API int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                             const float *Bs, uint16_t *C, int64_t M, int64_t N, int64_t K,

@@ -100,7 +100,8 @@ def test_gemm_validation(lib):
     assert f(*args, 128, 250, 256, 0, None, 0, None) == ESHAPE       # N % 8
     assert f(*args, 128, 256, 200, 0, None, 0, None) == ESHAPE       # K % 128
     assert f(A16 + 1, *args[1:], 128, 256, 256, 0, None, 0, None) == EALIGN
-    assert f(*args[:3], A16 + 4, A16, 128, 256, 256, 2, None, 0, None) == EALIGN  # wgrad Bs
+    assert f(*args[:3], A16 + 2, A16, 128, 256, 256, 2, None, 0, None) == EALIGN  # Bs
+    assert f(A16, A16 + 1, *args[2:], 128, 256, 256, 1, None, 0, None) == EALIGN  # As
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
