@@ -9,7 +9,7 @@ linears plus the 151936-wide head) over one micro-batch of 2 x 4096 = 8192 token
   backward sweep (head, blocks 27..0):  quantise dY (1x128 along tokens + row-wise, one
                                         read), quantise X along tokens, dgrad and wgrad
 That is 7 launches per linear, 791 per step, 84.56 TFLOP of GEMM work (2MNK, i.e.
-6 x linear parameters x tokens) and ~40 GB of quantiser traffic. Inputs are seeded
+6 x linear parameters x tokens) and 48.2 GB of quantiser traffic. Inputs are seeded
 synthetic BF16 tensors resident in HBM (about 21 GB, distinct per block, so every step
 reads far more than the 126 MB L2).
 
@@ -26,8 +26,10 @@ collective in the data path; the timing is the max over ranks).
 """
 
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -62,6 +64,40 @@ def _peaks():
             d = json.load(f)
         return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
     return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ DRAM traffic (ncu)
+
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "dram_traffic_qwen3_28L_lmhead_8192tok.md")
+KERNEL_SOURCES = {
+    "gemm": ["gemm.cu", "ptx.cuh"],
+    "quant": ["quant.cu", "quant_math.cuh", "ptx.cuh"],
+}
+
+
+def sources_sha256(kind):
+    """Hash of the CUDA sources a kernel family is built from."""
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "fp8_blockwise_scaled_e4m3_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kind):
+    """DRAM bytes (read + write) per launch of a kernel family, averaged over one step, as
+    recorded in the committed ncu summary; None if there is none or the family's sources
+    changed since it was captured."""
+    try:
+        with open(TRAFFIC_SUMMARY) as f:
+            text = f.read()
+    except OSError:
+        return None
+    sha = re.search(rf"^{kind}_sources_sha256: ([0-9a-f]{{64}})$", text, re.M)
+    val = re.search(rf"^{kind}_dram_bytes_per_launch: (\d+)$", text, re.M)
+    if sha is None or val is None or sha.group(1) != sources_sha256(kind):
+        return None
+    return int(val.group(1))
 
 
 # ------------------------------------------------------------------ clocks sampler
@@ -168,6 +204,16 @@ class Step:
             qb += T * n * (2 + 2) + 4 * (T * (n // 128) + (T // 128) * n)  # dY dual
             qb += T * k * (2 + 1) + 4 * (T // 128) * k                  # X along tokens
         self.quant_bytes = qb
+        # algorithmic GEMM bytes: FP8 operands and FP32 scales read once, BF16 output written
+        gb = 0
+        for _, x, w, dy, *_ in self.linears:
+            n, k = w.shape
+            gb += T * k + n * k + 4 * (T * k // 128 + (n // 128) * (k // 128)) + 2 * T * n   # fprop
+            gb += T * n + n * k + 4 * (T * n // 128 + (n // 128) * (k // 128)) + 2 * T * k   # dgrad
+            gb += n * T + k * T + 4 * (n + k) * (T // 128) + 2 * n * k                      # wgrad
+        self.gemm_bytes = gb
+        self.gemm_launches = 3 * len(self.linears)
+        self.quant_launches = 4 * len(self.linears)
         self.launches_per_step = 7 * len(self.linears)
 
     def run(self, ev=None, stream=None, after_wgrad=None):
@@ -368,11 +414,15 @@ def run_ours(args):
                      "frac": round(gemm_tflops / fp8_peak_measured, 4),
                      "peak_note": f"2 x {peak_src} sustained BF16 ({bf16_tf_sus}); "
                                   f"frac of nominal 4.5 PF = {gemm_tflops / FP8_DENSE_PEAK_TFLOPS:.4f}",
-                     "traffic": None,
+                     "traffic": ncu_traffic("gemm"),
+                     "traffic_unit": "DRAM bytes per launch (ncu, one step, mean over launches)",
+                     "algorithmic_bytes_per_launch": round(step.gemm_bytes / step.gemm_launches),
                      "launches_timed": n_gemm, "avg_launch_ms": round(t_gemm / max(n_gemm, 1), 4)},
         "roofline_quant": {"bound": "hbm", "kernel": "quantisers (k_quant_rows/cols/weight)",
                            "achieved": round(quant_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                            "frac": round(quant_gbs / hbm_gbs, 4),
+                           "traffic": ncu_traffic("quant"),
+                           "algorithmic_bytes_per_launch": round(step.quant_bytes / step.quant_launches),
                            "peak_note": f"{peak_src} copy bandwidth; frac of nominal 8 TB/s = "
                                         f"{quant_gbs / 8000:.4f}",
                            "launches_timed": n_quant, "avg_launch_ms": round(t_quant / max(n_quant, 1), 4)},
