@@ -13,12 +13,12 @@
 //   Q_DUAL    both of the above from one read of X
 //   Q_WEIGHT  one group per 128x128 tile:        Wq [R, C], S [ceil(R/128)][C/128],
 //             and optionally the same codes transposed, WqT [C, R]
-// Tiles arrive by TMA (two 64-column boxes with the 128-byte swizzle) into a 5-stage
-// mbarrier ring of shared memory, so the next tiles are in flight while the current
-// one is computed and nothing in flight occupies registers. Row-wise codes leave with
-// coalesced 8-byte stores; transposed codes are assembled in a swizzled shared tile
-// and written by one TMA tensor store. TMA zero-fills reads past the edge (no effect
-// on amax) and clips writes past it. Every wait is bounded.
+// Tiles arrive by TMA (two 64-column boxes with the 128-byte swizzle) into a 2-stage
+// mbarrier ring of shared memory per CTA (two CTAs per SM), so the next tiles are in
+// flight while the current one is computed and nothing in flight occupies registers.
+// Row-wise codes leave with coalesced 8-byte stores; transposed codes are assembled in a
+// swizzled shared tile and written by one TMA tensor store. TMA zero-fills reads past the
+// edge (no effect on amax) and clips writes past it. Every wait is bounded.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -39,19 +39,22 @@ namespace {
 enum QMode { Q_ROWS = 1, Q_COLS = 2, Q_DUAL = 3, Q_WEIGHT = 4 };
 
 constexpr int kTile = 128;
-// Threads per CTA: many warps hide the shared-memory and conversion latencies of the
-// per-tile work; the register budget (64K per SM) sets the count per mode.
+// Two CTAs per SM, each with its own 2-stage ring: the phases of one CTA's tile are
+// separated by CTA barriers, and the other CTA's work fills the SM while they drain.
+// Threads per CTA: the register budget (64K per SM, two CTAs) sets the count per mode.
 template <int MODE>
 struct Threads {
-  static constexpr int value = MODE == 1 ? 1024 : 512;
+  static constexpr int value = MODE == 1 ? 512 : 256;
 };
-constexpr int kStages = 5;
+constexpr int kStages = 2;
+constexpr int kCtasPerSm = 2;
 constexpr int kBoxBytes = kTile * 128;         // 128 rows x 64 BF16 (128 bytes), swizzled
 constexpr int kStageBytes = 2 * kBoxBytes;     // one 128 x 128 BF16 tile
 constexpr int kOffCodes = kStages * kStageBytes;
 constexpr int kOffPart = kOffCodes + kTile * kTile;  // 128 x 128 code tile, swizzled
 constexpr int kOffWarpMax = kOffPart + 16 * kTile * 4;   // up to 16 token groups
-constexpr int kOffBar = kOffWarpMax + 32 * 4;
+constexpr int kOffColDiv = kOffWarpMax + 32 * 4;     // per tile column: divisor s, 1/s
+constexpr int kOffBar = kOffColDiv + kTile * 8;
 constexpr int kOffMisc = kOffBar + 8 * kStages;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -71,12 +74,11 @@ struct QArgs {
 __device__ int g_quant_status;  // non-zero: a bounded wait gave up since the last read
 
 
-__device__ __forceinline__ float absmax8(const uint4 &v) {
-  float m = fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x)));
-  m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y))));
-  m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))));
-  m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w))));
-  return m;
+// Packed magnitude maximum of the 16 BF16 values in v0 and v1 (per half, see
+// bf16x2_absmax).
+__device__ __forceinline__ uint32_t absmax16(const uint4 &v0, const uint4 &v1) {
+  return bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(v0.x, v0.y), bf16x2_absmax(v0.z, v0.w)),
+                       bf16x2_absmax(bf16x2_absmax(v1.x, v1.y), bf16x2_absmax(v1.z, v1.w)));
 }
 
 __device__ __forceinline__ uint2 codes8(const uint4 &v, const BlockDivider &div) {
@@ -85,15 +87,15 @@ __device__ __forceinline__ uint2 codes8(const uint4 &v, const BlockDivider &div)
 
 // Scale of a block with absolute maximum `amax`, and the divider for its codes.
 __device__ __forceinline__ void block_scale(float amax, float &s, BlockDivider &div) {
-  s = __fdiv_rn(amax, 448.0f);
+  s = scale_of_amax(amax);
   div = amax > 0.0f ? make_divider(s) : zero_block_divider();
 }
 
-// Max over each group of 8 consecutive lanes.
-__device__ __forceinline__ float lane8_max(float v) {
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+// Packed magnitude maximum over each group of 8 consecutive lanes.
+__device__ __forceinline__ uint32_t lane8_absmax(uint32_t v) {
+  v = bf16x2_absmax(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  v = bf16x2_absmax(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  v = bf16x2_absmax(v, __shfl_xor_sync(0xffffffffu, v, 1));
   return v;
 }
 
@@ -155,7 +157,7 @@ __device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[TG],
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(Threads<MODE>::value, 1)
+__global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
     k_quant_tiles(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
                   const QArgs args) {
   constexpr bool kRows = MODE == Q_ROWS || MODE == Q_DUAL;
@@ -172,6 +174,7 @@ __global__ void __launch_bounds__(Threads<MODE>::value, 1)
   uint8_t *codes = smem + kOffCodes;
   float (*part)[kTile] = reinterpret_cast<float (*)[kTile]>(smem + kOffPart);
   float *warp_max = reinterpret_cast<float *>(smem + kOffWarpMax);
+  float2 *col_div = reinterpret_cast<float2 *>(smem + kOffColDiv);
   const uint32_t bar0 = sbase + kOffBar;
   volatile int *fail = reinterpret_cast<volatile int *>(smem + kOffMisc);
 
@@ -227,13 +230,14 @@ __global__ void __launch_bounds__(Threads<MODE>::value, 1)
     // ---------------------------------------------------------------- weight block
     BlockDivider wdiv = zero_block_divider();
     if (kWeight) {
-      float m = 0.0f;
+      uint32_t m2 = 0u;
 #pragma unroll
       for (int p = 0; p < kTile / RSTEP; ++p)
-        m = fmaxf(m, fmaxf(absmax8(row_chunk(stage, rg + RSTEP * p, 0, j8)),
-                           absmax8(row_chunk(stage, rg + RSTEP * p, 1, j8))));
+        m2 = bf16x2_absmax(m2, absmax16(row_chunk(stage, rg + RSTEP * p, 0, j8),
+                                        row_chunk(stage, rg + RSTEP * p, 1, j8)));
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      for (int o = 16; o > 0; o >>= 1) m2 = bf16x2_absmax(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+      const float m = bf16x2_absmax_to_f32(m2);
       if (lane == 0) warp_max[warp] = m;
       __syncthreads();
       float amax = warp_max[0];
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(Threads<MODE>::value, 1)
         const uint4 v1 = row_chunk(stage, r, 1, j8);
         BlockDivider div = wdiv;
         float srow = 0.0f;
-        if (kRows) block_scale(lane8_max(fmaxf(absmax8(v0), absmax8(v1))), srow, div);
+        if (kRows) block_scale(bf16x2_absmax_to_f32(lane8_absmax(absmax16(v0, v1))), srow, div);
         const uint2 q0 = codes8(v0, div);
         const uint2 q1 = codes8(v1, div);
         const int64_t row = r0 + r;
@@ -272,32 +276,37 @@ __global__ void __launch_bounds__(Threads<MODE>::value, 1)
       read_column_pairs<TG>(stage, w);
       BlockDivider d0 = wdiv, d1 = wdiv;
       if (kCols) {
-        float a0 = 0.0f, a1 = 0.0f;
+        uint32_t m2 = 0u;  // column 2cp in the low half, 2cp + 1 in the high half
 #pragma unroll
-        for (int k = 0; k < TG; ++k) {
-          a0 = fmaxf(a0, fabsf(bf16_lo(w[k])));
-          a1 = fmaxf(a1, fabsf(bf16_hi(w[k])));
-        }
-        part[g][2 * cp] = a0;
-        part[g][2 * cp + 1] = a1;
+        for (int k = 0; k < TG; ++k) m2 = bf16x2_absmax(m2, w[k]);
+        part[g][2 * cp] = __uint_as_float((m2 & 0x7FFFu) << 16);
+        part[g][2 * cp + 1] = __uint_as_float(m2 & 0x7FFF0000u);
       }
       __syncthreads();  // column partials ready; the code tile is free (thread 0 waited)
       if (kCols) {
-        float a0 = part[0][2 * cp], a1 = part[0][2 * cp + 1];
-#pragma unroll
-        for (int k = 1; k < NG; ++k) {
-          a0 = fmaxf(a0, part[k][2 * cp]);
-          a1 = fmaxf(a1, part[k][2 * cp + 1]);
-        }
-        float s0, s1;
-        block_scale(a0, s0, d0);
-        block_scale(a1, s1, d1);
+        // The first 64 threads finish the column maxima and form the 128 column scales
+        // and divisors once; every thread then reads the two it needs.
         if (g == 0) {
+          float a0 = part[0][2 * cp], a1 = part[0][2 * cp + 1];
+#pragma unroll
+          for (int k = 1; k < NG; ++k) {
+            a0 = fmaxf(a0, part[k][2 * cp]);
+            a1 = fmaxf(a1, part[k][2 * cp + 1]);
+          }
+          float s0, s1;
+          block_scale(a0, s0, d0);
+          block_scale(a1, s1, d1);
+          col_div[2 * cp] = make_float2(d0.s, d0.fast ? d0.r : 0.0f);
+          col_div[2 * cp + 1] = make_float2(d1.s, d1.fast ? d1.r : 0.0f);
           const int64_t c = c0 + 2 * cp;
           float *strow = args.st + static_cast<int64_t>(tr) * args.C;
           if (c < args.C) strow[c] = s0;
           if (c + 1 < args.C) strow[c + 1] = s1;
         }
+        __syncthreads();
+        const float2 e0 = col_div[2 * cp], e1 = col_div[2 * cp + 1];
+        d0 = BlockDivider{e0.x, e0.y, e0.y != 0.0f};
+        d1 = BlockDivider{e1.x, e1.y, e1.y != 0.0f};
       }
       column_codes_to_smem<TG>(w, d0, d1, codes);
       fence_proxy_async_smem();
@@ -395,7 +404,7 @@ int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *
   args.tiles_c = static_cast<int>((C + kTile - 1) / kTile);
   args.timeout_ns = wait_timeout_ns();
   const int64_t tiles = static_cast<int64_t>(args.tiles_r) * args.tiles_c;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  const int grid = static_cast<int>(tiles < kCtasPerSm * sms ? tiles : kCtasPerSm * sms);
   auto kern = k_quant_tiles<MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
       cudaSuccess)

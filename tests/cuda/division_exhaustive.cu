@@ -1,4 +1,5 @@
-// Test-only kernel: the quantisers' per-block quotient (Markstein's correction with a
+// Test-only kernels: the quantisers' block scale s = RN(amax / 448) against IEEE division
+// for every positive finite BF16 amax, and their per-block quotient (Markstein's correction with a
 // correctly rounded reciprocal, IEEE division for tiny scales) against CUDA's
 // correctly rounded division, for every pair the quantisers can meet: every positive
 // finite BF16 amax, its scale s = RN(amax / 448), and every BF16 x with |x| <= amax.
@@ -59,7 +60,48 @@ __global__ void k_check(unsigned long long *counts, unsigned int *first_bad) {
   }
 }
 
+// Block scales: scale_of_amax(amax) against __fdiv_rn(amax, 448) for every positive finite
+// BF16 amax. counts[0] = bit mismatches, counts[1] = values checked.
+__global__ void k_scale_check(unsigned long long *counts, unsigned int *first_bad) {
+  const uint32_t amax_bits = blockIdx.x * blockDim.x + threadIdx.x + 1;  // 0x0001 ..
+  unsigned long long bad = 0, n = 0;
+  if (amax_bits <= 0x7F7Fu) {
+    const float amax = __uint_as_float(amax_bits << 16);
+    ++n;
+    if (__float_as_uint(puro::scale_of_amax(amax)) != __float_as_uint(__fdiv_rn(amax, 448.0f))) {
+      ++bad;
+      atomicCAS(first_bad, 0u, amax_bits);
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    n += __shfl_xor_sync(0xffffffffu, n, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(counts + 0, bad);
+    atomicAdd(counts + 1, n);
+  }
+}
+
 }  // namespace
+
+extern "C" int run_scale_check(unsigned long long *host_counts, unsigned int *host_first_bad) {
+  unsigned long long *counts = nullptr;
+  unsigned int *first = nullptr;
+  if (cudaMalloc(&counts, 2 * sizeof(unsigned long long)) != cudaSuccess) return 1;
+  if (cudaMalloc(&first, sizeof(unsigned int)) != cudaSuccess) return 2;
+  cudaMemset(counts, 0, 2 * sizeof(unsigned long long));
+  cudaMemset(first, 0, sizeof(unsigned int));
+  k_scale_check<<<(0x7F7F + 255) / 256, 256>>>(counts, first);
+  if (cudaGetLastError() != cudaSuccess) return 3;
+  if (cudaMemcpy(host_counts, counts, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return 4;
+  cudaMemcpy(host_first_bad, first, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+  cudaFree(counts);
+  cudaFree(first);
+  return 0;
+}
 
 extern "C" int run_division_check(unsigned long long *host_counts, unsigned int *host_first_bad) {
   unsigned long long *counts = nullptr;
