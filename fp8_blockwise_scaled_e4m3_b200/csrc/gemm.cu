@@ -240,8 +240,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
         for (int kb = 0; kb < kblocks; ++kb, ++use) {
           const uint32_t b = use % NBUF;
-          if (!mbar_wait(tempty_bar(b), ((use / NBUF) & 1u) ^ 1u, tmo, abort) ||
-              !mbar_wait(full_bar(s), ph, tmo, abort)) {
+          // The stage's operands are normally in long before its TMEM buffer is free, so
+          // that wait comes first and its cost overlaps the promotion still draining the
+          // buffer.
+          if (!mbar_wait(full_bar(s), ph, tmo, abort) ||
+              !mbar_wait(tempty_bar(b), ((use / NBUF) & 1u) ^ 1u, tmo, abort)) {
             ok = false;
             break;
           }
