@@ -56,13 +56,19 @@ constexpr int THREADS = 32 * (EPI_FIRST_WARP + EPI_WARPS);  // 384: three warpgr
 // Register split. The CTA is launched with LAUNCH_REGS per thread (what ptxas gets for
 // 384 threads and one CTA per SM); warpgroup 0 (TMA, MMA, scale loader, one idle warp) gives
 // registers back and the two promotion warpgroups take them:
-//   128 * PRODUCER_REGS + 256 * CONSUMER_REGS == 384 * LAUNCH_REGS  (64512)
-// and per SM sub-partition (one warp of each warpgroup) 32 * (56 + 2 * 224) <= 16384.
+//   128 * producer + 256 * consumer == 384 * LAUNCH_REGS  (64512)
+// and per SM sub-partition (one warp of each warpgroup) 32 * (producer + 2 * consumer)
+// <= 16384. fprop/dgrad hold 128 accumulator columns per promotion thread (56 / 224);
+// wgrad holds 64 and gives the producer side more (72 / 216).
 constexpr int LAUNCH_REGS = 168;
-constexpr int PRODUCER_REGS = 56;
-constexpr int CONSUMER_REGS = 224;
-static_assert(128 * PRODUCER_REGS + 256 * CONSUMER_REGS == THREADS * LAUNCH_REGS,
-              "register split must add up to the launch allocation");
+template <int LAYOUT>
+struct RegSplit {
+  static constexpr int producer = LAYOUT == PURO_WGRAD ? 72 : 56;
+  static constexpr int consumer = LAYOUT == PURO_WGRAD ? 216 : 224;
+  static_assert(128 * producer + 256 * consumer == THREADS * LAUNCH_REGS,
+                "register split must add up to the launch allocation");
+  static_assert(32 * (producer + 2 * consumer) <= 16384, "per sub-partition register file");
+};
 constexpr int A_BYTES = BM * BK;          // 16 KB
 constexpr int STG_BOX_BYTES = 32 * 128;   // 32 rows x 64 BF16 columns, 128B-swizzled
 
@@ -199,8 +205,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp < EPI_FIRST_WARP) {
     // Each role's code sits inside the branch that set its register limit, so ptxas
-    // allocates the promotion path with CONSUMER_REGS and this one with PRODUCER_REGS.
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PRODUCER_REGS));
+    // allocates the promotion path with the consumer share and this one with the producer's.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(RegSplit<LAYOUT>::producer));
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -319,7 +325,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     cp_async_wait_all();  // no copy may land after the CTA has exited
   }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(CONSUMER_REGS));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(RegSplit<LAYOUT>::consumer));
     // ------------------------------------------------------------ promotion + epilogue
     constexpr int WCOLS = C::WCOLS;
     const int quad = warp & 3;
@@ -398,34 +404,47 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (c + 2 < NCH) tmem_wait_ld_dep(ra);
           }
         } else {
-          // wgrad: a factor per column, t = sA * sB[n], formed while the partials are
-          // on their way from TMEM; then one FMA per partial.
+          // wgrad: a factor per element, sA[row] * sB[column]. The partials are read in the
+          // 16x256b shape, so a thread holds 4 rows x 16 columns of its warp's 32 x 64 block
+          // (rows g, g+8, g+16, g+24 with g = lane / 4; columns 8j + c, 8j + c + 1 with
+          // c = 2 * (lane % 4)) and needs 4 row scales and 16 column scales per K block
+          // instead of 1 and 64: a quarter of the shared-memory traffic.
           static_assert(WCOLS == 64, "wgrad promotion reads 64 columns per warp");
+          const int g = lane >> 2, c = 2 * (lane & 3);
+          const float *sav = slot + kq * BM + quad * 32 + g;
+          const float sa0 = sav[0], sa1 = sav[8], sa2 = sav[16], sa3 = sav[24];
+          const float *sbv = slot + KPS * BM + kq * C::SB_STRIDE + half * WCOLS + c;
+          uint64_t sbp[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sbp[j] = *reinterpret_cast<const uint64_t *>(sbv + 8 * j);
+          release_slot();
           if (!mbar_wait(tfull_bar(b), (use / NBUF) & 1u, tmo, abort)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
           const uint32_t taddr = tmem + lane_base + b * BN + half * WCOLS;
-          uint32_t r[64];
-          tmem_ld_64cols(taddr, r);
-          uint64_t t2[32];
-          const float *sbv = sbk + half * WCOLS;
-          const uint64_t sa2 = pack2(sa, sa);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float4 sb4 = *reinterpret_cast<const float4 *>(sbv + 4 * j);
-            t2[2 * j] = fmul2(sa2, pack2(sb4.x, sb4.y));
-            t2[2 * j + 1] = fmul2(sa2, pack2(sb4.z, sb4.w));
-          }
-          release_slot();
-          tmem_wait_ld_dep(r);
+          uint32_t r0[32], r1[32];
+          tmem_ld_16x256b_x8(taddr, r0);                // rows g, g + 8
+          tmem_ld_16x256b_x8(taddr + (16u << 16), r1);  // rows g + 16, g + 24
+          tmem_wait_ld_dep(r0);
+          tmem_wait_ld_dep(r1);
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty_bar(b));
+          const uint64_t s0 = pack2(sa0, sa0), s1 = pack2(sa1, sa1);
+          const uint64_t s2 = pack2(sa2, sa2), s3 = pack2(sa3, sa3);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            acc[i] = ffma2(pack2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), t2[i], acc[i]);
+          for (int j = 0; j < 8; ++j) {
+            acc[j] = ffma2(pack2(__uint_as_float(r0[4 * j]), __uint_as_float(r0[4 * j + 1])),
+                           fmul2(s0, sbp[j]), acc[j]);
+            acc[8 + j] = ffma2(pack2(__uint_as_float(r0[4 * j + 2]), __uint_as_float(r0[4 * j + 3])),
+                               fmul2(s1, sbp[j]), acc[8 + j]);
+            acc[16 + j] = ffma2(pack2(__uint_as_float(r1[4 * j]), __uint_as_float(r1[4 * j + 1])),
+                                fmul2(s2, sbp[j]), acc[16 + j]);
+            acc[24 + j] = ffma2(pack2(__uint_as_float(r1[4 * j + 2]), __uint_as_float(r1[4 * j + 3])),
+                                fmul2(s3, sbp[j]), acc[24 + j]);
+          }
         }
       }
       if (!ok) break;
@@ -434,18 +453,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST_WARP) * C::STG_WARP_BYTES;
       if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores left the buffer
       __syncwarp();
+      if constexpr (LAYOUT != PURO_WGRAD) {
+        // thread = row `lane`, columns in order
 #pragma unroll
-      for (int j = 0; j < WCOLS / 8; ++j) {
-        float v[8];
-        unpack2(acc[4 * j], v[0], v[1]);
-        unpack2(acc[4 * j + 1], v[2], v[3]);
-        unpack2(acc[4 * j + 2], v[4], v[5]);
-        unpack2(acc[4 * j + 3], v[6], v[7]);
-        const uint32_t addr = stg + (j >> 3) * STG_BOX_BYTES + lane * 128 + (((j & 7) ^ (lane & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                     "r"(bf16x2_bits(v[0], v[1])), "r"(bf16x2_bits(v[2], v[3])),
-                     "r"(bf16x2_bits(v[4], v[5])), "r"(bf16x2_bits(v[6], v[7]))
-                     : "memory");
+        for (int j = 0; j < WCOLS / 8; ++j) {
+          float v[8];
+          unpack2(acc[4 * j], v[0], v[1]);
+          unpack2(acc[4 * j + 1], v[2], v[3]);
+          unpack2(acc[4 * j + 2], v[4], v[5]);
+          unpack2(acc[4 * j + 3], v[6], v[7]);
+          const uint32_t addr =
+              stg + (j >> 3) * STG_BOX_BYTES + lane * 128 + (((j & 7) ^ (lane & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "r"(bf16x2_bits(v[0], v[1])), "r"(bf16x2_bits(v[2], v[3])),
+                       "r"(bf16x2_bits(v[4], v[5])), "r"(bf16x2_bits(v[6], v[7]))
+                       : "memory");
+        }
+      } else {
+        // 16x256b ownership: acc[8x + j] is row g + 8x, columns 8j + c, 8j + c + 1; one
+        // 4-byte BF16 pair per store, bank-conflict free under the swizzle.
+        const int g = lane >> 2, c = 2 * (lane & 3);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float lo, hi;
+            unpack2(acc[8 * x + j], lo, hi);
+            const int r = g + 8 * x;
+            const uint32_t addr = stg + r * 128 + ((j ^ (r & 7)) << 4) + 2 * c;
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(bf16x2_bits(lo, hi)) : "memory");
+          }
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
