@@ -9,21 +9,21 @@
 // running FP32 sum with its two scales:
 //     C[m, n] = sum_kb  sA(kb, m) * sB(kb, n) * P_kb[m, n],   P_kb = Aq[m, kb] . Bq[n, kb]
 //
-// One persistent CTA per SM, tiles of 128 x TN (TN = 256 for fprop/dgrad, 128 for
-// wgrad), warp-specialised:
-//   warp 0      TMA producer: A and B tiles of one K block per ring stage
-//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one of the
-//               512 / TN TMEM buffers, committed to the stage's "empty" barrier and
+// One persistent CTA per SM, tiles of 128 x 256, warp-specialised:
+//   warp 0      TMA producer: A and B tiles of one K block per ring stage (3 stages)
+//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one of the two
+//               256-column TMEM buffers, committed to the stage's "empty" barrier and
 //               the buffer's "full" barrier; also owns the TMEM allocation
 //   warp 2      scale loader: for every K block, the tile's 128 row scales of A and its
 //               column scales of B (one per 128-column block, or one per column for
-//               wgrad) are copied with cp.async into an 8-slot shared-memory ring, so
-//               the promotion never waits on a global load
+//               wgrad) are copied with cp.async into a shared-memory ring, so the
+//               promotion never waits on a global load
 //   warp 3      idle (it completes warpgroup 0, which hands its registers over)
-//   warps 4..11 promotion + epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 and
-//               columns (TN/2)*((w-4)/4) .. +TN/2-1, i.e. one output row and TN/2
-//               columns per thread; partial * (sA * sB) is added into FP32 registers
-//               with packed FP32x2 FMAs; at the end of the tile each warp rounds its
+//   warps 4..11 promotion + epilogue: warp w owns TMEM lanes 32*(w%4) .. +31 (output rows)
+//               and columns 128*((w-4)/4) .. +127; partial * (sA * sB) is added into FP32
+//               registers with packed FP32x2 FMAs (fprop/dgrad: one row per thread, read
+//               in the 32x32b shape; wgrad: 4 rows x 32 columns per thread, read in the
+//               16x256b shape, see below); at the end of the tile each warp rounds its
 //               sums to BF16 into a 128B-swizzled staging buffer and hands it to TMA
 //               tensor stores, so the warps go straight back to the next tile (stores
 //               outside M x N are clipped by the TMA unit).
@@ -48,8 +48,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 128;                  // one scale block of K per stage
-constexpr int KPS = 4;        // K blocks of scales per scale-ring slot
-constexpr int SC_STAGES = 4;  // scale-ring slots, i.e. 16 K blocks of look-ahead
+constexpr int SC_STAGES = 4;  // scale-ring slots of KPS K blocks each
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_FIRST_WARP = 4;               // warps 0-3 form warpgroup 0
 constexpr int THREADS = 32 * (EPI_FIRST_WARP + EPI_WARPS);  // 384: three warpgroups
@@ -58,13 +57,12 @@ constexpr int THREADS = 32 * (EPI_FIRST_WARP + EPI_WARPS);  // 384: three warpgr
 // registers back and the two promotion warpgroups take them:
 //   128 * producer + 256 * consumer == 384 * LAUNCH_REGS  (64512)
 // and per SM sub-partition (one warp of each warpgroup) 32 * (producer + 2 * consumer)
-// <= 16384. fprop/dgrad hold 128 accumulator columns per promotion thread (56 / 224);
-// wgrad holds 64 and gives the producer side more (72 / 216).
+// <= 16384. Every promotion thread holds 128 FP32 sums.
 constexpr int LAUNCH_REGS = 168;
 template <int LAYOUT>
 struct RegSplit {
-  static constexpr int producer = LAYOUT == PURO_WGRAD ? 72 : 56;
-  static constexpr int consumer = LAYOUT == PURO_WGRAD ? 216 : 224;
+  static constexpr int producer = 56;
+  static constexpr int consumer = 224;
   static_assert(128 * producer + 256 * consumer == THREADS * LAUNCH_REGS,
                 "register split must add up to the launch allocation");
   static_assert(32 * (producer + 2 * consumer) <= 16384, "per sub-partition register file");
@@ -84,6 +82,9 @@ struct Cfg {
   // Scale-ring slot, KPS K blocks: KPS x 128 row scales of A, then KPS x SB_STRIDE
   // scales of B (TN column scales for wgrad, one per 128-column block otherwise).
   static constexpr int SB_STRIDE = LAYOUT == PURO_WGRAD ? TN : 4;
+  // K blocks of scales per slot (wgrad's 256 column scales per K block fill shared
+  // memory faster, so its slots are half as deep)
+  static constexpr int KPS = LAYOUT == PURO_WGRAD ? 2 : 4;
   static constexpr int SC_SLOT_FLOATS = KPS * (BM + SB_STRIDE);
   static constexpr int SC_SLOT_BYTES = SC_SLOT_FLOATS * 4;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -101,11 +102,11 @@ struct Cfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
-// fprop and dgrad carry one scalar scale per 128-column block and keep the wide tile;
-// wgrad scales every column, and its longer promotion gains more from four buffers.
+// Every layout uses 256-wide tiles (two TMEM buffers): measured faster than 128-wide
+// tiles with four buffers, for wgrad too once its promotion reads the 16x256b shape.
 template <int LAYOUT>
 struct TileFor {
-  static constexpr int TN = LAYOUT == PURO_WGRAD ? 128 : 256;
+  static constexpr int TN = 256;
 };
 
 struct GemmArgs {
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_STG = C::OFF_STG, OFF_SC = C::OFF_SC;
   constexpr int OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC, N_BARS = C::N_BARS;
+  constexpr int KPS = C::KPS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -405,18 +407,18 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else {
           // wgrad: a factor per element, sA[row] * sB[column]. The partials are read in the
-          // 16x256b shape, so a thread holds 4 rows x 16 columns of its warp's 32 x 64 block
-          // (rows g, g+8, g+16, g+24 with g = lane / 4; columns 8j + c, 8j + c + 1 with
-          // c = 2 * (lane % 4)) and needs 4 row scales and 16 column scales per K block
-          // instead of 1 and 64: a quarter of the shared-memory traffic.
-          static_assert(WCOLS == 64, "wgrad promotion reads 64 columns per warp");
+          // 16x256b shape, so a thread holds 4 rows x 32 columns of its warp's 32 x 128
+          // block (rows g, g+8, g+16, g+24 with g = lane / 4; columns 8p + c, 8p + c + 1
+          // with c = 2 * (lane % 4)) and needs 4 row scales and 32 column scales per K
+          // block instead of 1 and 128: a quarter of the shared-memory traffic.
+          static_assert(WCOLS == 128, "wgrad promotion reads 128 columns per warp");
           const int g = lane >> 2, c = 2 * (lane & 3);
           const float *sav = slot + kq * BM + quad * 32 + g;
           const float sa0 = sav[0], sa1 = sav[8], sa2 = sav[16], sa3 = sav[24];
           const float *sbv = slot + KPS * BM + kq * C::SB_STRIDE + half * WCOLS + c;
-          uint64_t sbp[8];
+          uint64_t sbp[16];  // column pairs 8p + c, 8p + c + 1
 #pragma unroll
-          for (int j = 0; j < 8; ++j) sbp[j] = *reinterpret_cast<const uint64_t *>(sbv + 8 * j);
+          for (int p = 0; p < 16; ++p) sbp[p] = *reinterpret_cast<const uint64_t *>(sbv + 8 * p);
           release_slot();
           if (!mbar_wait(tfull_bar(b), (use / NBUF) & 1u, tmo, abort)) {
             ok = false;
@@ -424,26 +426,42 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           tc_fence_after_sync();
           const uint32_t taddr = tmem + lane_base + b * BN + half * WCOLS;
-          uint32_t r0[32], r1[32];
-          tmem_ld_16x256b_x8(taddr, r0);                // rows g, g + 8
-          tmem_ld_16x256b_x8(taddr + (16u << 16), r1);  // rows g + 16, g + 24
-          tmem_wait_ld_dep(r0);
-          tmem_wait_ld_dep(r1);
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(b));
           const uint64_t s0 = pack2(sa0, sa0), s1 = pack2(sa1, sa1);
           const uint64_t s2 = pack2(sa2, sa2), s3 = pack2(sa3, sa3);
+          // 8 loads of 16 lanes x 32 columns: q = 2 * quarter + lane half; double-buffered.
+          uint32_t ra[16], rb[16];
+          auto issue = [&](int q, uint32_t (&r)[16]) {
+            tmem_ld_16x256b_x4(taddr + (static_cast<uint32_t>(16 * (q & 1)) << 16) + 32 * (q >> 1), r);
+          };
+          auto apply = [&](int q, const uint32_t (&r)[16]) {
+            const int lh = q & 1, cq = q >> 1;
+            const uint64_t sx = lh ? s2 : s0, sy = lh ? s3 : s1;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            acc[j] = ffma2(pack2(__uint_as_float(r0[4 * j]), __uint_as_float(r0[4 * j + 1])),
-                           fmul2(s0, sbp[j]), acc[j]);
-            acc[8 + j] = ffma2(pack2(__uint_as_float(r0[4 * j + 2]), __uint_as_float(r0[4 * j + 3])),
-                               fmul2(s1, sbp[j]), acc[8 + j]);
-            acc[16 + j] = ffma2(pack2(__uint_as_float(r1[4 * j]), __uint_as_float(r1[4 * j + 1])),
-                                fmul2(s2, sbp[j]), acc[16 + j]);
-            acc[24 + j] = ffma2(pack2(__uint_as_float(r1[4 * j + 2]), __uint_as_float(r1[4 * j + 3])),
-                                fmul2(s3, sbp[j]), acc[24 + j]);
+            for (int j = 0; j < 4; ++j) {
+              const int p = 4 * cq + j;
+              acc[(2 * lh) * 16 + p] = ffma2(pack2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])),
+                                             fmul2(sx, sbp[p]), acc[(2 * lh) * 16 + p]);
+              acc[(2 * lh + 1) * 16 + p] =
+                  ffma2(pack2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])),
+                        fmul2(sy, sbp[p]), acc[(2 * lh + 1) * 16 + p]);
+            }
+          };
+          issue(0, ra);
+          tmem_wait_ld_dep(ra);
+#pragma unroll
+          for (int q = 0; q < 8; q += 2) {
+            issue(q + 1, rb);
+            apply(q, ra);
+            tmem_wait_ld_dep(rb);
+            if (q + 2 < 8) {
+              issue(q + 2, ra);
+            } else {
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty_bar(b));
+            }
+            apply(q + 1, rb);
+            if (q + 2 < 8) tmem_wait_ld_dep(ra);
           }
         }
       }
@@ -476,11 +494,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int p = 0; p < 16; ++p) {
             float lo, hi;
-            unpack2(acc[8 * x + j], lo, hi);
-            const int r = g + 8 * x;
-            const uint32_t addr = stg + r * 128 + ((j ^ (r & 7)) << 4) + 2 * c;
+            unpack2(acc[16 * x + p], lo, hi);
+            const int r = g + 8 * x, j = p & 7;
+            const uint32_t addr = stg + (p >> 3) * STG_BOX_BYTES + r * 128 + ((j ^ (r & 7)) << 4) + 2 * c;
             asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(bf16x2_bits(lo, hi)) : "memory");
           }
         }
