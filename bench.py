@@ -217,20 +217,25 @@ class Step:
         self.quant_launches = 4 * len(self.linears)
         self.launches_per_step = 7 * len(self.linears)
 
-    def run(self, ev=None, stream=None, after_wgrad=None):
+    def run(self, ev=None, stream=None, after_wgrad=None, before_fwd=None, before_bwd=None):
         """Enqueue one step. ev: list to which (kind, event) pairs are appended after
-        each launch (an initial event must already be recorded). after_wgrad(i, dW) is
-        called right after linear i's wgrad is enqueued (its dW buffer is reused by the
+        each launch (an initial event must already be recorded). before_fwd(i) /
+        before_bwd(i) are called before linear i's forward / backward launches are
+        enqueued; after_wgrad(i, dW) right after its wgrad (the dW buffer is reused by the
         next linear of the same shape)."""
         pf = self.pf
         rec = (lambda kind: ev.append((kind, _record(self.torch)))) if ev is not None else (lambda kind: None)
-        for tag, x, w, dy, wq, wqt, ws in self.linears:
+        for i, (tag, x, w, dy, wq, wqt, ws) in enumerate(self.linears):
+            if before_fwd is not None:
+                before_fwd(i)
             s = self.scratch[tuple(w.shape)]
             pf.puro_fp8_quantize_1x128(x, s["xq"], s["xs"], stream); rec("q")
             pf.puro_fp8_quantize_128x128(w, wq, wqt, ws, stream); rec("q")
             pf.puro_fp8_gemm_blockwise(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, None, stream); rec("g")
         for i in range(len(self.linears) - 1, -1, -1):
             tag, x, w, dy, wq, wqt, ws = self.linears[i]
+            if before_bwd is not None:
+                before_bwd(i)
             s = self.scratch[tuple(w.shape)]
             pf.puro_fp8_quantize_1x128_transposed(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], stream); rec("q")
             pf.puro_fp8_quantize_1x128_transposed(x, s["xqt"], s["xst"], None, None, stream); rec("q")
@@ -455,7 +460,10 @@ def run_ours(args):
 def run_e2e(step, torch, pf, args, world):
     """The same step through the public API with host buffers: every step copies the BF16
     inputs (X, W, dY of every linear) from pinned host memory and reads the weight
-    gradients back into pinned host memory, inside the timed region."""
+    gradients back into pinned host memory, inside the timed region. The copies run on
+    their own streams in the order the step consumes the tensors (X and W per linear for
+    the forward sweep, then dY per linear for the backward sweep), and each linear's
+    kernels wait only for their own inputs, so compute overlaps the PCIe transfers."""
     try:
         host_in = []
         for lin in step.linears:
@@ -468,13 +476,41 @@ def run_e2e(step, torch, pf, args, world):
     h2d = sum(t.numel() * t.element_size() for ts in host_in for t in ts)
     d2h = sum(t.numel() * t.element_size() for t in host_dw)
 
+    comp = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    nlin = len(step.linears)
+
     def one_step():
-        for lin, hs in zip(step.linears, host_in):
-            for dev_t, h in zip(lin[1:4], hs):
-                dev_t.copy_(h, non_blocking=True)
-        step.run(after_wgrad=lambda i, dw: host_dw[i].copy_(dw, non_blocking=True))
+        h2d_s.wait_stream(comp)  # the previous step is done with every input buffer
+        fwd_ready, bwd_ready = [], [None] * nlin
+        with torch.cuda.stream(h2d_s):
+            for lin, hs in zip(step.linears, host_in):
+                lin[1].copy_(hs[0], non_blocking=True)
+                lin[2].copy_(hs[1], non_blocking=True)
+                fwd_ready.append(h2d_s.record_event())
+            for i in range(nlin - 1, -1, -1):
+                step.linears[i][3].copy_(host_in[i][2], non_blocking=True)
+                bwd_ready[i] = h2d_s.record_event()
+        read_back = {}  # per dW buffer: the read-back that must finish before it is reused
+
+        def before_bwd(i):
+            comp.wait_event(bwd_ready[i])
+            prev = read_back.get(tuple(step.linears[i][2].shape))
+            if prev is not None:
+                comp.wait_event(prev)
+
+        def after_wgrad(i, dw):
+            d2h_s.wait_event(comp.record_event())
+            with torch.cuda.stream(d2h_s):
+                host_dw[i].copy_(dw, non_blocking=True)
+            read_back[tuple(dw.shape)] = d2h_s.record_event()
+
+        step.run(stream=comp, before_fwd=lambda i: comp.wait_event(fwd_ready[i]), before_bwd=before_bwd,
+                 after_wgrad=after_wgrad)
+        comp.wait_stream(d2h_s)
 
     one_step()
+    comp.synchronize()
     _barrier_sync(world)
     steps = max(1, args.e2e_steps)
     t0 = _record(torch)
