@@ -83,6 +83,19 @@ int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *B
   return puro::launch_gemm_blockwise(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
 }
 
+int puro_fp8_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                                const float *Bs, float *C, int64_t M, int64_t N, int64_t K,
+                                puro_stream_t stream) {
+  if (Aq == nullptr || As == nullptr || Bq == nullptr || Bs == nullptr || C == nullptr)
+    return PURO_ERR_NULL;
+  if (M < 1 || N < 8 || N % 8 != 0 || K < 128 || K % 128 != 0) return PURO_ERR_SHAPE;
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
+  if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16) || !aligned(As, 4) || !aligned(Bs, 4))
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_gemm_wgrad_acc_f32(Aq, As, Bq, Bs, C, M, N, K, stream);
+}
+
 int puro_fp8_sync_status(puro_stream_t stream) {
   int gemm = 0, quant = 0;
   if (int e = puro::read_and_clear_device_status(stream, &gemm)) return e;

@@ -141,7 +141,9 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-template <int LAYOUT, int TN>
+// ACC32: instead of storing BF16, add the FP32 result into an FP32 C (main-gradient
+// accumulation of wgrad) with TMA reduce-add.
+template <int LAYOUT, int TN, bool ACC32>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
@@ -471,6 +473,49 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST_WARP) * C::STG_WARP_BYTES;
       if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores left the buffer
       __syncwarp();
+      if constexpr (ACC32) {
+        // FP32 out: four boxes of 32 rows x 32 columns (128-byte rows, 16-byte chunk k of
+        // row r at position k ^ (r % 8)), staged two at a time in the warp's 8 KB and
+        // added into C by the TMA unit.
+        static_assert(LAYOUT == PURO_WGRAD && WCOLS == 128, "FP32 accumulation is the wgrad epilogue");
+        const int g = lane >> 2, c = 2 * (lane & 3);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1) {
+            if (lane == 0) bulk_wait_group_read<0>();  // the first two boxes left the buffer
+            __syncwarp();
+          }
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int p = 4 * (2 * h + bb) + q;  // acc pair: columns 8p + c, 8p + c + 1
+                const int r = g + 8 * x;
+                const int k16 = 2 * q + (c >> 2);
+                const uint32_t addr = stg + bb * STG_BOX_BYTES + r * 128 + ((k16 ^ (r & 7)) << 4) + 4 * (c & 3);
+                float lo, hi;
+                unpack2(acc[16 * x + p], lo, hi);
+                asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(lo), "f"(hi) : "memory");
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int row0 = mt * BM + quad * 32;
+            if (row0 < args.M) {
+#pragma unroll
+              for (int bb = 0; bb < 2; ++bb) {
+                const int col = n_base + 32 * (2 * h + bb);
+                if (col < args.N) tma_reduce_add_2d(&tmC, stg + bb * STG_BOX_BYTES, col, row0);
+              }
+            }
+            bulk_commit_group();
+          }
+        }
+      } else {
       if constexpr (LAYOUT != PURO_WGRAD) {
         // thread = row `lane`, columns in order
 #pragma unroll
@@ -515,6 +560,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         bulk_commit_group();
       }
+      }  // BF16 store
     }
     if (lane == 0) bulk_wait_group_all();  // stores complete before the CTA exits
     if (!ok) raise_abort(abort, args.status);
@@ -579,9 +625,9 @@ int *device_status_ptr() {
   return p;
 }
 
-template <int LAYOUT>
-int launch_layout(const uint8_t *Aq, const uint8_t *Bq, uint16_t *Cout,
-                  GemmArgs args, int sms, cudaStream_t stream) {
+template <int LAYOUT, bool ACC32>
+int launch_layout(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
+                  cudaStream_t stream) {
   constexpr int TN = TileFor<LAYOUT>::TN;
   constexpr int SMEM_BYTES = Cfg<LAYOUT, TN>::SMEM_BYTES;
   const int64_t M = args.M, N = args.N, K = args.K;
@@ -590,14 +636,16 @@ int launch_layout(const uint8_t *Aq, const uint8_t *Bq, uint16_t *Cout,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, TN, BK,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
-                CU_TENSOR_MAP_SWIZZLE_128B))
+      !(ACC32 ? make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, N, 32, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B)
+              : make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
+                         CU_TENSOR_MAP_SWIZZLE_128B)))
     return PURO_ERR_CUDA;
   args.num_m = static_cast<int>((M + BM - 1) / BM);
   args.num_n = static_cast<int>((N + TN - 1) / TN);
   const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  auto kern = k_gemm_blockwise<LAYOUT, TN>;
+  auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32>;
   // The register split inside the kernel assumes exactly LAUNCH_REGS per thread at launch;
   // with any other count the promotion warps' setmaxnreg.inc could wait forever.
   cudaFuncAttributes fa{};
@@ -627,20 +675,20 @@ int launch_layout(const uint8_t *Aq, const uint8_t *Bq, uint16_t *Cout,
 
 }  // namespace
 
-int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs,
-                          uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
-                          cudaStream_t stream) {
-  int dev = 0, sms = 0;
+namespace {
+
+// Kernel arguments common to every launch; returns PURO_OK or an error status.
+int gemm_args(const float *As, const float *Bs, int64_t M, int64_t N, int64_t K, GemmArgs &args,
+              int &sms) {
+  int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return PURO_ERR_CUDA;
   int *status = device_status_ptr();
   if (status == nullptr) return PURO_ERR_CUDA;
-
-  GemmArgs args;
+  args = GemmArgs{};
   args.As = As;
   args.Bs = Bs;
-  args.C = C;
   args.M = static_cast<int>(M);
   args.N = static_cast<int>(N);
   args.K = static_cast<int>(K);
@@ -650,13 +698,33 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
   args.m_fastest = M <= N ? 1 : 0;
   args.timeout_ns = wait_timeout_ns();
   args.status = status;
+  return PURO_OK;
+}
 
+}  // namespace
+
+int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs,
+                          uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
+                          cudaStream_t stream) {
+  GemmArgs args;
+  int sms = 0;
+  if (int e = gemm_args(As, Bs, M, N, K, args, sms)) return e;
+  args.C = C;
   switch (layout) {
-    case PURO_FPROP: return launch_layout<PURO_FPROP>(Aq, Bq, C, args, sms, stream);
-    case PURO_DGRAD: return launch_layout<PURO_DGRAD>(Aq, Bq, C, args, sms, stream);
-    case PURO_WGRAD: return launch_layout<PURO_WGRAD>(Aq, Bq, C, args, sms, stream);
+    case PURO_FPROP: return launch_layout<PURO_FPROP, false>(Aq, Bq, C, args, sms, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD, false>(Aq, Bq, C, args, sms, stream);
+    case PURO_WGRAD: return launch_layout<PURO_WGRAD, false>(Aq, Bq, C, args, sms, stream);
     default: return PURO_ERR_LAYOUT;
   }
+}
+
+int launch_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                              const float *Bs, float *C, int64_t M, int64_t N, int64_t K,
+                              cudaStream_t stream) {
+  GemmArgs args;
+  int sms = 0;
+  if (int e = gemm_args(As, Bs, M, N, K, args, sms)) return e;
+  return launch_layout<PURO_WGRAD, true>(Aq, Bq, C, args, sms, stream);
 }
 
 int read_and_clear_device_status(cudaStream_t stream, int *status_out) {

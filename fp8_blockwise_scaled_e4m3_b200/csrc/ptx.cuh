@@ -98,6 +98,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
                "r"(src), "r"(c0), "r"(c1)
                : "memory");
 }
+// 2-D tiled bulk tensor reduce-add shared -> global: every element of the box inside the
+// tensor is added to its global value (the tensor map's element type, here FP32), once,
+// by the TMA unit; elements outside the tensor are skipped. Bulk async-group completion.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, uint32_t src, int32_t c0,
+                                                  int32_t c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

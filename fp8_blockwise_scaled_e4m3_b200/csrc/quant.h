@@ -24,6 +24,11 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                           uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
                           cudaStream_t stream);
 
+// wgrad with FP32 accumulation: C[M, N] (FP32) += the wgrad product.
+int launch_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                              const float *Bs, float *C, int64_t M, int64_t N, int64_t K,
+                              cudaStream_t stream);
+
 // Reads and clears the device status word of the GEMM kernels (after a stream sync).
 int read_and_clear_device_status(cudaStream_t stream, int *status_out);
 

@@ -39,6 +39,7 @@ def _load():
         "puro_fp8_quantize_128x128": [_p, _i64, _i64, _i64, _p, _p, _p, _p],
         "puro_fp8_gemm_blockwise": [_p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p,
                                     ctypes.c_size_t, _p],
+        "puro_fp8_gemm_wgrad_acc_f32": [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p],
         "puro_fp8_sync_status": [_p],
     }
     for name, args in sig.items():
@@ -140,6 +141,19 @@ def puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, workspace=None, stream=No
         _check(_lib.puro_fp8_gemm_blockwise(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
                                             int(layout), _ptr(workspace), ws_bytes, _stream(stream)),
                "puro_fp8_gemm_blockwise")
+
+
+def puro_fp8_gemm_wgrad_acc_f32(Aq, As, Bq, Bs, C, stream=None):
+    """C (float32 [M, N]) += the wgrad product of the operands (see the C declaration)."""
+    _need(Aq, torch.uint8, "Aq"); _need(Bq, torch.uint8, "Bq"); _need(C, torch.float32, "C")
+    _need(As, torch.float32, "As"); _need(Bs, torch.float32, "Bs")
+    for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C")):
+        _dense(t, n)
+    M, K = Aq.shape
+    N = Bq.shape[0]
+    with torch.cuda.device(Aq.device):
+        _check(_lib.puro_fp8_gemm_wgrad_acc_f32(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
+                                                _stream(stream)), "puro_fp8_gemm_wgrad_acc_f32")
 
 
 def puro_fp8_sync_status(stream=None):

@@ -139,6 +139,27 @@ PURO_API int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const u
                             puro_stream_t stream);
 
 /*
+ * Weight gradient with FP32 accumulation:
+ *     C[m, n] += sum_kb sA(kb, m) * sB(kb, n) * sum_{k in kb} A[m, k] B[n, k]
+ * the PURO_WGRAD product of puro_fp8_gemm_blockwise (same operands, same FP32 promotion),
+ * added into an FP32 main-gradient buffer instead of written as BF16. Source: "Lever 2: use
+ * blockwise FP8 from step zero" (master weights and gradients stay in BF16/FP32; FP8 is the
+ * compute format of the GEMMs only): each micro-step's FP8 weight gradient is accumulated
+ * at FP32.
+ *
+ *   Aq  [M, K] E4M3 codes = dY^T quantised 1x128 along the tokens, As [K/128, M]
+ *   Bq  [N, K] E4M3 codes = X^T quantised 1x128 along the tokens,  Bs [K/128, N]
+ *   C   [M, N] FP32, dense, read and written: every element gets exactly one FP32 add
+ *       (round to nearest) of its FP32 product per call, done by the TMA unit at L2.
+ * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, Bq, C 16-byte aligned,
+ * As, Bs 4-byte aligned. Calls that add into the same C must not overlap on the GPU.
+ * Status codes as for puro_fp8_gemm_blockwise.
+ */
+PURO_API int puro_fp8_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                                         const float *Bs, float *C, int64_t M, int64_t N,
+                                         int64_t K, puro_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that kernels
  * set when a bounded wait gives up. Returns PURO_OK, PURO_ERR_TIMEOUT, or
  * PURO_ERR_CUDA if the synchronisation itself reported an error.

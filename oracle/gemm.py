@@ -75,6 +75,14 @@ def gemm_ref_rows(aq, a_s, bq, b_s, layout: str, rows) -> np.ndarray:
     return a_rows @ b.T
 
 
+def wgrad_accumulate_ref(c_in, aq, a_s, bq, b_s) -> np.ndarray:
+    """FP32 main-gradient accumulation of a weight gradient: C_in + dW, with dW the wgrad
+    contraction above (the pages keep master weights in BF16/FP32; accumulating each
+    micro-step's dW into an FP32 buffer is the plain reading of that). float64 result; the
+    GPU's FP32 add rounds it once."""
+    return np.asarray(c_in, dtype=np.float64) + gemm_ref(aq, a_s, bq, b_s, "wgrad")
+
+
 def row_col_norms(aq, a_s, bq, b_s, layout: str, rows=None):
     """||A_deq[m, :]||_2 and ||B_deq[n, :]||_2, for the elementwise error bound."""
     if rows is None:

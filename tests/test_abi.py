@@ -41,12 +41,10 @@ def exported_symbols(path):
 
 
 def test_header_declares_the_entry_points():
-    names = declared_functions()
-    assert names == sorted([
+    assert declared_functions() == sorted([
         "puro_fp8_quantize_1x128", "puro_fp8_quantize_1x128_transposed", "puro_fp8_quantize_128x128",
-        "puro_fp8_gemm_blockwise", "puro_fp8_sync_status", "puro_strerror"]) or set(names) >= {
-        "puro_fp8_quantize_1x128", "puro_fp8_quantize_1x128_transposed", "puro_fp8_quantize_128x128",
-        "puro_fp8_gemm_blockwise", "puro_fp8_sync_status", "puro_strerror"}
+        "puro_fp8_gemm_blockwise", "puro_fp8_gemm_wgrad_acc_f32", "puro_fp8_sync_status",
+        "puro_strerror"])
 
 
 def test_library_exports_exactly_the_declared_symbols(lib):
@@ -107,3 +105,13 @@ def test_gemm_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
 def test_without_gpu_calls_report_cuda_error(lib):
     assert lib.puro_fp8_sync_status(None) == ECUDA
+
+
+def test_wgrad_acc_f32_rejects_bad_arguments(lib):
+    f = lib.puro_fp8_gemm_wgrad_acc_f32
+    args = [A16, A16, A16, A16, A16]
+    assert f(None, *args[1:], 128, 256, 256, None) == ENULL
+    assert f(*args, 0, 256, 256, None) == ESHAPE
+    assert f(*args, 128, 250, 256, None) == ESHAPE       # N % 8
+    assert f(*args, 128, 256, 200, None) == ESHAPE       # K % 128
+    assert f(*args[:4], A16 + 4, 128, 256, 256, None) == EALIGN   # C not 16-byte aligned

@@ -140,3 +140,80 @@ def test_lm_head_full_size_sampled(pf, tokens):
 
 def test_status_clean_after_parity_runs(pf):
     pf.puro_fp8_sync_status()
+
+
+# ------------------------------------------------------------------ FP32 wgrad accumulation
+
+def _exact_integer_operands(layout, m, n, k, seed):
+    """Codes in {0, +-0.5, +-1, +-2} and power-of-two scales (as in the exact-integer case
+    above): with K <= 1024 every FP32 partial, product and sum is exact."""
+    rng = np.random.default_rng(seed)
+    codes = np.array([0x00, 0x30, 0xB0, 0x38, 0xB8, 0x40, 0xC0], dtype=np.uint8)
+    aq = codes[rng.integers(0, 7, size=(m, k))]
+    bq = codes[rng.integers(0, 7, size=(n, k))]
+    a_s = (2.0 ** rng.integers(-3, 3, size=(k // 128, m))).astype(np.float32)
+    b_s = (2.0 ** rng.integers(-3, 3, size=_b_scale_shape(layout, n, k))).astype(np.float32)
+    return aq, a_s, bq, b_s
+
+
+# puro_fp8_gemm_wgrad_acc_f32: C (FP32) += the wgrad product, one FP32 add per element.
+
+@pytest.mark.parametrize("m,n,k", [(128, 256, 128), (200, 264, 384), (1, 8, 128), (300, 520, 1024)])
+def test_wgrad_acc_f32_exact_integer_bitexact(pf, m, n, k):
+    aq, a_s, bq, b_s = _exact_integer_operands("wgrad", m, n, k, 5 * m + n + k)
+    rng = np.random.default_rng(m * n)
+    c_in = rng.integers(-4096, 4096, size=(m, n)).astype(np.float32) / 4   # exact with the sums
+    dw = ogemm.gemm_ref(aq, a_s, bq, b_s, "wgrad")
+    c = torch.from_numpy(c_in).to(DEV)
+    ops = _to_dev(aq, a_s, bq, b_s)
+    pf.puro_fp8_gemm_wgrad_acc_f32(*ops, c)
+    once = c.cpu().numpy().astype(np.float64)
+    want = ogemm.wgrad_accumulate_ref(c_in, aq, a_s, bq, b_s)
+    assert np.array_equal(want, want.astype(np.float32).astype(np.float64))
+    mism = np.argwhere(once != want)
+    assert mism.size == 0, f"{len(mism)} mismatches, first at {mism[:4].tolist()}"
+    pf.puro_fp8_gemm_wgrad_acc_f32(*ops, c)      # accumulating again adds dW once more
+    assert np.array_equal(c.cpu().numpy().astype(np.float64), c_in + 2 * dw)
+
+
+def test_wgrad_acc_f32_random_codes_tolerance(pf):
+    m, n, k = 520, 776, 1280
+    rng = np.random.default_rng(17)
+    aq = rng.integers(0, 256, size=(m, k)).astype(np.uint8)
+    bq = rng.integers(0, 256, size=(n, k)).astype(np.uint8)
+    aq[(aq & 0x7F) == 0x7F] = 0x38
+    bq[(bq & 0x7F) == 0x7F] = 0xB8
+    a_s = (rng.random((k // 128, m)) * 2.0 ** -6).astype(np.float32)
+    b_s = (rng.random((k // 128, n)) * 2.0 ** -6).astype(np.float32)
+    ref = ogemm.gemm_ref(aq, a_s, bq, b_s, "wgrad")
+    c_in = (rng.standard_normal((m, n)) * np.abs(ref).mean()).astype(np.float32)
+    c = torch.from_numpy(c_in).to(DEV)
+    pf.puro_fp8_gemm_wgrad_acc_f32(*_to_dev(aq, a_s, bq, b_s), c)
+    got = c.cpu().numpy().astype(np.float64)
+    an, bn = ogemm.row_col_norms(aq, a_s, bq, b_s, "wgrad")
+    # the added product meets the GEMM tolerance; the final FP32 add rounds once more
+    check_gemm(got - c_in.astype(np.float64), ref, an, bn, "wgrad acc f32",
+               extra_abs=np.abs(c_in.astype(np.float64) + ref) * 2.0 ** -23)
+    assert np.allclose(got, ogemm.wgrad_accumulate_ref(c_in, aq, a_s, bq, b_s), rtol=0,
+                       atol=float((1e-2 * an[:, None] * bn[None, :]).max()))
+
+
+def test_wgrad_acc_f32_layer_full_size_sampled(pf):
+    """gate/up weight gradient of a Qwen3-1.7B-shaped layer at 4096 tokens, from the
+    workload's BF16 tensors through the library's quantisers, accumulated onto a nonzero
+    FP32 main gradient; sampled against the oracle."""
+    T = 4096
+    (name, x, w) = wl.layer_forward(1, T, DEV)[2]
+    (_, dy) = wl.layer_grads(2, T, DEV)[2]
+    dyt, dyst = pf.quantize_1x128_transposed(dy)
+    xt, xst = pf.quantize_1x128_transposed(x)
+    n_out, k_in = w.shape
+    main = torch.randn(n_out, k_in, device=DEV) * 1e-3
+    start = main.clone()
+    pf.puro_fp8_gemm_wgrad_acc_f32(dyt, dyst, xt, xst, main)
+    rows, nblocks = _sample(n_out, 48, 4), _sample(k_in // 128, 2, 5)
+    c_ref, cols, an, bn = oracle_gemm_sampled("wgrad", dy, x, rows, nblocks)
+    ri, ci = torch.as_tensor(rows, device=DEV), torch.as_tensor(cols, device=DEV)
+    added = (main[ri][:, ci].double() - start[ri][:, ci].double()).cpu().numpy()
+    check_gemm(added, c_ref, an, bn, f"{name} wgrad acc f32",
+               extra_abs=np.abs(start[ri][:, ci].double().cpu().numpy() + c_ref) * 2.0 ** -23)

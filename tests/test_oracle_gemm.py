@@ -139,3 +139,29 @@ def test_blockwise_beats_per_tensor_on_outlier_channels():
     err_t = np.linalg.norm(per_tensor - exact) / np.linalg.norm(exact)
     assert err_b < err_t
     assert err_b < 0.05
+
+
+def test_wgrad_accumulate_is_input_plus_contraction():
+    """The accumulation reference adds the wgrad contraction to the given buffer: zero
+    input gives the contraction itself, and accumulating twice equals adding 2 dW (exact
+    here: integer-valued operands)."""
+    rng = np.random.default_rng(5)
+    codes = np.array([0x00, 0x38, 0xB8, 0x40, 0xC0], dtype=np.uint8)   # 0, +-1, +-2
+    m, n, k = 40, 24, 256
+    aq = codes[rng.integers(0, 5, size=(m, k))]
+    bq = codes[rng.integers(0, 5, size=(n, k))]
+    a_s = np.ones((k // 128, m), np.float32)
+    b_s = np.full((k // 128, n), 2.0, np.float32)
+    dw = gemm.gemm_ref(aq, a_s, bq, b_s, "wgrad")
+    assert np.array_equal(gemm.wgrad_accumulate_ref(np.zeros((m, n), np.float32), aq, a_s, bq, b_s), dw)
+    c0 = rng.integers(-1000, 1000, size=(m, n)).astype(np.float32)
+    once = gemm.wgrad_accumulate_ref(c0, aq, a_s, bq, b_s)
+    twice = gemm.wgrad_accumulate_ref(once, aq, a_s, bq, b_s)
+    assert np.array_equal(twice, c0 + 2 * dw)
+    # brute force on a tiny case: dW[m, n] = sum_t dY[t, m] X[t, n] with the token scales
+    brute = np.zeros((m, n))
+    dec = e4m3.decode(aq) * np.repeat(a_s.T, 128, axis=1), e4m3.decode(bq) * np.repeat(b_s.T, 128, axis=1)
+    for i in range(m):
+        for j in range(n):
+            brute[i, j] = float(np.dot(dec[0][i], dec[1][j]))
+    assert np.array_equal(once, c0 + brute)
