@@ -195,6 +195,7 @@ class Step:
                     dyqt=e(n, T), dyst=e(T // 128, n, dt=f32),
                     xqt=e(k, T), xst=e(T // 128, k, dt=f32),
                     y=e(T, n, dt=bf), dx=e(T, k, dt=bf), dw=e(n, k, dt=bf))
+        self.side = torch.cuda.Stream(device=device)  # weight quantisers and wgrad (overlap mode)
         self.gemm_flops = sum(3 * 2 * T * lin[2].shape[0] * lin[2].shape[1] for lin in self.linears)
         # algorithmic quantiser bytes: BF16 read + code writes + FP32 scale writes
         qb = 0
@@ -217,33 +218,73 @@ class Step:
         self.quant_launches = 4 * len(self.linears)
         self.launches_per_step = 7 * len(self.linears)
 
-    def run(self, ev=None, stream=None, after_wgrad=None, before_fwd=None, before_bwd=None):
-        """Enqueue one step. ev: list to which (kind, event) pairs are appended after
-        each launch (an initial event must already be recorded). before_fwd(i) /
-        before_bwd(i) are called before linear i's forward / backward launches are
-        enqueued; after_wgrad(i, dW) right after its wgrad (the dW buffer is reused by the
-        next linear of the same shape)."""
-        pf = self.pf
-        rec = (lambda kind: ev.append((kind, _record(self.torch)))) if ev is not None else (lambda kind: None)
+    def run(self, ev=None, stream=None, overlap=False, before_fwd=None, before_bwd=None,
+            before_wgrad=None, after_wgrad=None):
+        """Enqueue one step on `stream` (default: the current one).
+
+        Order: every weight is quantised first (weights are known before the forward),
+        then the forward sweep (quantise X, fprop) and the backward sweep (quantise dY with
+        both outputs, quantise X along tokens, dgrad, wgrad). With overlap=True the weight
+        quantisers and the wgrads run on a second stream: in a backward pass only dgrad
+        feeds the next layer, so wgrad is off the critical path and its kernels fill the
+        SMs the other stream's kernels leave idle. Events order every producer before its
+        consumers and every reuse of a per-shape scratch buffer after its last reader.
+
+        ev: list to which (kind, event) pairs are appended after each launch (serial mode
+        only; an initial event must already be recorded). Hooks, each given the stream its
+        next launch goes to: before_fwd(i, st) before linear i's inputs are first read
+        (weight quantiser and forward), before_bwd(i, st) before its dY is first read,
+        before_wgrad(i, st) before its wgrad writes the shared dW buffer, after_wgrad(i,
+        dW, st) right after that wgrad is enqueued."""
+        torch, pf = self.torch, self.pf
+        if overlap and ev is not None:
+            raise ValueError("per-launch events need the serial order")
+        main = stream if stream is not None else torch.cuda.current_stream()
+        side = self.side if overlap else main
+        rec = (lambda kind: ev.append((kind, _record(torch)))) if ev is not None else (lambda kind: None)
+        if overlap:
+            side.wait_stream(main)  # the previous step is done with every buffer
+        w_ready = []
+        with torch.cuda.stream(side):
+            for i, (tag, x, w, dy, wq, wqt, ws) in enumerate(self.linears):
+                if before_fwd is not None:
+                    before_fwd(i, side)
+                pf.puro_fp8_quantize_128x128(w, wq, wqt, ws, side); rec("q")
+                w_ready.append(side.record_event() if overlap else None)
         for i, (tag, x, w, dy, wq, wqt, ws) in enumerate(self.linears):
-            if before_fwd is not None:
-                before_fwd(i)
+            if before_fwd is not None and overlap:
+                before_fwd(i, main)
             s = self.scratch[tuple(w.shape)]
-            pf.puro_fp8_quantize_1x128(x, s["xq"], s["xs"], stream); rec("q")
-            pf.puro_fp8_quantize_128x128(w, wq, wqt, ws, stream); rec("q")
-            pf.puro_fp8_gemm_blockwise(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, None, stream); rec("g")
+            pf.puro_fp8_quantize_1x128(x, s["xq"], s["xs"], main); rec("q")
+            if overlap:
+                main.wait_event(w_ready[i])
+            pf.puro_fp8_gemm_blockwise(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, None, main); rec("g")
+        wgrad_done = {}  # per shape: the last wgrad that read the shape's token-dim operands
         for i in range(len(self.linears) - 1, -1, -1):
             tag, x, w, dy, wq, wqt, ws = self.linears[i]
+            key = tuple(w.shape)
+            s = self.scratch[key]
             if before_bwd is not None:
-                before_bwd(i)
-            s = self.scratch[tuple(w.shape)]
-            pf.puro_fp8_quantize_1x128_transposed(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], stream); rec("q")
-            pf.puro_fp8_quantize_1x128_transposed(x, s["xqt"], s["xst"], None, None, stream); rec("q")
-            pf.puro_fp8_gemm_blockwise(s["dyq"], s["dys"], wqt, ws, s["dx"], pf.PURO_DGRAD, None, stream); rec("g")
-            pf.puro_fp8_gemm_blockwise(s["dyqt"], s["dyst"], s["xqt"], s["xst"], s["dw"], pf.PURO_WGRAD, None,
-                                       stream); rec("g")
-            if after_wgrad is not None:
-                after_wgrad(i, s["dw"])
+                before_bwd(i, main)
+            if overlap and key in wgrad_done:
+                main.wait_event(wgrad_done[key])  # the quantisers below overwrite its operands
+            pf.puro_fp8_quantize_1x128_transposed(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], main); rec("q")
+            pf.puro_fp8_quantize_1x128_transposed(x, s["xqt"], s["xst"], None, None, main); rec("q")
+            q_ready = main.record_event() if overlap else None
+            pf.puro_fp8_gemm_blockwise(s["dyq"], s["dys"], wqt, ws, s["dx"], pf.PURO_DGRAD, None, main); rec("g")
+            if overlap:
+                side.wait_event(q_ready)
+            if before_wgrad is not None:
+                before_wgrad(i, side)
+            with torch.cuda.stream(side):
+                pf.puro_fp8_gemm_blockwise(s["dyqt"], s["dyst"], s["xqt"], s["xst"], s["dw"], pf.PURO_WGRAD, None,
+                                           side); rec("g")
+                if after_wgrad is not None:
+                    after_wgrad(i, s["dw"], side)
+            if overlap:
+                wgrad_done[key] = side.record_event()
+        if overlap:
+            main.wait_stream(side)
 
 
 def _record(torch):
@@ -370,7 +411,7 @@ def run_ours(args):
     clocks = Clocks(torch.cuda.current_device())
     clocks.start()  # sampling starts before the warm-up; only the timed region is kept
     for _ in range(args.warmup):
-        step.run(stream=stream)
+        step.run(stream=stream, overlap=True)
     pf.puro_fp8_sync_status()
     _barrier_sync(world)
 
@@ -379,7 +420,7 @@ def run_ours(args):
     t_begin = time.time()
     start = _record(torch)
     for _ in range(args.steps):
-        step.run(stream=stream)
+        step.run(stream=stream, overlap=True)
     end = _record(torch)
     end.synchronize()
     _barrier_sync(world)
@@ -493,19 +534,19 @@ def run_e2e(step, torch, pf, args, world):
                 bwd_ready[i] = h2d_s.record_event()
         read_back = {}  # per dW buffer: the read-back that must finish before it is reused
 
-        def before_bwd(i):
-            comp.wait_event(bwd_ready[i])
+        def before_wgrad(i, st):
             prev = read_back.get(tuple(step.linears[i][2].shape))
             if prev is not None:
-                comp.wait_event(prev)
+                st.wait_event(prev)
 
-        def after_wgrad(i, dw):
-            d2h_s.wait_event(comp.record_event())
+        def after_wgrad(i, dw, st):
+            d2h_s.wait_event(st.record_event())
             with torch.cuda.stream(d2h_s):
                 host_dw[i].copy_(dw, non_blocking=True)
             read_back[tuple(dw.shape)] = d2h_s.record_event()
 
-        step.run(stream=comp, before_fwd=lambda i: comp.wait_event(fwd_ready[i]), before_bwd=before_bwd,
+        step.run(stream=comp, overlap=True, before_fwd=lambda i, st: st.wait_event(fwd_ready[i]),
+                 before_bwd=lambda i, st: st.wait_event(bwd_ready[i]), before_wgrad=before_wgrad,
                  after_wgrad=after_wgrad)
         comp.wait_stream(d2h_s)
 
