@@ -4,12 +4,13 @@
 One step = every quantise and GEMM call of one training micro-step of a
 Qwen3-1.7B-shaped model with an untied LM head (28 blocks of QKV, O, gate/up and down
 linears plus the 151936-wide head) over one micro-batch of 2 x 4096 = 8192 tokens:
-  forward sweep  (blocks 0..27, head):  quantise X (1x128), quantise W (128x128, with
-                                        the transposed codes), fprop GEMM
-  backward sweep (head, blocks 27..0):  quantise dY (1x128 along tokens + row-wise, one
-                                        read), quantise X along tokens, dgrad and wgrad
-That is 7 launches per linear, 791 per step, 84.56 TFLOP of GEMM work (2MNK, i.e.
-6 x linear parameters x tokens) and 48.2 GB of quantiser traffic. Inputs are seeded
+  weights:        quantise every W (128x128, with the transposed codes)
+  forward sweep  (blocks 0..27, head):  quantise X (1x128 row-wise for fprop and along
+                                        the tokens for wgrad, one read), fprop GEMM
+  backward sweep (head, blocks 27..0):  quantise dY (row-wise + along the tokens, one
+                                        read), dgrad and wgrad
+That is 6 launches per linear, 678 per step, 84.56 TFLOP of GEMM work (2MNK, i.e.
+6 x linear parameters x tokens) and 42.5 GB of quantiser traffic. Inputs are seeded
 synthetic BF16 tensors resident in HBM (about 21 GB, distinct per block, so every step
 reads far more than the 126 MB L2).
 
@@ -170,7 +171,7 @@ class Step:
         self.pf, self.torch = pf, torch
         T = tokens
         self.tokens = T
-        self.linears = []  # (tag, X, W, dY, wq, wqt, ws) in forward order
+        self.linears = []  # (tag, X, W, dY, wq, wqt, ws, xqt, xst) in forward order
         for l in range(layers):
             fwd = wl.layer_forward(seed, T, device, layer=l)
             grads = wl.layer_grads(seed, T, device, layer=l)
@@ -186,14 +187,16 @@ class Step:
             n, k = w.shape
             lin += [torch.empty((n, k), dtype=u8, device=device),           # Wq
                     torch.empty((k, n), dtype=u8, device=device),           # WqT
-                    torch.empty(((n + 127) // 128, k // 128), dtype=f32, device=device)]  # Ws
+                    torch.empty(((n + 127) // 128, k // 128), dtype=f32, device=device),  # Ws
+                    # X's codes along the tokens, made in the forward, used by wgrad
+                    torch.empty((k, T), dtype=u8, device=device),           # XqT
+                    torch.empty((T // 128, k), dtype=f32, device=device)]   # XsT
             if (n, k) not in self.scratch:
                 e = lambda *s, dt=u8: torch.empty(s, dtype=dt, device=device)
                 self.scratch[(n, k)] = dict(
                     xq=e(T, k), xs=e(k // 128, T, dt=f32),
                     dyq=e(T, n), dys=e(n // 128, T, dt=f32),
                     dyqt=e(n, T), dyst=e(T // 128, n, dt=f32),
-                    xqt=e(k, T), xst=e(T // 128, k, dt=f32),
                     y=e(T, n, dt=bf), dx=e(T, k, dt=bf), dw=e(n, k, dt=bf))
         self.side = torch.cuda.Stream(device=device)  # weight quantisers and wgrad (overlap mode)
         self.gemm_flops = sum(3 * 2 * T * lin[2].shape[0] * lin[2].shape[1] for lin in self.linears)
@@ -201,10 +204,9 @@ class Step:
         qb = 0
         for _, x, w, dy, *_ in self.linears:
             n, k = w.shape
-            qb += T * k * (2 + 1) + 4 * T * (k // 128)                  # X row-wise
+            qb += T * k * (2 + 2) + 4 * (T * (k // 128) + (T // 128) * k)  # X dual
             qb += n * k * (2 + 2) + 4 * (n // 128) * (k // 128)         # W + WqT
             qb += T * n * (2 + 2) + 4 * (T * (n // 128) + (T // 128) * n)  # dY dual
-            qb += T * k * (2 + 1) + 4 * (T // 128) * k                  # X along tokens
         self.quant_bytes = qb
         # algorithmic GEMM bytes: FP8 operands and FP32 scales read once, BF16 output written
         gb = 0
@@ -215,8 +217,8 @@ class Step:
             gb += n * T + k * T + 4 * (n + k) * (T // 128) + 2 * n * k                      # wgrad
         self.gemm_bytes = gb
         self.gemm_launches = 3 * len(self.linears)
-        self.quant_launches = 4 * len(self.linears)
-        self.launches_per_step = 7 * len(self.linears)
+        self.quant_launches = 3 * len(self.linears)
+        self.launches_per_step = 6 * len(self.linears)
 
     def run(self, ev=None, stream=None, overlap=False, before_fwd=None, before_bwd=None,
             before_wgrad=None, after_wgrad=None):
@@ -246,30 +248,29 @@ class Step:
             side.wait_stream(main)  # the previous step is done with every buffer
         w_ready = []
         with torch.cuda.stream(side):
-            for i, (tag, x, w, dy, wq, wqt, ws) in enumerate(self.linears):
+            for i, (tag, x, w, dy, wq, wqt, ws, xqt, xst) in enumerate(self.linears):
                 if before_fwd is not None:
                     before_fwd(i, side)
                 pf.puro_fp8_quantize_128x128(w, wq, wqt, ws, side); rec("q")
                 w_ready.append(side.record_event() if overlap else None)
-        for i, (tag, x, w, dy, wq, wqt, ws) in enumerate(self.linears):
+        for i, (tag, x, w, dy, wq, wqt, ws, xqt, xst) in enumerate(self.linears):
             if before_fwd is not None and overlap:
                 before_fwd(i, main)
             s = self.scratch[tuple(w.shape)]
-            pf.puro_fp8_quantize_1x128(x, s["xq"], s["xs"], main); rec("q")
+            pf.puro_fp8_quantize_1x128_transposed(x, xqt, xst, s["xq"], s["xs"], main); rec("q")
             if overlap:
                 main.wait_event(w_ready[i])
             pf.puro_fp8_gemm_blockwise(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, None, main); rec("g")
         wgrad_done = {}  # per shape: the last wgrad that read the shape's token-dim operands
         for i in range(len(self.linears) - 1, -1, -1):
-            tag, x, w, dy, wq, wqt, ws = self.linears[i]
+            tag, x, w, dy, wq, wqt, ws, xqt, xst = self.linears[i]
             key = tuple(w.shape)
             s = self.scratch[key]
             if before_bwd is not None:
                 before_bwd(i, main)
             if overlap and key in wgrad_done:
-                main.wait_event(wgrad_done[key])  # the quantisers below overwrite its operands
+                main.wait_event(wgrad_done[key])  # the quantiser below overwrites its dY operands
             pf.puro_fp8_quantize_1x128_transposed(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], main); rec("q")
-            pf.puro_fp8_quantize_1x128_transposed(x, s["xqt"], s["xst"], None, None, main); rec("q")
             q_ready = main.record_event() if overlap else None
             pf.puro_fp8_gemm_blockwise(s["dyq"], s["dys"], wqt, ws, s["dx"], pf.PURO_DGRAD, None, main); rec("g")
             if overlap:
@@ -277,7 +278,7 @@ class Step:
             if before_wgrad is not None:
                 before_wgrad(i, side)
             with torch.cuda.stream(side):
-                pf.puro_fp8_gemm_blockwise(s["dyqt"], s["dyst"], s["xqt"], s["xst"], s["dw"], pf.PURO_WGRAD, None,
+                pf.puro_fp8_gemm_blockwise(s["dyqt"], s["dyst"], xqt, xst, s["dw"], pf.PURO_WGRAD, None,
                                            side); rec("g")
                 if after_wgrad is not None:
                     after_wgrad(i, s["dw"], side)
