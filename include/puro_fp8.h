@@ -12,7 +12,8 @@
  * amax history); a code is E4M3(x / s) with a correctly rounded FP32 division, then
  * round-to-nearest-even saturating to +-448; an all-zero block has s = 0 and signed
  * zero codes. GEMM partial sums are FP32 per 128-wide K block, promoted with the two
- * scales in FP32, output BF16 (round to nearest even).
+ * scales in FP32, output BF16 (round to nearest even), or, for the accumulating weight
+ * gradient, added into an FP32 buffer.
  *
  * Conventions for every entry point:
  *  - Every pointer is a DEVICE pointer to memory the caller owns and allocated; the
