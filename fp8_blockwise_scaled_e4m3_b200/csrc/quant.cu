@@ -84,20 +84,10 @@ __device__ __forceinline__ uint32_t absmax16(const uint4 &v0, const uint4 &v1) {
 __device__ __forceinline__ uint2 codes8(const uint4 &v, const BlockDivider &div) {
   return make_uint2(block_codes4(v.x, v.y, div), block_codes4(v.z, v.w, div));
 }
-
-// Scale of a block with absolute maximum `amax`, and the divider for its codes.
-__device__ __forceinline__ void block_scale(float amax, float &s, BlockDivider &div) {
-  s = scale_of_amax(amax);
-  div = amax > 0.0f ? make_divider(s) : zero_block_divider();
+__device__ __forceinline__ uint2 codes8_fast(const uint4 &v, uint64_t nr2, uint64_t s2) {
+  return make_uint2(block_codes4_fast(v.x, v.y, nr2, s2), block_codes4_fast(v.z, v.w, nr2, s2));
 }
 
-// Packed magnitude maximum over each group of 8 consecutive lanes.
-__device__ __forceinline__ uint32_t lane8_absmax(uint32_t v) {
-  v = bf16x2_absmax(v, __shfl_xor_sync(0xffffffffu, v, 4));
-  v = bf16x2_absmax(v, __shfl_xor_sync(0xffffffffu, v, 2));
-  v = bf16x2_absmax(v, __shfl_xor_sync(0xffffffffu, v, 1));
-  return v;
-}
 
 // The tile in a stage: box b = columns 64b .. 64b+63; row r of a box is 128 bytes with
 // its 16-byte chunk k stored at chunk position k ^ (r % 8).
@@ -127,7 +117,7 @@ __device__ __forceinline__ void read_column_pairs(const uint8_t *stage, uint32_t
 // Codes of the held column pair into the code tile: code-tile row = tile column (128
 // bytes = the 128 tile rows), 16-byte chunk k at position k ^ (row % 8). TG = 16 gives
 // one chunk per column, TG = 32 two.
-template <int TG>
+template <int TG, bool FAST>
 __device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[TG],
                                                      const BlockDivider &div0,
                                                      const BlockDivider &div1, uint8_t *codes) {
@@ -138,10 +128,17 @@ __device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[TG],
 #pragma unroll
   for (int i = 0; i < TG / 4; ++i) {
     // column 2cp is the low half of each word, column 2cp+1 the high half
-    q0[i] = block_codes4(__byte_perm(w[4 * i], w[4 * i + 1], 0x5410),
-                         __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x5410), div0);
-    q1[i] = block_codes4(__byte_perm(w[4 * i], w[4 * i + 1], 0x7632),
-                         __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x7632), div1);
+    const uint32_t a0 = __byte_perm(w[4 * i], w[4 * i + 1], 0x5410);
+    const uint32_t a1 = __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x5410);
+    const uint32_t b0 = __byte_perm(w[4 * i], w[4 * i + 1], 0x7632);
+    const uint32_t b1 = __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x7632);
+    if constexpr (FAST) {
+      q0[i] = block_codes4_fast(a0, a1, pack2(-div0.r, -div0.r), pack2(div0.s, div0.s));
+      q1[i] = block_codes4_fast(b0, b1, pack2(-div1.r, -div1.r), pack2(div1.s, div1.s));
+    } else {
+      q0[i] = block_codes4(a0, a1, div0);
+      q1[i] = block_codes4(b0, b1, div1);
+    }
   }
   const int r0 = 2 * cp, r1 = 2 * cp + 1;
   uint8_t *row0 = codes + r0 * 128;
@@ -250,22 +247,64 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
 
     // ---------------------------------------------------------------- row-wise codes
     if (kRows || kWeight) {
+      // A thread holds 16 columns of NP rows. All NP rows are loaded and their scales
+      // formed before any code, and the codes take the fast path without a branch when
+      // every block the warp holds allows it (the slow path only serves tiny, infinite
+      // or NaN maxima).
+      constexpr int NP = kTile / RSTEP;
+      uint4 v0[NP], v1[NP];
 #pragma unroll
-      for (int p = 0; p < kTile / RSTEP; ++p) {
-        const int r = rg + RSTEP * p;
-        const uint4 v0 = row_chunk(stage, r, 0, j8);
-        const uint4 v1 = row_chunk(stage, r, 1, j8);
-        BlockDivider div = wdiv;
-        float srow = 0.0f;
-        if (kRows) block_scale(bf16x2_absmax_to_f32(lane8_absmax(absmax16(v0, v1))), srow, div);
-        const uint2 q0 = codes8(v0, div);
-        const uint2 q1 = codes8(v1, div);
-        const int64_t row = r0 + r;
+      for (int p = 0; p < NP; ++p) {
+        v0[p] = row_chunk(stage, rg + RSTEP * p, 0, j8);
+        v1[p] = row_chunk(stage, rg + RSTEP * p, 1, j8);
+      }
+      float srow[NP], amax[NP];
+      BlockDivider div[NP];
+      bool ok = true;
+      if (kRows) {
+        uint32_t m[NP];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) m[p] = absmax16(v0[p], v1[p]);
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1)
+#pragma unroll
+          for (int p = 0; p < NP; ++p) m[p] = bf16x2_absmax(m[p], __shfl_xor_sync(0xffffffffu, m[p], o));
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          bool okp;
+          amax[p] = bf16x2_absmax_to_f32(m[p]);
+          block_scale_fast(amax[p], srow[p], div[p], okp);
+          ok = ok && okp;
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) div[p] = wdiv;
+        ok = wdiv.fast;
+      }
+      uint2 q0[NP], q1[NP];
+      if (__all_sync(0xffffffffu, ok)) {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          const uint64_t nr2 = pack2(-div[p].r, -div[p].r), s2 = pack2(div[p].s, div[p].s);
+          q0[p] = codes8_fast(v0[p], nr2, s2);
+          q1[p] = codes8_fast(v1[p], nr2, s2);
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          if (kRows) block_scale(amax[p], srow[p], div[p]);
+          q0[p] = codes8(v0[p], div[p]);
+          q1[p] = codes8(v1[p], div[p]);
+        }
+      }
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const int64_t row = r0 + rg + RSTEP * p;
         if (row < args.R) {  // C is a multiple of 128 in these modes
           uint8_t *qrow = args.q + row * args.ldq + c0 + 8 * j8;
-          *reinterpret_cast<uint2 *>(qrow) = q0;
-          *reinterpret_cast<uint2 *>(qrow + 64) = q1;
-          if (kRows && j8 == 0) args.s[(c0 / kTile) * args.R + row] = srow;
+          *reinterpret_cast<uint2 *>(qrow) = q0[p];
+          *reinterpret_cast<uint2 *>(qrow + 64) = q1[p];
+          if (kRows && j8 == 0) args.s[(c0 / kTile) * args.R + row] = srow[p];
         }
       }
     }
@@ -283,9 +322,12 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
         part[g][2 * cp + 1] = __uint_as_float(m2 & 0x7FFF0000u);
       }
       __syncthreads();  // column partials ready; the code tile is free (thread 0 waited)
+      bool tile_fast = wdiv.fast;
       if (kCols) {
         // The first 64 threads finish the column maxima and form the 128 column scales
-        // and divisors once; every thread then reads the two it needs.
+        // and divisors once; every thread then reads the two it needs. A column off the
+        // fast path stores r = -1, and sends the whole tile to the general code.
+        bool ok = true;
         if (g == 0) {
           float a0 = part[0][2 * cp], a1 = part[0][2 * cp + 1];
 #pragma unroll
@@ -294,21 +336,28 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
             a1 = fmaxf(a1, part[k][2 * cp + 1]);
           }
           float s0, s1;
-          block_scale(a0, s0, d0);
-          block_scale(a1, s1, d1);
-          col_div[2 * cp] = make_float2(d0.s, d0.fast ? d0.r : 0.0f);
-          col_div[2 * cp + 1] = make_float2(d1.s, d1.fast ? d1.r : 0.0f);
+          bool ok0, ok1;
+          block_scale_fast(a0, s0, d0, ok0);
+          block_scale_fast(a1, s1, d1, ok1);
+          if (!ok0) block_scale(a0, s0, d0);
+          if (!ok1) block_scale(a1, s1, d1);
+          ok = ok0 && ok1;
+          col_div[2 * cp] = make_float2(d0.s, d0.fast ? d0.r : -1.0f);
+          col_div[2 * cp + 1] = make_float2(d1.s, d1.fast ? d1.r : -1.0f);
           const int64_t c = c0 + 2 * cp;
           float *strow = args.st + static_cast<int64_t>(tr) * args.C;
           if (c < args.C) strow[c] = s0;
           if (c + 1 < args.C) strow[c + 1] = s1;
         }
-        __syncthreads();
+        tile_fast = __syncthreads_and(ok);
         const float2 e0 = col_div[2 * cp], e1 = col_div[2 * cp + 1];
-        d0 = BlockDivider{e0.x, e0.y, e0.y != 0.0f};
-        d1 = BlockDivider{e1.x, e1.y, e1.y != 0.0f};
+        d0 = BlockDivider{e0.x, e0.y, e0.y >= 0.0f};
+        d1 = BlockDivider{e1.x, e1.y, e1.y >= 0.0f};
       }
-      column_codes_to_smem<TG>(w, d0, d1, codes);
+      if (tile_fast)
+        column_codes_to_smem<TG, true>(w, d0, d1, codes);
+      else
+        column_codes_to_smem<TG, false>(w, d0, d1, codes);
       fence_proxy_async_smem();
     }
     __syncthreads();  // the stage and (if any) the code tile are complete
