@@ -474,7 +474,7 @@ def run_ours(args):
                      "traffic_unit": "DRAM bytes per launch (ncu, one step, mean over launches)",
                      "algorithmic_bytes_per_launch": round(step.gemm_bytes / step.gemm_launches),
                      "launches_measured": n_gemm, "avg_launch_ms": round(t_gemm / max(n_gemm, 1), 4)},
-        "roofline_quant": {"bound": "hbm", "kernel": "quantisers (k_quant_rows/cols/weight)",
+        "roofline_quant": {"bound": "hbm", "kernel": "k_quant_tiles (dual X and dY, 128x128 weight + WqT launches)",
                            "achieved": round(quant_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                            "frac": round(quant_gbs / hbm_gbs, 4),
                            "traffic": ncu_traffic("quant"),
