@@ -34,6 +34,7 @@ import os
 import re
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -110,9 +111,23 @@ class Clocks:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # PURO_CLOCKS_DIR keeps the raw samples; by default they go to a temporary file.
+        keep = os.environ.get("PURO_CLOCKS_DIR")
+        if keep:
+            self.path = os.path.join(keep, f"clocks_gpu{gpu_index}.csv")
+        else:
+            fd, self.path = tempfile.mkstemp(prefix=f"puro_clocks_gpu{gpu_index}_", suffix=".csv")
+            os.close(fd)
+        self.temporary = not keep
         self.proc = None
         self.gpu_index = gpu_index
+
+    def _drop(self):
+        if self.temporary:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
 
     def start(self):
         try:
@@ -129,6 +144,7 @@ class Clocks:
         """Stops sampling; summarises the samples taken between host times t_begin and t_end."""
         import datetime
         if self.proc is None:
+            self._drop()
             return None
         self.proc.terminate()
         try:
@@ -155,6 +171,7 @@ class Clocks:
                 for name, v in zip(names, c[5:9]):
                     if v.lower() == "active":
                         reasons.add(name)
+        self._drop()
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
