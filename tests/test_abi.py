@@ -115,3 +115,27 @@ def test_wgrad_acc_f32_rejects_bad_arguments(lib):
     assert f(*args, 128, 250, 256, None) == ESHAPE       # N % 8
     assert f(*args, 128, 256, 200, None) == ESHAPE       # K % 128
     assert f(*args[:4], A16 + 4, 128, 256, 256, None) == EALIGN   # C not 16-byte aligned
+
+
+def test_empty_and_negative_dimensions_are_shape_errors(lib):
+    """Every entry point rejects zero and negative sizes on the host, before any launch."""
+    q1 = lib.puro_fp8_quantize_1x128
+    assert q1(A16, -4, 128, 128, A16, 128, A16, None) == ESHAPE
+    assert q1(A16, 4, 0, 128, A16, 128, A16, None) == ESHAPE
+    qt = lib.puro_fp8_quantize_1x128_transposed
+    assert qt(A16, 0, 64, 64, A16, A16, None, None, None) == ESHAPE
+    assert qt(A16, -128, 64, 64, A16, A16, None, None, None) == ESHAPE
+    assert qt(A16, 256, 0, 64, A16, A16, None, None, None) == ESHAPE
+    qw = lib.puro_fp8_quantize_128x128
+    assert qw(A16, 0, 256, 256, A16, None, A16, None) == ESHAPE
+    assert qw(A16, -1, 256, 256, A16, None, A16, None) == ESHAPE
+    assert qw(A16, 300, 0, 256, A16, None, A16, None) == ESHAPE
+    g = lib.puro_fp8_gemm_blockwise
+    args = [A16, A16, A16, A16, A16]
+    for layout in (0, 1, 2):
+        assert g(*args, 128, 0, 256, layout, None, 0, None) == ESHAPE
+        assert g(*args, 128, 256, 0, layout, None, 0, None) == ESHAPE
+        assert g(*args, -128, 256, 256, layout, None, 0, None) == ESHAPE
+    acc = lib.puro_fp8_gemm_wgrad_acc_f32
+    assert acc(*args, 128, 0, 256, None) == ESHAPE
+    assert acc(*args, 128, 256, 0, None) == ESHAPE
