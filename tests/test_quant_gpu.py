@@ -120,6 +120,56 @@ def test_128x128_small(pf, R, C, transposed):
         np.testing.assert_array_equal(as_np(wqt), qt_ref)
 
 
+def _slow_and_zero_groups():
+    """BF16 [256, 512]: heavy-tailed, with groups that leave the kernels' fast path (tiny
+    maxima: scales below 2^-90, and below 2^-100 where the scale itself needs IEEE
+    division) or take it with r = 0 (all-zero groups), placed so that a warp or a tile
+    mixes them with ordinary groups.
+
+    Tile (0, 0): column 5 holds BF16 subnormals only, column 6 signed zeros, column 7
+    values scaled by 2^-95; the other columns are ordinary. Tile (0, 1) is all zero, with
+    signed zeros. Tile (1, 2) holds subnormals only. In tile (1, 3), row 140 is scaled by
+    2^-110 while the other rows stay ordinary."""
+    g = torch.Generator().manual_seed(77)
+    x = wl.heavy_tailed((256, 512), 1.0, g, "cpu")
+    x[:128, 5] *= 2.0 ** -130
+    x[:128, 6] = 0.0
+    x[1:128:3, 6] = -0.0
+    x[:128, 7] *= 2.0 ** -95
+    x[:128, 128:256] = 0.0
+    x[:128:5, 128:256] = -0.0
+    x[128:256, 256:384] *= 2.0 ** -130
+    x[140, 384:512] *= 2.0 ** -110
+    return wl.bf16(x)
+
+
+def test_slow_and_zero_groups_in_every_mode(pf):
+    x = _slow_and_zero_groups().to(DEV)
+    bits = host_bits(x)
+    _check_rows(pf, x)
+    qt, st, q, s = pf.quantize_1x128_transposed(x, dual=True)
+    qt_ref, st_ref = oquant.quant_1x128_transposed(bits)
+    q_ref, s_ref = oquant.quant_1x128(bits)
+    np.testing.assert_array_equal(as_np(qt), qt_ref)
+    np.testing.assert_array_equal(as_np(st).view(np.uint32), st_ref.view(np.uint32))
+    np.testing.assert_array_equal(as_np(q), q_ref)
+    np.testing.assert_array_equal(as_np(s).view(np.uint32), s_ref.view(np.uint32))
+    qt2, st2 = pf.quantize_1x128_transposed(x, dual=False)
+    np.testing.assert_array_equal(as_np(qt2), qt_ref)
+    np.testing.assert_array_equal(as_np(st2).view(np.uint32), st_ref.view(np.uint32))
+    wq, wqt, ws = pf.quantize_128x128(x, transposed=True)
+    wq_ref, wqt_ref, ws_ref = oquant.quant_128x128(bits)
+    np.testing.assert_array_equal(as_np(wq), wq_ref)
+    np.testing.assert_array_equal(as_np(wqt), wqt_ref)
+    np.testing.assert_array_equal(as_np(ws).view(np.uint32), ws_ref.view(np.uint32))
+    # the constructed groups are what the docstring says
+    st_np = st_ref.view(np.float32)
+    assert st_np[0, 6] == 0.0 and 0.0 < st_np[0, 5] < 2.0 ** -90 and 0.0 < st_np[0, 7] < 2.0 ** -90
+    assert ws_ref[0, 1] == 0.0 and 0.0 < ws_ref[1, 2] < 2.0 ** -90
+    s_np = s_ref.view(np.float32)
+    assert 0.0 < s_np[3, 140] < 2.0 ** -100 / 448 * 2 and s_np[3, 141] > 2.0 ** -90
+
+
 # ------------------------------------------------------------------ full-size workloads
 
 def _sample(n, k, seed):
