@@ -11,6 +11,12 @@ namespace {
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The kernels walk their tiles with 32-bit indices (tile + grid stays below 2^31).
+bool tiles_fit(int64_t rows, int64_t row_tile, int64_t cols, int64_t col_tile) {
+  const int64_t tr = (rows + row_tile - 1) / row_tile, tc = (cols + col_tile - 1) / col_tile;
+  return tr <= ((1ll << 31) - (1ll << 16)) / tc;
+}
+
 // The kernels are built for sm_100a only: refuse any other device up front.
 int check_device() {
   int dev = 0, major = 0, minor = 0;
@@ -29,7 +35,7 @@ int puro_fp8_quantize_1x128(const uint16_t *X, int64_t R, int64_t C, int64_t ldx
                             int64_t ldq, float *S, puro_stream_t stream) {
   if (X == nullptr || Xq == nullptr || S == nullptr) return PURO_ERR_NULL;
   if (R < 1 || C < 128 || C % 128 != 0 || ldx < C || ldq < C) return PURO_ERR_SHAPE;
-  if (R > (1ll << 31) - 1 || C / 128 > 65535) return PURO_ERR_SHAPE;
+  if (R > (1ll << 31) - 1 || C / 128 > 65535 || !tiles_fit(R, 128, C, 128)) return PURO_ERR_SHAPE;
   if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(S, 4) || ldx % 8 != 0 || ldq % 16 != 0)
     return PURO_ERR_ALIGN;
   if (int d = check_device()) return d;
@@ -43,7 +49,8 @@ int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, int64_t C, 
   if ((Xq == nullptr) != (S == nullptr)) return PURO_ERR_NULL;
   if (T < 128 || T % 128 != 0 || C < 8 || C % 8 != 0 || ldx < C) return PURO_ERR_SHAPE;
   if (Xq != nullptr && C % 128 != 0) return PURO_ERR_SHAPE;
-  if (T / 128 > 65535 || (C + 127) / 128 > (1ll << 31) - 1) return PURO_ERR_SHAPE;
+  if (T / 128 > 65535 || (C + 127) / 128 > (1ll << 31) - 1 || !tiles_fit(T, 128, C, 128))
+    return PURO_ERR_SHAPE;
   if (!aligned(X, 16) || !aligned(XqT, 16) || !aligned(ST, 4) || ldx % 8 != 0)
     return PURO_ERR_ALIGN;
   if (Xq != nullptr && (!aligned(Xq, 16) || !aligned(S, 4))) return PURO_ERR_ALIGN;
@@ -55,7 +62,8 @@ int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t l
                               uint8_t *WqT, float *S, puro_stream_t stream) {
   if (W == nullptr || Wq == nullptr || S == nullptr) return PURO_ERR_NULL;
   if (R < 1 || C < 128 || C % 128 != 0 || ldw < C) return PURO_ERR_SHAPE;
-  if ((R + 127) / 128 > 65535 || C / 128 > (1ll << 31) - 1) return PURO_ERR_SHAPE;
+  if ((R + 127) / 128 > 65535 || C / 128 > (1ll << 31) - 1 || !tiles_fit(R, 128, C, 128))
+    return PURO_ERR_SHAPE;
   if (WqT != nullptr && R % 16 != 0) return PURO_ERR_SHAPE;
   if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(S, 4) || ldw % 8 != 0)
     return PURO_ERR_ALIGN;
@@ -76,6 +84,7 @@ int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *B
   if (M < 1 || N < 8 || N % 8 != 0 || K < 128 || K % 128 != 0) return PURO_ERR_SHAPE;
   // 32-bit tensor-map coordinates and kernel indices
   if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
+  if (!tiles_fit(M, 128, N, 256)) return PURO_ERR_SHAPE;
   if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16) || !aligned(As, 4) ||
       !aligned(Bs, 4))
     return PURO_ERR_ALIGN;
@@ -90,6 +99,7 @@ int puro_fp8_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_
     return PURO_ERR_NULL;
   if (M < 1 || N < 8 || N % 8 != 0 || K < 128 || K % 128 != 0) return PURO_ERR_SHAPE;
   if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
+  if (!tiles_fit(M, 128, N, 256)) return PURO_ERR_SHAPE;
   if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16) || !aligned(As, 4) || !aligned(Bs, 4))
     return PURO_ERR_ALIGN;
   if (int d = check_device()) return d;

@@ -50,7 +50,8 @@ typedef enum {
   PURO_OK = 0,
   PURO_ERR_NULL = -1,      /* a required pointer is NULL                               */
   PURO_ERR_SHAPE = -2,     /* a size is <= 0, a reduction dim is not a multiple of 128,
-                              or a leading dimension is smaller than the row length     */
+                              a leading dimension is smaller than the row length, or
+                              the sizes are too large for 32-bit tile indices           */
   PURO_ERR_ALIGN = -3,     /* a pointer or leading dimension breaks the 16-byte rule    */
   PURO_ERR_LAYOUT = -4,    /* unknown GEMM layout                                       */
   PURO_ERR_LAUNCH = -5,    /* the CUDA launch failed (cudaGetLastError after launch)    */

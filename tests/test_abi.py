@@ -139,3 +139,20 @@ def test_empty_and_negative_dimensions_are_shape_errors(lib):
     acc = lib.puro_fp8_gemm_wgrad_acc_f32
     assert acc(*args, 128, 0, 256, None) == ESHAPE
     assert acc(*args, 128, 256, 0, None) == ESHAPE
+
+
+def test_tile_counts_beyond_32_bit_indices_are_shape_errors(lib):
+    """Sizes that pass every per-dimension bound but whose tile count would overflow the
+    kernels' 32-bit tile indices are rejected on the host."""
+    big = (1 << 31) - 256
+    g = lib.puro_fp8_gemm_blockwise
+    args = [A16, A16, A16, A16, A16]
+    assert g(*args, big, big, 128, 0, None, 0, None) == ESHAPE
+    assert lib.puro_fp8_gemm_wgrad_acc_f32(*args, big, big, 128, None) == ESHAPE
+    q1 = lib.puro_fp8_quantize_1x128
+    c = 65535 * 128
+    assert q1(A16, (1 << 31) - 1, c, c, A16, c, A16, None) == ESHAPE
+    qt = lib.puro_fp8_quantize_1x128_transposed
+    assert qt(A16, 65535 * 128, 1 << 30, 1 << 30, A16, A16, None, None, None) == ESHAPE
+    qw = lib.puro_fp8_quantize_128x128
+    assert qw(A16, 65535 * 128, 1 << 30, 1 << 30, A16, None, A16, None) == ESHAPE
