@@ -1,9 +1,10 @@
 """Python binding of libpuro_fp8.so: argument marshalling only.
 
 Every function with a ``puro_`` name mirrors the C entry point of the same name in
-``include/puro_fp8.h``: it takes torch tensors that already live on the GPU, passes
-their device pointers, sizes and the current CUDA stream, and raises ``PuroError`` on a
-non-zero status. The convenience functions below them allocate the outputs with torch
+``include/puro_fp8.h``: it takes torch tensors that already live on the GPU, checks that
+each has the dtype and exact shape the declaration gives (``ValueError`` otherwise, so a
+kernel never writes past a tensor), passes their device pointers, sizes and the current
+CUDA stream, and raises ``PuroError`` on a non-zero status. The convenience functions below them allocate the outputs with torch
 and call the same entry points. Nothing here computes: every step runs in the CUDA
 kernels, and importing this module fails if the library has not been built.
 """
@@ -94,23 +95,39 @@ def _dense(t, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _shape(t, shape, name):
+    """The kernels write (and read) exactly the extents the C declaration gives; a tensor of
+    any other shape would be overrun or misread, so it is refused here."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _matrix(t, name):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got {t.dim()}-D")
+    return t.shape
+
+
 # ------------------------------------------------------------------ C-ABI mirrors
 
 def puro_fp8_quantize_1x128(X, Xq, S, stream=None):
+    R, C = _matrix(X, "X")
+    _shape(Xq, (R, C), "Xq"); _shape(S, (C // 128, R), "S")
     _need(X, torch.bfloat16, "X"); _need(Xq, torch.uint8, "Xq"); _need(S, torch.float32, "S")
     _dense(S, "S")
-    R, C = X.shape
     with torch.cuda.device(X.device):
         _check(_lib.puro_fp8_quantize_1x128(_ptr(X), R, C, X.stride(0), _ptr(Xq), Xq.stride(0),
                                             _ptr(S), _stream(stream)), "puro_fp8_quantize_1x128")
 
 
 def puro_fp8_quantize_1x128_transposed(X, XqT, ST, Xq=None, S=None, stream=None):
+    T, C = _matrix(X, "X")
+    _shape(XqT, (C, T), "XqT"); _shape(ST, (T // 128, C), "ST")
+    _shape(Xq, (T, C), "Xq"); _shape(S, (C // 128, T), "S")
     _need(X, torch.bfloat16, "X"); _need(XqT, torch.uint8, "XqT"); _need(ST, torch.float32, "ST")
     _need(Xq, torch.uint8, "Xq"); _need(S, torch.float32, "S")
     for t, n in ((XqT, "XqT"), (ST, "ST"), (Xq, "Xq"), (S, "S")):
         _dense(t, n)
-    T, C = X.shape
     with torch.cuda.device(X.device):
         _check(_lib.puro_fp8_quantize_1x128_transposed(_ptr(X), T, C, X.stride(0), _ptr(XqT), _ptr(ST),
                                                        _ptr(Xq), _ptr(S), _stream(stream)),
@@ -118,39 +135,51 @@ def puro_fp8_quantize_1x128_transposed(X, XqT, ST, Xq=None, S=None, stream=None)
 
 
 def puro_fp8_quantize_128x128(W, Wq, WqT, S, stream=None):
+    R, C = _matrix(W, "W")
+    _shape(Wq, (R, C), "Wq"); _shape(WqT, (C, R), "WqT"); _shape(S, ((R + 127) // 128, C // 128), "S")
     _need(W, torch.bfloat16, "W"); _need(Wq, torch.uint8, "Wq"); _need(WqT, torch.uint8, "WqT")
     _need(S, torch.float32, "S")
     for t, n in ((Wq, "Wq"), (WqT, "WqT"), (S, "S")):
         _dense(t, n)
-    R, C = W.shape
     with torch.cuda.device(W.device):
         _check(_lib.puro_fp8_quantize_128x128(_ptr(W), R, C, W.stride(0), _ptr(Wq), _ptr(WqT), _ptr(S),
                                               _stream(stream)), "puro_fp8_quantize_128x128")
 
 
+def _gemm_shapes(Aq, As, Bq, Bs, C, bs_shape):
+    M, K = _matrix(Aq, "Aq")
+    N = _matrix(Bq, "Bq")[0]
+    _shape(Bq, (N, K), "Bq"); _shape(C, (M, N), "C"); _shape(As, (K // 128, M), "As")
+    _shape(Bs, bs_shape(N, K), "Bs")
+    return M, N, K
+
+
 def puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, workspace=None, stream=None):
-    layout = LAYOUTS.get(layout, layout)
+    layout = int(LAYOUTS.get(layout, layout))
+    if layout not in (PURO_FPROP, PURO_DGRAD, PURO_WGRAD):
+        raise ValueError(f"unknown layout {layout}")
+    bs_shape = {PURO_FPROP: lambda n, k: ((n + 127) // 128, k // 128),
+                PURO_DGRAD: lambda n, k: (k // 128, (n + 127) // 128),
+                PURO_WGRAD: lambda n, k: (k // 128, n)}[layout]
+    M, N, K = _gemm_shapes(Aq, As, Bq, Bs, C, bs_shape)
     _need(Aq, torch.uint8, "Aq"); _need(Bq, torch.uint8, "Bq"); _need(C, torch.bfloat16, "C")
     _need(As, torch.float32, "As"); _need(Bs, torch.float32, "Bs")
     for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C")):
         _dense(t, n)
-    M, K = Aq.shape
-    N = Bq.shape[0]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(Aq.device):
         _check(_lib.puro_fp8_gemm_blockwise(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
-                                            int(layout), _ptr(workspace), ws_bytes, _stream(stream)),
+                                            layout, _ptr(workspace), ws_bytes, _stream(stream)),
                "puro_fp8_gemm_blockwise")
 
 
 def puro_fp8_gemm_wgrad_acc_f32(Aq, As, Bq, Bs, C, stream=None):
     """C (float32 [M, N]) += the wgrad product of the operands (see the C declaration)."""
+    M, N, K = _gemm_shapes(Aq, As, Bq, Bs, C, lambda n, k: (k // 128, n))
     _need(Aq, torch.uint8, "Aq"); _need(Bq, torch.uint8, "Bq"); _need(C, torch.float32, "C")
     _need(As, torch.float32, "As"); _need(Bs, torch.float32, "Bs")
     for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C")):
         _dense(t, n)
-    M, K = Aq.shape
-    N = Bq.shape[0]
     with torch.cuda.device(Aq.device):
         _check(_lib.puro_fp8_gemm_wgrad_acc_f32(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
                                                 _stream(stream)), "puro_fp8_gemm_wgrad_acc_f32")

@@ -156,3 +156,40 @@ def test_tile_counts_beyond_32_bit_indices_are_shape_errors(lib):
     assert qt(A16, 65535 * 128, 1 << 30, 1 << 30, A16, A16, None, None, None) == ESHAPE
     qw = lib.puro_fp8_quantize_128x128
     assert qw(A16, 65535 * 128, 1 << 30, 1 << 30, A16, None, A16, None) == ESHAPE
+
+
+def test_binding_refuses_tensors_of_the_wrong_shape(lib):
+    """The Python wrappers check every output and scale tensor against the extents the C
+    declaration gives before anything reaches the device (CPU tensors suffice)."""
+    from fp8_blockwise_scaled_e4m3_b200 import puro_fp8 as pf
+    bf, u8, f32 = torch.bfloat16, torch.uint8, torch.float32
+    z = lambda *s, dt=f32: torch.zeros(s, dtype=dt)
+    X = z(256, 384, dt=bf)
+    cases = [
+        (lambda: pf.puro_fp8_quantize_1x128(X, z(256, 256, dt=u8), z(3, 256)), "Xq"),
+        (lambda: pf.puro_fp8_quantize_1x128(X, z(256, 384, dt=u8), z(256, 3)), "S"),
+        (lambda: pf.puro_fp8_quantize_1x128(z(2, 256, 384, dt=bf), z(256, 384, dt=u8), z(3, 256)), "2-D"),
+        (lambda: pf.puro_fp8_quantize_1x128_transposed(X, z(256, 384, dt=u8), z(2, 384)), "XqT"),
+        (lambda: pf.puro_fp8_quantize_1x128_transposed(X, z(384, 256, dt=u8), z(384, 2)), "ST"),
+        (lambda: pf.puro_fp8_quantize_1x128_transposed(X, z(384, 256, dt=u8), z(2, 384),
+                                                       z(256, 128, dt=u8), z(3, 256)), "Xq"),
+        (lambda: pf.puro_fp8_quantize_128x128(X, z(256, 384, dt=u8), z(256, 384, dt=u8), z(2, 3)), "WqT"),
+        (lambda: pf.puro_fp8_quantize_128x128(X, z(256, 384, dt=u8), None, z(3, 2)), "S"),
+    ]
+    M, N, K = 256, 384, 512
+    Aq, Bq, C = z(M, K, dt=u8), z(N, K, dt=u8), z(M, N, dt=bf)
+    As = z(K // 128, M)
+    cases += [
+        (lambda: pf.puro_fp8_gemm_blockwise(Aq, As, z(N, 256, dt=u8), z(3, 4), C, "fprop"), "Bq"),
+        (lambda: pf.puro_fp8_gemm_blockwise(Aq, As, Bq, z(4, 3), C, "fprop"), "Bs"),
+        (lambda: pf.puro_fp8_gemm_blockwise(Aq, As, Bq, z(3, 4), C, "dgrad"), "Bs"),
+        (lambda: pf.puro_fp8_gemm_blockwise(Aq, As, Bq, z(4, 3), C, "wgrad"), "Bs"),
+        (lambda: pf.puro_fp8_gemm_blockwise(Aq, z(M, K // 128), Bq, z(3, 4), C, "fprop"), "As"),
+        (lambda: pf.puro_fp8_gemm_blockwise(Aq, As, Bq, z(3, 4), z(N, M, dt=bf), "fprop"), "C"),
+        (lambda: pf.puro_fp8_gemm_blockwise(Aq, As, Bq, z(3, 4), C, 7), "layout"),
+        (lambda: pf.puro_fp8_gemm_wgrad_acc_f32(Aq, As, Bq, z(K // 128, N - 8), z(M, N)), "Bs"),
+        (lambda: pf.puro_fp8_gemm_wgrad_acc_f32(Aq, As, Bq, z(K // 128, N), z(M, N - 8)), "C"),
+    ]
+    for call, what in cases:
+        with pytest.raises(ValueError, match=what):
+            call()
