@@ -165,3 +165,37 @@ def test_wgrad_accumulate_is_input_plus_contraction():
         for j in range(n):
             brute[i, j] = float(np.dot(dec[0][i], dec[1][j]))
     assert np.array_equal(once, c0 + brute)
+
+
+def _brute_norm(values):
+    """sqrt of an exactly accumulated sum of squares (Fraction), as a float."""
+    ss = sum((v * v for v in values), Fraction(0))
+    return float(ss) ** 0.5
+
+
+def test_row_col_norms_bruteforce_all_layouts_with_tails():
+    """row_col_norms gives ||A_deq[m, :]||_2 and ||B_deq[n, :]||_2, the factors of the GEMM
+    tolerance's elementwise bound. Brute force: every code decoded from the field formula,
+    times its own scale looked up with the layout's index rule, squared and summed exactly.
+    Scales are random and far from 1 and the scale grids are not square, so squared norms,
+    norms of the raw codes, or the B scales of another layout all fail this."""
+    rng = np.random.default_rng(11)
+    m, n, k = 5, 259, 384   # an M tail, and an N tail that ends a 128-row weight block early
+    for layout in gemm.LAYOUTS:
+        aq, bq = _rand_codes(rng, (m, k)), _rand_codes(rng, (n, k))
+        a_s = _rand_scales(rng, (k // 128, m))
+        b_s = _rand_scales(rng, _b_scale_shape(layout, n, k))
+        an, bn = gemm.row_col_norms(aq, a_s, bq, b_s, layout)
+        assert an.shape == (m,) and bn.shape == (n,)
+        for i in range(m):
+            want = _brute_norm([Fraction(e4m3.decode_code(int(aq[i, kk]))) * Fraction(float(a_s[kk // 128][i]))
+                                for kk in range(k)])
+            assert abs(an[i] - want) <= 1e-12 * want, (layout, "A", i)
+        for j in range(n):
+            want = _brute_norm([Fraction(e4m3.decode_code(int(bq[j, kk])))
+                                * Fraction(float(_b_scale(layout, b_s, j, kk))) for kk in range(k)])
+            assert abs(bn[j] - want) <= 1e-12 * want, (layout, "B", j)
+        # the rows= form (used on sampled full-size outputs) gives the same A norms
+        rows = [4, 0, 2]
+        an_rows, bn_rows = gemm.row_col_norms(aq, a_s, bq, b_s, layout, rows=rows)
+        assert np.array_equal(an_rows, an[rows]) and np.array_equal(bn_rows, bn)
