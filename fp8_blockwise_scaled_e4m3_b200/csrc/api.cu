@@ -107,6 +107,9 @@ int puro_fp8_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_
 }
 
 int puro_fp8_sync_status(puro_stream_t stream) {
+  // The status words are per device and collect timeouts from kernels on every stream:
+  // join the whole device first so that none is missed.
+  if (cudaDeviceSynchronize() != cudaSuccess) return PURO_ERR_CUDA;
   int gemm = 0, quant = 0;
   if (int e = puro::read_and_clear_device_status(stream, &gemm)) return e;
   if (int e = puro::read_and_clear_quant_status(stream, &quant)) return e;

@@ -64,9 +64,20 @@ def strerror(status: int) -> str:
     return _lib.puro_strerror(int(status)).decode()
 
 
-def _check(status: int, where: str):
+# With PURO_CHECK_EACH_CALL=1 every call below is followed by puro_fp8_sync_status(), so a
+# device-side wait that gave up is reported by the call whose kernel gave up (and the call
+# becomes synchronous). Off by default: the calls then stay asynchronous, and a caller that
+# needs valid outputs calls puro_fp8_sync_status() itself after the calls it depends on.
+CHECK_EACH_CALL = os.environ.get("PURO_CHECK_EACH_CALL", "0") == "1"
+
+
+def _check(status: int, where: str, stream=None):
     if status != 0:
         raise PuroError(status, where)
+    if CHECK_EACH_CALL and stream is not None:
+        st = _lib.puro_fp8_sync_status(stream)
+        if st != 0:
+            raise PuroError(st, f"{where} (status after the call)")
 
 
 def _stream(stream):
@@ -116,8 +127,9 @@ def puro_fp8_quantize_1x128(X, Xq, S, stream=None):
     _need(X, torch.bfloat16, "X"); _need(Xq, torch.uint8, "Xq"); _need(S, torch.float32, "S")
     _dense(S, "S")
     with torch.cuda.device(X.device):
+        st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_quantize_1x128(_ptr(X), R, C, X.stride(0), _ptr(Xq), Xq.stride(0),
-                                            _ptr(S), _stream(stream)), "puro_fp8_quantize_1x128")
+                                            _ptr(S), st), "puro_fp8_quantize_1x128", st)
 
 
 def puro_fp8_quantize_1x128_transposed(X, XqT, ST, Xq=None, S=None, stream=None):
@@ -129,9 +141,9 @@ def puro_fp8_quantize_1x128_transposed(X, XqT, ST, Xq=None, S=None, stream=None)
     for t, n in ((XqT, "XqT"), (ST, "ST"), (Xq, "Xq"), (S, "S")):
         _dense(t, n)
     with torch.cuda.device(X.device):
+        st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_quantize_1x128_transposed(_ptr(X), T, C, X.stride(0), _ptr(XqT), _ptr(ST),
-                                                       _ptr(Xq), _ptr(S), _stream(stream)),
-               "puro_fp8_quantize_1x128_transposed")
+                                                       _ptr(Xq), _ptr(S), st), "puro_fp8_quantize_1x128_transposed", st)
 
 
 def puro_fp8_quantize_128x128(W, Wq, WqT, S, stream=None):
@@ -142,8 +154,9 @@ def puro_fp8_quantize_128x128(W, Wq, WqT, S, stream=None):
     for t, n in ((Wq, "Wq"), (WqT, "WqT"), (S, "S")):
         _dense(t, n)
     with torch.cuda.device(W.device):
+        st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_quantize_128x128(_ptr(W), R, C, W.stride(0), _ptr(Wq), _ptr(WqT), _ptr(S),
-                                              _stream(stream)), "puro_fp8_quantize_128x128")
+                                              st), "puro_fp8_quantize_128x128", st)
 
 
 def _gemm_shapes(Aq, As, Bq, Bs, C, bs_shape):
@@ -168,9 +181,9 @@ def puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, workspace=None, stream=No
         _dense(t, n)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(Aq.device):
+        st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_gemm_blockwise(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
-                                            layout, _ptr(workspace), ws_bytes, _stream(stream)),
-               "puro_fp8_gemm_blockwise")
+                                            layout, _ptr(workspace), ws_bytes, st), "puro_fp8_gemm_blockwise", st)
 
 
 def puro_fp8_gemm_wgrad_acc_f32(Aq, As, Bq, Bs, C, stream=None):
@@ -181,8 +194,9 @@ def puro_fp8_gemm_wgrad_acc_f32(Aq, As, Bq, Bs, C, stream=None):
     for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C")):
         _dense(t, n)
     with torch.cuda.device(Aq.device):
+        st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_gemm_wgrad_acc_f32(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
-                                                _stream(stream)), "puro_fp8_gemm_wgrad_acc_f32")
+                                                st), "puro_fp8_gemm_wgrad_acc_f32", st)
 
 
 def puro_fp8_sync_status(stream=None):

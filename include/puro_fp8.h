@@ -3,8 +3,8 @@
  *
  * The method ("Paper walkthrough: Puro-2B -- pretraining a 2B model from scratch for
  * $6.9K on consumer GPUs", section "Lever 2: use blockwise FP8 from step zero"): only
- * the linear-layer GEMMs run in FP8, FP8 is a compute format and not a storage format,
- * and scales are local -- activations and their gradients get one scale per 128
+ * the linear-layer GEMMs run in FP8, tensors are converted to FP8 only for the GEMM that
+ * consumes them, and scales are local -- activations and their gradients get one scale per 128
  * consecutive elements along the reduction dimension, weights one scale per 128x128
  * block. Readings this library takes where the page is silent: the FP8 format is E4M3
  * (bias 7, max 448, no infinities, 0x7F/0xFF NaN); a block's scale is s = amax / 448,
@@ -24,8 +24,14 @@
  *  - Arguments are checked on the host before anything is launched; a failed check
  *    returns a negative puro_status and enqueues nothing.
  *  - Inputs must be finite (no NaN / Inf); this is not checked.
- *  - Calls are stateless and thread-safe; the only global state is the device status
- *    word read by puro_fp8_sync_status().
+ *  - Calls keep no state between them and may be made from several host threads. The
+ *    one piece of global state is a status word per device: any kernel of this library,
+ *    on any stream, sets it when one of its bounded device-side waits gives up (the
+ *    kernel then stops early and leaves its outputs partly written). A call's outputs
+ *    are therefore valid only once a puro_fp8_sync_status() issued after it has
+ *    returned PURO_OK. That function joins the whole device, so it sees timeouts from
+ *    every stream; if several threads call it, the first one after the timeout gets the
+ *    report, because reading the word clears it.
  */
 #ifndef PURO_FP8_H
 #define PURO_FP8_H
@@ -56,7 +62,7 @@ typedef enum {
   PURO_ERR_LAYOUT = -4,    /* unknown GEMM layout                                       */
   PURO_ERR_LAUNCH = -5,    /* the CUDA launch failed (cudaGetLastError after launch)    */
   PURO_ERR_TIMEOUT = -6,   /* a bounded device-side wait gave up (see sync_status)      */
-  PURO_ERR_WORKSPACE = -7, /* workspace too small for the requested split               */
+  PURO_ERR_WORKSPACE = -7, /* reserved; not returned by this version                     */
   PURO_ERR_CUDA = -8,      /* another CUDA runtime / driver call failed                 */
   PURO_ERR_DEVICE = -9     /* the current device is not sm_100 (B200-class)             */
 } puro_status;
@@ -131,7 +137,8 @@ PURO_API int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, 
  *     PURO_DGRAD  dX = dY W:    Bq = WqT, Bs = S of W  [K/128, ceil(N/128)]
  *     PURO_WGRAD  dW = dY^T X:  Bq = XqT, Bs = ST of X [K/128, N]
  *   C   [M, N] BF16, dense            output
- *   workspace, ws_bytes   reserved for split-K; may be NULL / 0.
+ *   workspace, ws_bytes   ignored: no layout of this version needs scratch memory.
+ *                         Pass NULL / 0 (any value is accepted).
  * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, Bq, C 16-byte aligned;
  * As, Bs 4-byte aligned. M and N need not be multiples of the tile size.
  */
@@ -162,8 +169,11 @@ PURO_API int puro_fp8_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, con
                                          int64_t K, puro_stream_t stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device status word that kernels
- * set when a bounded wait gives up. Returns PURO_OK, PURO_ERR_TIMEOUT, or
+ * Waits for all work on the current device (every stream, not only `stream`), then
+ * reads and clears the device's status word, which any kernel of this library sets
+ * when a bounded wait gives up. `stream` carries the two small copies of the word.
+ * Returns PURO_OK (every call enqueued before this one finished and its outputs are
+ * valid), PURO_ERR_TIMEOUT (some kernel gave up; its outputs are partly written), or
  * PURO_ERR_CUDA if the synchronisation itself reported an error.
  */
 PURO_API int puro_fp8_sync_status(puro_stream_t stream);
