@@ -5,6 +5,7 @@
 #include <cstdint>
 
 #include "../../include/puro_fp8.h"
+#include "host_cache.h"
 #include "quant.h"
 
 namespace {
@@ -18,13 +19,20 @@ bool tiles_fit(int64_t rows, int64_t row_tile, int64_t cols, int64_t col_tile) {
 }
 
 // The kernels are built for sm_100a only: refuse any other device up front.
+// (The answer is cached per device.)
 int check_device() {
-  int dev = 0, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PURO_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+  static puro::PerDevice<int> verdict;
+  int v = PURO_ERR_CUDA;
+  if (!verdict.get(v, [](int dev, int &out) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+          return false;
+        out = (major == 10 && minor == 0) ? PURO_OK : PURO_ERR_DEVICE;
+        return true;
+      }))
     return PURO_ERR_CUDA;
-  return (major == 10 && minor == 0) ? PURO_OK : PURO_ERR_DEVICE;
+  return v;
 }
 
 }  // namespace

@@ -40,6 +40,7 @@
 #include <cstdlib>
 
 #include "../../include/puro_fp8.h"
+#include "host_cache.h"
 #include "ptx.cuh"
 #include "quant.h"
 
@@ -120,6 +121,17 @@ struct GemmArgs {
 };
 
 __device__ int g_status;  // non-zero: a bounded wait gave up since the last read
+
+#ifdef PURO_TEST_HOOKS
+// Test builds only, never libpuro_fp8.so: while set, the promotion warps do not hand TMEM
+// buffer 0 back after its first use, so the MMA warp's bounded wait for it runs out. The
+// failure-detection test uses this to check that a give-up inside the GEMM reaches the
+// status word and that the kernel drains and exits with the context intact.
+__device__ int g_test_skip_release;
+#define PURO_SKIP_RELEASE(use) (g_test_skip_release != 0 && (use) == 0)
+#else
+#define PURO_SKIP_RELEASE(use) false
+#endif
 
 __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mt, int &nt) {
   if (a.m_fastest) {
@@ -390,7 +402,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (c == WCOLS / 64 - 1) {
               tc_fence_before_sync();
               __syncwarp();
-              if (lane == 0) mbar_arrive(tempty_bar(b));
+              if (lane == 0 && !PURO_SKIP_RELEASE(use)) mbar_arrive(tempty_bar(b));
             }
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -451,7 +463,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             } else {
               tc_fence_before_sync();
               __syncwarp();
-              if (lane == 0) mbar_arrive(tempty_bar(b));
+              if (lane == 0 && !PURO_SKIP_RELEASE(use)) mbar_arrive(tempty_bar(b));
             }
             apply(q + 1, rb);
             if (q + 2 < 4) tmem_wait_ld_dep(ra);
@@ -610,9 +622,14 @@ unsigned long long wait_timeout_ns() {
   return ns;
 }
 
+// Device address of g_status on the current device (looked up once per device).
 int *device_status_ptr() {
+  static PerDevice<int *> cache;
   int *p = nullptr;
-  if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_status) != cudaSuccess) return nullptr;
+  if (!cache.get(p, [](int, int *&v) {
+        return cudaGetSymbolAddress(reinterpret_cast<void **>(&v), g_status) == cudaSuccess;
+      }))
+    return nullptr;
   return p;
 }
 
@@ -637,23 +654,35 @@ int launch_layout(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs arg
   const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32>;
-  // The register split inside the kernel assumes exactly LAUNCH_REGS per thread at launch;
-  // with any other count the promotion warps' setmaxnreg.inc could wait forever.
-  cudaFuncAttributes fa{};
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PURO_ERR_CUDA;
-  if (fa.numRegs != LAUNCH_REGS || fa.maxThreadsPerBlock < THREADS) {
-    std::fprintf(stderr, "puro_fp8: GEMM kernel built with %d registers (expected %d); not launched\n",
-                 fa.numRegs, LAUNCH_REGS);
-    return PURO_ERR_LAUNCH;
-  }
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e != cudaSuccess) {
-    std::fprintf(stderr, "puro_fp8: cudaFuncSetAttribute: %s\n", cudaGetErrorString(e));
+  // Once per device: the register split inside the kernel assumes exactly LAUNCH_REGS per
+  // thread at launch (with any other count the promotion warps' setmaxnreg.inc could wait
+  // forever), and the kernel needs its dynamic shared memory opted in.
+  static PerDevice<int> prepared;
+  int prep = PURO_ERR_CUDA;
+  if (!prepared.get(prep, [&](int, int &v) {
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+        if (fa.numRegs != LAUNCH_REGS || fa.maxThreadsPerBlock < THREADS) {
+          std::fprintf(stderr, "puro_fp8: GEMM kernel built with %d registers (expected %d); not launched\n",
+                       fa.numRegs, LAUNCH_REGS);
+          v = PURO_ERR_LAUNCH;
+          return true;
+        }
+        const cudaError_t se = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (se != cudaSuccess) {
+          std::fprintf(stderr, "puro_fp8: cudaFuncSetAttribute: %s\n", cudaGetErrorString(se));
+          return false;
+        }
+        v = PURO_OK;
+        return true;
+      }))
     return PURO_ERR_CUDA;
-  }
+  if (prep != PURO_OK) return prep;
   kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, args);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, kern);
     std::fprintf(stderr,
                  "puro_fp8: GEMM launch (grid %d, %d threads, %d B smem): %s "
                  "[kernel: %d regs, max %d threads/block, max dyn smem %d]\n",
@@ -671,10 +700,7 @@ namespace {
 // Kernel arguments common to every launch; returns PURO_OK or an error status.
 int gemm_args(const float *As, const float *Bs, int64_t M, int64_t N, int64_t K, GemmArgs &args,
               int &sms) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return PURO_ERR_CUDA;
+  if (!sm_count(sms)) return PURO_ERR_CUDA;
   int *status = device_status_ptr();
   if (status == nullptr) return PURO_ERR_CUDA;
   args = GemmArgs{};
@@ -732,3 +758,9 @@ int read_and_clear_device_status(cudaStream_t stream, int *status_out) {
 }
 
 }  // namespace puro
+
+#ifdef PURO_TEST_HOOKS
+extern "C" __attribute__((visibility("default"))) int puro_test_set_skip_release(int on) {
+  return cudaMemcpyToSymbol(puro::g_test_skip_release, &on, sizeof(int)) == cudaSuccess ? 0 : -1;
+}
+#endif

@@ -29,6 +29,7 @@
 #include <cstdlib>
 
 #include "../../include/puro_fp8.h"
+#include "host_cache.h"
 #include "ptx.cuh"
 #include "quant.h"
 #include "quant_math.cuh"
@@ -431,11 +432,12 @@ unsigned long long wait_timeout_ns() {
 template <int MODE>
 int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *qt, QArgs args,
                  cudaStream_t stream) {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return PURO_ERR_CUDA;
-  if (cudaGetSymbolAddress(reinterpret_cast<void **>(&args.status), g_quant_status) != cudaSuccess)
+  int sms = 0;
+  if (!sm_count(sms)) return PURO_ERR_CUDA;
+  static PerDevice<int *> status_addr;  // g_quant_status on this device, looked up once
+  if (!status_addr.get(args.status, [](int, int *&v) {
+        return cudaGetSymbolAddress(reinterpret_cast<void **>(&v), g_quant_status) == cudaSuccess;
+      }))
     return PURO_ERR_CUDA;
   CUtensorMap tmX, tmT;
   if (!make_map(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, C, ldx, kTile, 64))
@@ -455,8 +457,13 @@ int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *
   const int64_t tiles = static_cast<int64_t>(args.tiles_r) * args.tiles_c;
   const int grid = static_cast<int>(tiles < kCtasPerSm * sms ? tiles : kCtasPerSm * sms);
   auto kern = k_quant_tiles<MODE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-      cudaSuccess)
+  static PerDevice<bool> smem_opt_in;  // dynamic shared memory opted in once per device
+  bool done = false;
+  if (!smem_opt_in.get(done, [&](int, bool &v) {
+        v = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) ==
+            cudaSuccess;
+        return v;
+      }))
     return PURO_ERR_CUDA;
   kern<<<grid, Threads<MODE>::value, kSmemBytes, stream>>>(tmX, tmT, args);
   const cudaError_t e = cudaGetLastError();
