@@ -57,6 +57,10 @@ def _args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--config", default="5",
+                   help="workload: 1 small outlier GEMM, 2 one layer's forward linears, 3 its backward, "
+                        "4 the LM head, 5 the full 28-layer step (default), or 'all' for 1-4 then 5")
+    p.add_argument("--reps", type=int, default=10, help="timed repetitions of configs 1-4")
     return p.parse_args()
 
 
@@ -587,8 +591,14 @@ def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
-    else:
-        run_ours(args)
+        return
+    if args.config in ("1", "2", "3", "4", "all"):
+        from bench_configs import run_config
+        for c in ((1, 2, 3, 4) if args.config == "all" else (int(args.config),)):
+            run_config(c, args)
+        if args.config != "all":
+            return
+    run_ours(args)
 
 
 if __name__ == "__main__":

@@ -1,0 +1,267 @@
+"""Per-workload measurements of the blockwise-FP8 (E4M3) path, for `bench.py --config 1..4`.
+
+Each workload is one of the five configurations the benchmark is specified on (the fifth,
+the full 28-layer micro-step, is bench.py's default line):
+
+  1  one small GEMM with outlier channels: A [256, 512] (columns 17, 130, 131, 400 x50),
+     W [384, 512]; quantise A (1x128) and W (128x128), then fprop. Latency-bound: the
+     line's value is microseconds for the three launches.
+  2  one Qwen3-1.7B-shaped block's forward linears at 4096 tokens: for QKV, O, gate/up and
+     down, quantise the weight (128x128 with its transposed codes), the input (1x128), fprop.
+  3  the same block's backward: for each linear, quantise dY (row-wise and along the tokens
+     from one read), quantise X along the tokens, dgrad, wgrad (the weight codes of 2 are
+     reused, as in training).
+  4  the untied LM head at 4096 tokens: weight, hidden states (both directions), fprop
+     logits, dlogits (both directions), dgrad, wgrad.
+
+Inputs are the seeded synthetic tensors of `workloads.py` (configuration c uses seed c - 1),
+resident in HBM. Every repetition first writes a 512 MB buffer, so no operand is left in
+the 126 MB L2 from the previous repetition; each launch is bracketed by CUDA events on the
+stream it runs on, and the median over repetitions is reported. The CPU oracle runs the
+same calls (on a bounded sample for the LM head) on the host cores beside it.
+"""
+
+import json
+import statistics
+import time
+
+import torch
+
+from bench import FP8_DENSE_PEAK_TFLOPS, METRIC, Clocks, _cpu_threads, _peaks
+from fp8_blockwise_scaled_e4m3_b200 import puro_fp8 as pf
+from fp8_blockwise_scaled_e4m3_b200 import workloads as wl
+
+NOMINAL_HBM_GBS = 8000.0
+T4096 = 4096
+
+
+def _qbytes_rows(r, c):      # 1x128 row-wise: BF16 read, codes, scales
+    return r * c * 3 + 4 * r * (c // 128)
+
+
+def _qbytes_dual(t, c):      # both directions from one read
+    return t * c * 4 + 4 * (t * (c // 128) + (t // 128) * c)
+
+
+def _qbytes_cols(t, c):      # along the tokens only
+    return t * c * 3 + 4 * (t // 128) * c
+
+
+def _qbytes_weight(n, k, transposed=True):
+    return n * k * (4 if transposed else 3) + 4 * (-(-n // 128)) * (k // 128)
+
+
+class Op:
+    """One library call of a workload: kind 'q' (quantiser) or 'g' (GEMM), its algorithmic
+    bytes or FLOPs, and a closure that enqueues it."""
+
+    def __init__(self, kind, name, work, fn):
+        self.kind, self.name, self.work, self.fn = kind, name, work, fn
+
+
+def _empty(shape, dtype, dev):
+    return torch.empty(shape, dtype=dtype, device=dev)
+
+
+def _weight_ops(name, w, dev, transposed=True):
+    n, k = w.shape
+    wq = _empty((n, k), torch.uint8, dev)
+    wqt = _empty((k, n), torch.uint8, dev) if transposed else None
+    ws = _empty((-(-n // 128), k // 128), torch.float32, dev)
+    op = Op("q", f"{name} W 128x128", _qbytes_weight(n, k, transposed),
+            lambda st: pf.puro_fp8_quantize_128x128(w, wq, wqt, ws, st))
+    return op, (wq, wqt, ws)
+
+
+def _rows_ops(name, x, dev):
+    t, c = x.shape
+    xq, xs = _empty((t, c), torch.uint8, dev), _empty((c // 128, t), torch.float32, dev)
+    op = Op("q", f"{name} 1x128", _qbytes_rows(t, c), lambda st: pf.puro_fp8_quantize_1x128(x, xq, xs, st))
+    return op, (xq, xs)
+
+
+def _cols_ops(name, x, dev, dual):
+    t, c = x.shape
+    qt, st_ = _empty((c, t), torch.uint8, dev), _empty((t // 128, c), torch.float32, dev)
+    q = s = None
+    if dual:
+        q, s = _empty((t, c), torch.uint8, dev), _empty((c // 128, t), torch.float32, dev)
+    op = Op("q", f"{name} {'dual' if dual else 'along tokens'}", _qbytes_dual(t, c) if dual else _qbytes_cols(t, c),
+            lambda st: pf.puro_fp8_quantize_1x128_transposed(x, qt, st_, q, s, st))
+    return op, (qt, st_, q, s)
+
+
+def _gemm_op(name, layout, a, a_s, b, b_s, dev):
+    m, k = a.shape
+    n = b.shape[0]
+    c = _empty((m, n), torch.bfloat16, dev)
+    lay = {"fprop": pf.PURO_FPROP, "dgrad": pf.PURO_DGRAD, "wgrad": pf.PURO_WGRAD}[layout]
+    return Op("g", f"{name} {layout} {m}x{n}x{k}", 2.0 * m * n * k,
+              lambda st: pf.puro_fp8_gemm_blockwise(a, a_s, b, b_s, c, lay, None, st))
+
+
+def build_config(c, dev):
+    """(ops, description) of workload c (1-4), inputs already on `dev`."""
+    ops = []
+    if c == 1:
+        a, w = (t.to(dev) for t in wl.small_gemm(seed=0))
+        qa, (aq, a_s) = _rows_ops("A", a, dev)
+        qw, (wq, _, ws) = _weight_ops("W", w, dev, transposed=False)
+        ops = [qa, qw, _gemm_op("small", "fprop", aq, a_s, wq, ws, dev)]
+        return ops, "small outlier GEMM 256x384x512: quantise A (1x128), W (128x128), fprop; seed 0"
+    if c in (2, 3):
+        fwd = wl.layer_forward(1, T4096, dev)
+        grads = wl.layer_grads(2, T4096, dev)
+        for (name, x, w), (_, dy) in zip(fwd, grads):
+            qw, (wq, wqt, ws) = _weight_ops(name, w, dev)
+            if c == 2:
+                qx, (xq, xs) = _rows_ops(f"{name} X", x, dev)
+                ops += [qw, qx, _gemm_op(name, "fprop", xq, xs, wq, ws, dev)]
+            else:
+                qw.fn(None)  # the weight codes come from the forward; not part of this workload
+                qdy, (dyqt, dyst, dyq, dys) = _cols_ops(f"{name} dY", dy, dev, dual=True)
+                qx, (xqt, xst, _, _) = _cols_ops(f"{name} X", x, dev, dual=False)
+                ops += [qdy, _gemm_op(name, "dgrad", dyq, dys, wqt, ws, dev), qx,
+                        _gemm_op(name, "wgrad", dyqt, dyst, xqt, xst, dev)]
+        what = "forward linears" if c == 2 else "backward (dgrad + wgrad) of the linears"
+        return ops, f"one Qwen3-1.7B-shaped block's {what} at 4096 tokens (QKV, O, gate/up, down); seeds 1, 2"
+    if c == 4:
+        h, w, dl = wl.lm_head(3, T4096, dev)
+        qw, (wq, wqt, ws) = _weight_ops("W_head", w, dev)
+        qh, (hqt, hst, hq, hs) = _cols_ops("H", h, dev, dual=True)
+        qd, (dqt, dst_, dq, ds) = _cols_ops("dlogits", dl, dev, dual=True)
+        ops = [qw, qh, _gemm_op("lm_head", "fprop", hq, hs, wq, ws, dev), qd,
+               _gemm_op("lm_head", "dgrad", dq, ds, wqt, ws, dev),
+               _gemm_op("lm_head", "wgrad", dqt, dst_, hqt, hst, dev)]
+        return ops, "untied LM head 2048 -> 151936 at 4096 tokens: fprop, dgrad, wgrad and their quantisers; seed 3"
+    raise ValueError(c)
+
+
+def oracle_config(c):
+    """Runs workload c's calls in the CPU oracle on the host cores. Returns (GEMM FLOPs of
+    the sample, seconds, sample description)."""
+    import numpy as np
+    from oracle import gemm as og
+    from oracle import quant as oq
+    bits = wl.bf16_bits
+    t0 = time.perf_counter()
+    flops = 0.0
+    if c == 1:
+        a, w = wl.small_gemm(seed=0)
+        aq, a_s = oq.quant_1x128(bits(a))
+        wq, _, ws = oq.quant_128x128(bits(w))
+        og.gemm_ref(aq, a_s, wq, ws, "fprop")
+        flops, sample = 2.0 * 256 * 384 * 512, "the whole workload"
+    elif c in (2, 3):
+        fwd = wl.layer_forward(1, T4096, "cpu")
+        grads = wl.layer_grads(2, T4096, "cpu")
+        t0 = time.perf_counter()  # input generation is not the oracle's work
+        for (name, x, w), (_, dy) in zip(fwd, grads):
+            wq, wqt, ws = oq.quant_128x128(bits(w))
+            n, k = w.shape
+            if c == 2:
+                xq, xs = oq.quant_1x128(bits(x))
+                og.gemm_ref(xq, xs, wq, ws, "fprop")
+                flops += 2.0 * T4096 * n * k
+            else:
+                dyq, dys = oq.quant_1x128(bits(dy))
+                dyt, dyst = oq.quant_1x128_transposed(bits(dy))
+                xt, xst = oq.quant_1x128_transposed(bits(x))
+                og.gemm_ref(dyq, dys, wqt, ws, "dgrad")
+                og.gemm_ref(dyt, dyst, xt, xst, "wgrad")
+                flops += 4.0 * T4096 * n * k
+        sample = "the whole workload"
+    elif c == 4:
+        tok, rows = 512, 74 * 128  # a bounded sample: 512 of 4096 tokens, 74 of 1187 vocabulary blocks
+        h, w, dl = wl.lm_head(3, tok, "cpu")   # timing sample only, not a parity input
+        w, dl = w[:rows], dl[:, :rows].contiguous()
+        t0 = time.perf_counter()
+        wq, wqt, ws = oq.quant_128x128(bits(w))
+        hq, hs = oq.quant_1x128(bits(h))
+        og.gemm_ref(hq, hs, wq, ws, "fprop")
+        dq, ds = oq.quant_1x128(bits(dl))
+        dt_, dst_ = oq.quant_1x128_transposed(bits(dl))
+        ht, hst = oq.quant_1x128_transposed(bits(h))
+        og.gemm_ref(dq, ds, wqt, ws, "dgrad")
+        og.gemm_ref(dt_, dst_, ht, hst, "wgrad")
+        flops = 6.0 * tok * rows * 2048
+        sample = f"{tok} of 4096 tokens x {rows} of 151936 vocabulary rows, all six calls"
+    else:
+        raise ValueError(c)
+    return flops, time.perf_counter() - t0, sample
+
+
+def run_config(c, args):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
+    fp8_burst = 2.0 * bf16_tf   # isolated kernels: the burst figure, x2 for FP8 (nominal ratio)
+    ops, desc = build_config(c, dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 * 2 ** 20 // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    per_op = [[] for _ in ops]
+    whole = []
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()
+    t_begin = None
+    for rep in range(args.warmup + args.reps):
+        if rep == args.warmup:
+            pf.puro_fp8_sync_status()
+            t_begin = time.time()
+        flush.zero_()   # evicts the previous repetition's operands from L2
+        evs = [torch.cuda.Event(enable_timing=True)]
+        evs[0].record(stream)
+        for op in ops:
+            op.fn(stream)
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            evs.append(e)
+        evs[-1].synchronize()
+        if rep >= args.warmup:
+            for i in range(len(ops)):
+                per_op[i].append(evs[i].elapsed_time(evs[i + 1]))
+            whole.append(evs[0].elapsed_time(evs[-1]))
+    clk = clocks.stop(t_begin, time.time())
+    pf.puro_fp8_sync_status()
+    med = [statistics.median(t) for t in per_op]
+    ms_whole = statistics.median(whole)
+    g_flops = sum(op.work for op in ops if op.kind == "g")
+    q_bytes = sum(op.work for op in ops if op.kind == "q")
+    g_ms = sum(m for m, op in zip(med, ops) if op.kind == "g")
+    q_ms = sum(m for m, op in zip(med, ops) if op.kind == "q")
+    g_tf = g_flops / (g_ms * 1e-3) / 1e12
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    line = {"metric": METRIC, "n_gpus": 1, "steps": args.reps, "warmup": args.warmup,
+            "dtype": "e4m3", "data": "synthetic", "scaling": "weak", "vs_baseline": None,
+            "config": {"workload": desc, "config_index": c,
+                       "l2": "flushed before every repetition (512 MB write)"},
+            "ms_per_step": round(ms_whole, 4), "gpu_launches": len(ops) * args.reps, "clocks": clk}
+    if c == 1:
+        line.update({"value": round(ms_whole * 1e3, 2), "unit": "us", "higher_is_better": False,
+                     "note": "latency-bound (6 output tiles on 148 SMs); TFLOP/s is context only",
+                     "gemm_tflops": round(g_tf, 2)})
+    else:
+        line.update({"value": round(g_flops / (ms_whole * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                     "higher_is_better": True})
+    line["roofline"] = {"bound": "tensor", "kernel": "k_gemm_blockwise", "achieved": round(g_tf, 1),
+                        "peak": round(fp8_burst, 1), "unit": "TFLOP/s", "frac": round(g_tf / fp8_burst, 4),
+                        "frac_of_nominal_4500": round(g_tf / FP8_DENSE_PEAK_TFLOPS, 4),
+                        "peak_note": f"2 x {peak_src} burst BF16 ({bf16_tf})", "traffic": None}
+    line["roofline_quant"] = {"bound": "hbm", "kernel": "k_quant_tiles", "achieved": round(q_gbs, 1),
+                              "peak": hbm_gbs, "unit": "GB/s", "frac": round(q_gbs / hbm_gbs, 4),
+                              "frac_of_nominal_8000": round(q_gbs / NOMINAL_HBM_GBS, 4),
+                              "peak_note": f"{peak_src} copy bandwidth"}
+    line["ops"] = [{"op": op.name, "us": round(m * 1e3, 2),
+                    ("tflops" if op.kind == "g" else "gbs"): round(op.work / (m * 1e-3) / (1e12 if op.kind == "g" else 1e9), 1)}
+                   for m, op in zip(med, ops)]
+    if not args.no_cpu_baseline:
+        flops, secs, sample = oracle_config(c)
+        cb = {"kind": "oracle", "cores": _cpu_threads(), "sample": sample, "seconds": round(secs, 3)}
+        if c == 1:
+            cb.update({"value": round(secs * 1e6, 1), "unit": "us"})
+        else:
+            cb.update({"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s"})
+        line["cpu_baseline"] = cb
+    print(json.dumps(line), flush=True)
+    del ops, flush
+    torch.cuda.empty_cache()

@@ -11,14 +11,17 @@
 //
 // One persistent CTA per SM, tiles of 128 x 256, warp-specialised:
 //   warp 0      TMA producer: A and B tiles of one K block per ring stage (3 stages)
-//   warp 1      MMA issuer: 4 x tcgen05.mma (K = 32 each) per K block into one of the two
-//               256-column TMEM buffers, committed to the stage's "empty" barrier and
-//               the buffer's "full" barrier; also owns the TMEM allocation
+//   warps 1, 3  MMA issuers, one per TMEM buffer: warp 1 takes the even K blocks (buffer
+//               0), warp 3 the odd ones (buffer 1); each issues 4 x tcgen05.mma (K = 32
+//               each) per K block into its 256-column buffer, committed to the stage's
+//               "empty" barrier and the buffer's "full" barrier. One issuing thread
+//               sustains only about 880 clk per K block (4 MMAs + its loop), against 511 of
+//               tensor work; two issue at the full rate. Warp 1 also owns the TMEM allocation.
 //   warp 2      scale loader: for every K block, the tile's 128 row scales of A and its
 //               column scales of B (one per 128-column block, or one per column for
-//               wgrad) are copied with cp.async into a shared-memory ring, so the
-//               promotion never waits on a global load
-//   warp 3      idle (it completes warpgroup 0, which hands its registers over)
+//               wgrad) are copied with cp.async into a shared-memory ring (16-byte copies
+//               where the scale rows are 16-byte aligned), so the promotion never waits
+//               on a global load
 //   warps 4..11 promotion + epilogue: warp w owns TMEM lanes 32*(w%4) .. +31 (output rows)
 //               and columns 128*((w-4)/4) .. +127; partial * (sA * sB) is added into FP32
 //               registers with packed FP32x2 FMAs (fprop/dgrad: one row per thread, read
@@ -96,7 +99,7 @@ struct Cfg {
   static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;  // output staging, one per warp
   static constexpr int OFF_SC = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
   static constexpr int OFF_BAR = OFF_SC + SC_STAGES * SC_SLOT_BYTES;
-  static constexpr int N_BARS = 2 * STAGES + 2 * NBUF + 2 * SC_STAGES + 1;
+  static constexpr int N_BARS = 2 * STAGES + 2 * NBUF + 2 * SC_STAGES + 2;  // + a drain barrier per MMA issuer
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-B alignment
   static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
@@ -116,6 +119,8 @@ struct GemmArgs {
   uint16_t *C;
   int M, N, K;
   int num_m, num_n, kblocks, m_fastest;
+  int vec_a;  // As rows are 16-byte aligned (As aligned, M % 4 == 0): 16-byte scale copies
+  int vec_b;  // wgrad: Bs rows are 16-byte aligned (Bs aligned; N % 8 == 0 always)
   unsigned long long timeout_ns;
   int *status;
 };
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * STAGES + NBUF + b); };
   auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 * NBUF + s); };
   auto sempty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 2 * NBUF + SC_STAGES + s); };
-  const uint32_t drain_bar = bar0 + 8u * (N_BARS - 1);
+  auto drain_bar = [&](int issuer) { return bar0 + 8u * (N_BARS - 2 + issuer); };
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
   volatile int *abort = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
   const float *sc_smem = reinterpret_cast<const float *>(smem + OFF_SC);
@@ -197,7 +202,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(sfull_bar(s), 32);  // one cp.async completion arrival per loader lane
       mbar_init(sempty_bar(s), EPI_WARPS);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_bar(0), 1);
+    mbar_init(drain_bar(1), 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -253,15 +259,19 @@ __global__ void __launch_bounds__(THREADS, 1)
           if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    static_assert(NBUF == 2, "one MMA issuer per TMEM buffer");
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, use = 0;
+      const uint32_t mine = warp == 1 ? 0u : 1u;  // the buffer, and the parity of its K blocks
+      uint32_t use = 0;                            // K blocks of this CTA so far, both issuers
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
         for (int kb = 0; kb < kblocks; ++kb, ++use) {
-          const uint32_t b = use % NBUF;
+          if ((use & 1u) != mine) continue;
+          const int s = static_cast<int>(use % STAGES);
+          const uint32_t ph = (use / STAGES) & 1u;
+          const uint32_t b = mine;
           // The stage's operands are normally in long before its TMEM buffer is free, so
           // that wait comes first and its cost overlaps the promotion still draining the
           // buffer.
@@ -280,13 +290,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                      k > 0 ? 1u : 0u);
           mma_commit(empty_bar(s));
           mma_commit(tfull_bar(b));
-          if (++s == STAGES) s = 0, ph ^= 1u;
         }
       }
       if (!ok) {
         raise_abort(abort, args.status);
-        mma_commit(drain_bar);  // arrives once every MMA issued above has finished
-        mbar_wait(drain_bar, 0, tmo, nullptr);
+        mma_commit(drain_bar(mine));  // arrives once every MMA this thread issued has finished
+        mbar_wait(drain_bar(mine), 0, tmo, nullptr);
       }
     }
   } else if (warp == 2) {
@@ -309,20 +318,37 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int q = 0; q < nk; ++q) {
           const int kb = kb0 + q;
           const float *a_row = args.As + static_cast<int64_t>(kb) * args.M;
+          if (args.vec_a) {
+            // one 16-byte copy per lane: rows 4 * lane .. +3 of the tile
+            const int m0 = mt * BM + 4 * lane;
+            const int valid = min(max(args.M - m0, 0), 4);
+            cp_async_16(dst + 4 * (q * BM) + 16 * lane, valid > 0 ? a_row + m0 : args.As, 4 * valid);
+          } else {
 #pragma unroll 1
-          for (int i = lane; i < BM; i += 32) {
-            const int m = mt * BM + i;
-            const bool v = m < args.M;
-            cp_async_4(dst + 4 * (q * BM + i), v ? a_row + m : args.As, v);
+            for (int i = lane; i < BM; i += 32) {
+              const int m = mt * BM + i;
+              const bool v = m < args.M;
+              cp_async_4(dst + 4 * (q * BM + i), v ? a_row + m : args.As, v);
+            }
           }
           const uint32_t dsb = dst + 4 * (KPS * BM + q * C::SB_STRIDE);
           if (LAYOUT == PURO_WGRAD) {
             const float *b_row = args.Bs + static_cast<int64_t>(kb) * args.N;
+            if (args.vec_b) {
+#pragma unroll
+              for (int h = 0; h < BN / 128; ++h) {
+                const int i = 4 * (lane + 32 * h);
+                const int n0 = nt * BN + i;
+                const int valid = min(max(args.N - n0, 0), 4);
+                cp_async_16(dsb + 4 * i, valid > 0 ? b_row + n0 : args.Bs, 4 * valid);
+              }
+            } else {
 #pragma unroll 1
-            for (int i = lane; i < BN; i += 32) {
-              const int n = nt * BN + i;
-              const bool v = n < args.N;
-              cp_async_4(dsb + 4 * i, v ? b_row + n : args.Bs, v);
+              for (int i = lane; i < BN; i += 32) {
+                const int n = nt * BN + i;
+                const bool v = n < args.N;
+                cp_async_4(dsb + 4 * i, v ? b_row + n : args.Bs, v);
+              }
             }
           } else if (lane < BN / 128) {
             const int nb = nt * (BN / 128) + lane;
@@ -713,6 +739,8 @@ int gemm_args(const float *As, const float *Bs, int64_t M, int64_t N, int64_t K,
   // Walk the smaller operand fastest so that it stays resident in L2 while the larger
   // one streams through once.
   args.m_fastest = M <= N ? 1 : 0;
+  args.vec_a = (reinterpret_cast<uintptr_t>(As) % 16 == 0 && M % 4 == 0) ? 1 : 0;
+  args.vec_b = (reinterpret_cast<uintptr_t>(Bs) % 16 == 0) ? 1 : 0;  // used by wgrad only
   args.timeout_ns = wait_timeout_ns();
   args.status = status;
   return PURO_OK;

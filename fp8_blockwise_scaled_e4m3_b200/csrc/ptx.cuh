@@ -135,6 +135,13 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, bool v
                "r"(valid ? 4 : 0)
                : "memory");
 }
+// Asynchronous 16-byte copy global -> shared, through L2 only: the first `src_bytes` (0..16)
+// bytes are read and the rest of the 16 zero-filled. Both addresses 16-byte aligned; with
+// src_bytes 0 nothing is read (`src` must still be a mapped address).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
 // Arrives on the mbarrier once all of this thread's earlier cp.async copies have landed.
 // The arrival is not added to the pending count: the barrier's expected count includes it.
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
