@@ -76,13 +76,18 @@ constexpr int STG_BOX_BYTES = 32 * 128;   // 32 rows x 64 BF16 columns, 128B-swi
 
 // Tile width TN (256 or 128) sets the rest. TMEM holds 512 FP32 columns, i.e.
 // 512 / TN partial buffers; each promotion warp owns TN / 2 columns of one lane quadrant.
-template <int LAYOUT, int TN>
+// PAIR: a cluster of two CTAs computes a 256 x TN tile with cta_group::2 MMAs. Each CTA
+// holds its own 128 rows of A and half (TN / 2 rows) of B in shared memory and receives
+// its 128 rows x TN columns of the product in its TMEM, so per output element each SM
+// stages and reads half as many B bytes as a single CTA does.
+template <int LAYOUT, int TN, bool PAIR>
 struct Cfg {
   static constexpr int BN = TN;
   static constexpr int NBUF = 512 / TN;            // TMEM partial buffers
   static constexpr int WCOLS = TN / 2;             // columns per promotion warp
-  static constexpr int STAGES = TN == 256 ? 3 : 5;
-  static constexpr int B_BYTES = TN * BK;
+  static constexpr int B_ROWS = PAIR ? TN / 2 : TN;  // rows of B this CTA stages
+  static constexpr int B_BYTES = B_ROWS * BK;
+  static constexpr int STAGES = PAIR ? 4 : (TN == 256 ? 3 : 5);
   // Scale-ring slot, KPS K blocks: KPS x 128 row scales of A, then KPS x SB_STRIDE
   // scales of B (TN column scales for wgrad, one per 128-column block otherwise).
   static constexpr int SB_STRIDE = LAYOUT == PURO_WGRAD ? TN : 4;
@@ -92,7 +97,7 @@ struct Cfg {
   static constexpr int SC_SLOT_FLOATS = KPS * (BM + SB_STRIDE);
   static constexpr int SC_SLOT_BYTES = SC_SLOT_FLOATS * 4;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t IDESC = idesc_e4m3_f32(BM, TN);
+  static constexpr uint32_t IDESC = idesc_e4m3_f32(PAIR ? 2 * BM : BM, TN);
   static constexpr int STG_WARP_BYTES = (WCOLS / 64) * STG_BOX_BYTES;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -160,11 +165,11 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 
 // ACC32: instead of storing BF16, add the FP32 result into an FP32 C (main-gradient
 // accumulation of wgrad) with TMA reduce-add.
-template <int LAYOUT, int TN, bool ACC32>
+template <int LAYOUT, int TN, bool ACC32, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
-  using C = Cfg<LAYOUT, TN>;
+  using C = Cfg<LAYOUT, TN, PAIR>;
   constexpr int BN = C::BN, NBUF = C::NBUF, STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_STG = C::OFF_STG, OFF_SC = C::OFF_SC;
@@ -188,6 +193,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // PAIR: rank 0 of the cluster is the leader (it issues the MMAs for both CTAs and holds
+  // the barriers they report to); tiles are walked per cluster.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // first output row of this CTA in tile row mt
+  auto row_base = [&](int mt) { return PAIR ? mt * 2 * BM + static_cast<int>(rank) * BM : mt * BM; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -196,7 +209,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), EPI_WARPS);
+      mbar_init(tempty_bar(b), PAIR ? 2 * EPI_WARPS : EPI_WARPS);  // PAIR: both CTAs' warps
     }
     for (int s = 0; s < SC_STAGES; ++s) {
       mbar_init(sfull_bar(s), 32);  // one cp.async completion arrival per loader lane
@@ -213,11 +226,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // both CTAs' barriers exist before either reports to the other
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
@@ -236,7 +257,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t ph = 0;
       uint32_t issued = 0, issued_parity = 0;  // per-stage bit masks
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
         int mt, nt;
         tile_coords(tile, args, mt, nt);
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -244,9 +265,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
-          tma_load_2d(sbase + OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
-          tma_load_2d(sbase + OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
+          if constexpr (PAIR) {
+            // Both CTAs' loads are counted on the leader's barrier, which the leader arms
+            // with the pair's bytes. A peer's load for the next use of a stage can only
+            // start after the MMA that read the stage completed (the empty barrier), so
+            // it never lands in the leader's barrier before the previous phase is over.
+            const uint32_t fb = map_to_rank(full_bar(s), 0);
+            if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (A_BYTES + B_BYTES));
+            tma_load_2d_pair(sbase + OFF_A + s * A_BYTES, &tmA, fb, kb * BK, row_base(mt));
+            tma_load_2d_pair(sbase + OFF_B + s * B_BYTES, &tmB, fb, kb * BK,
+                             nt * BN + static_cast<int>(rank) * C::B_ROWS);
+          } else {
+            mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+            tma_load_2d(sbase + OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
+            tma_load_2d(sbase + OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
+          }
           issued |= 1u << s;
           issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
           if (++s == STAGES) s = 0, ph ^= 1u;
@@ -254,19 +287,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!ok) {
         raise_abort(abort, args.status);
-        // Let every issued tensor load land before the CTA can exit.
-        for (int i = 0; i < STAGES; ++i)
-          if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
+        // Let every issued tensor load land before the CTA can exit. (A peer's loads are
+        // counted on the leader's barriers, which the leader drains; the peer stays alive
+        // until then through the cluster barrier at the end of the kernel.)
+        if (leader)
+          for (int i = 0; i < STAGES; ++i)
+            if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
       }
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
     static_assert(NBUF == 2, "one MMA issuer per TMEM buffer");
-    if (lane == 0) {
+    if (lane == 0 && leader) {  // PAIR: the leader issues for both CTAs
       const uint32_t mine = warp == 1 ? 0u : 1u;  // the buffer, and the parity of its K blocks
       uint32_t use = 0;                            // K blocks of this CTA so far, both issuers
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
         for (int kb = 0; kb < kblocks; ++kb, ++use) {
           if ((use & 1u) != mine) continue;
           const int s = static_cast<int>(use % STAGES);
@@ -284,17 +320,30 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t d = tmem + b * BN;
           const uint32_t a_addr = sbase + OFF_A + s * A_BYTES;
           const uint32_t b_addr = sbase + OFF_B + s * B_BYTES;
+          if constexpr (PAIR) {
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k)
-            mma_e4m3(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), C::IDESC,
-                     k > 0 ? 1u : 0u);
-          mma_commit(empty_bar(s));
-          mma_commit(tfull_bar(b));
+            for (int k = 0; k < BK / 32; ++k)
+              mma_e4m3_pair(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), C::IDESC,
+                            k > 0 ? 1u : 0u);
+            mma_commit_pair_mc(empty_bar(s), 0x3);  // both CTAs' stage s is free again
+            mma_commit_pair_mc(tfull_bar(b), 0x3);  // both CTAs' partial is in TMEM
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k)
+              mma_e4m3(d, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k), C::IDESC,
+                       k > 0 ? 1u : 0u);
+            mma_commit(empty_bar(s));
+            mma_commit(tfull_bar(b));
+          }
         }
       }
       if (!ok) {
         raise_abort(abort, args.status);
-        mma_commit(drain_bar(mine));  // arrives once every MMA this thread issued has finished
+        // arrives once every MMA this thread issued has finished
+        if constexpr (PAIR)
+          mma_commit_pair(drain_bar(mine));
+        else
+          mma_commit(drain_bar(mine));
         mbar_wait(drain_bar(mine), 0, tmo, nullptr);
       }
     }
@@ -305,9 +354,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     int ss = 0;
     uint32_t sph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+    for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
       int mt, nt;
       tile_coords(tile, args, mt, nt);
+      const int m_first = row_base(mt);
       for (int kb0 = 0; kb0 < kblocks; kb0 += KPS) {
         if (!mbar_wait(sempty_bar(ss), sph ^ 1u, tmo, abort)) {
           ok = false;
@@ -320,13 +370,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float *a_row = args.As + static_cast<int64_t>(kb) * args.M;
           if (args.vec_a) {
             // one 16-byte copy per lane: rows 4 * lane .. +3 of the tile
-            const int m0 = mt * BM + 4 * lane;
+            const int m0 = m_first + 4 * lane;
             const int valid = min(max(args.M - m0, 0), 4);
             cp_async_16(dst + 4 * (q * BM) + 16 * lane, valid > 0 ? a_row + m0 : args.As, 4 * valid);
           } else {
 #pragma unroll 1
             for (int i = lane; i < BM; i += 32) {
-              const int m = mt * BM + i;
+              const int m = m_first + i;
               const bool v = m < args.M;
               cp_async_4(dst + 4 * (q * BM + i), v ? a_row + m : args.As, v);
             }
@@ -378,10 +428,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     int ss = 0;
     uint32_t sph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+    // PAIR: the TMEM buffer goes back to the leader's MMA issuer, which waits for both CTAs
+    const uint32_t tempty_target0 = PAIR ? map_to_rank(tempty_bar(0), 0) : tempty_bar(0);
+    for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
       int mt, nt;
       tile_coords(tile, args, mt, nt);
       const int n_base = nt * BN + half * WCOLS;  // first column of this warp
+      const int m_first = row_base(mt);
       uint64_t acc[WCOLS / 2];
 #pragma unroll
       for (int i = 0; i < WCOLS / 2; ++i) acc[i] = 0;
@@ -428,7 +481,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (c == WCOLS / 64 - 1) {
               tc_fence_before_sync();
               __syncwarp();
-              if (lane == 0 && !PURO_SKIP_RELEASE(use)) mbar_arrive(tempty_bar(b));
+              if (lane == 0 && !PURO_SKIP_RELEASE(use)) {
+                if constexpr (PAIR)
+                  mbar_arrive_cluster(tempty_target0 + 8u * b);
+                else
+                  mbar_arrive(tempty_bar(b));
+              }
             }
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -489,7 +547,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             } else {
               tc_fence_before_sync();
               __syncwarp();
-              if (lane == 0 && !PURO_SKIP_RELEASE(use)) mbar_arrive(tempty_bar(b));
+              if (lane == 0 && !PURO_SKIP_RELEASE(use)) {
+                if constexpr (PAIR)
+                  mbar_arrive_cluster(tempty_target0 + 8u * b);
+                else
+                  mbar_arrive(tempty_bar(b));
+              }
             }
             apply(q + 1, rb);
             if (q + 2 < 4) tmem_wait_ld_dep(ra);
@@ -533,7 +596,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            const int row0 = mt * BM + quad * 32;
+            const int row0 = m_first + quad * 32;
             if (row0 < args.M) {
 #pragma unroll
               for (int bb = 0; bb < 2; ++bb) {
@@ -580,7 +643,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        const int row0 = mt * BM + quad * 32;
+        const int row0 = m_first + quad * 32;
         if (row0 < args.M) {
 #pragma unroll
           for (int box = 0; box < WCOLS / 64; ++box)
@@ -596,10 +659,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // neither CTA leaves while the other may still use its shared memory or TMEM
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -659,31 +728,46 @@ int *device_status_ptr() {
   return p;
 }
 
-template <int LAYOUT, bool ACC32>
-int launch_layout(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
+// Which kernel shape serves a GEMM: the CTA-pair kernel (256-row tiles) unless the output
+// has at most 128 rows. PURO_GEMM_PAIR=0 or 1 forces one of them (read once per process).
+bool use_pair(int64_t M) {
+  static const int mode = [] {
+    const char *e = std::getenv("PURO_GEMM_PAIR");
+    return e == nullptr ? -1 : std::atoi(e);
+  }();
+  if (mode == 0) return false;
+  if (mode == 1) return true;
+  return M > BM;
+}
+
+template <int LAYOUT, bool ACC32, bool PAIR>
+int launch_kernel(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
                   cudaStream_t stream) {
   constexpr int TN = TileFor<LAYOUT>::TN;
-  constexpr int SMEM_BYTES = Cfg<LAYOUT, TN>::SMEM_BYTES;
+  using CF = Cfg<LAYOUT, TN, PAIR>;
+  constexpr int SMEM_BYTES = CF::SMEM_BYTES;
   const int64_t M = args.M, N = args.N, K = args.K;
   CUtensorMap ta, tb, tc;
   if (!make_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, TN, BK,
+      !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, CF::B_ROWS, BK,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !(ACC32 ? make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, N, 32, 32,
                          CU_TENSOR_MAP_SWIZZLE_128B)
               : make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
                          CU_TENSOR_MAP_SWIZZLE_128B)))
     return PURO_ERR_CUDA;
-  args.num_m = static_cast<int>((M + BM - 1) / BM);
+  const int tile_rows = PAIR ? 2 * BM : BM;
+  args.num_m = static_cast<int>((M + tile_rows - 1) / tile_rows);
   args.num_n = static_cast<int>((N + TN - 1) / TN);
   const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32>;
+  auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32, PAIR>;
   // Once per device: the register split inside the kernel assumes exactly LAUNCH_REGS per
   // thread at launch (with any other count the promotion warps' setmaxnreg.inc could wait
-  // forever), and the kernel needs its dynamic shared memory opted in.
-  static PerDevice<int> prepared;
+  // forever), the kernel needs its dynamic shared memory opted in, and a pair kernel's
+  // grid is sized by the clusters that can be resident at once (a persistent grid with
+  // more would leave the extra clusters to run after the others).
+  static PerDevice<int> prepared;  // PURO_OK or an error; for PAIR, the resident clusters
   int prep = PURO_ERR_CUDA;
   if (!prepared.get(prep, [&](int, int &v) {
         cudaFuncAttributes fa{};
@@ -700,23 +784,72 @@ int launch_layout(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs arg
           return false;
         }
         v = PURO_OK;
+        if constexpr (PAIR) {
+          cudaLaunchConfig_t cfg{};
+          cudaLaunchAttribute attr[1];
+          attr[0].id = cudaLaunchAttributeClusterDimension;
+          attr[0].val.clusterDim.x = 2;
+          attr[0].val.clusterDim.y = 1;
+          attr[0].val.clusterDim.z = 1;
+          cfg.gridDim = dim3(2 * (sms / 2));
+          cfg.blockDim = dim3(THREADS);
+          cfg.dynamicSmemBytes = SMEM_BYTES;
+          cfg.attrs = attr;
+          cfg.numAttrs = 1;
+          int clusters = 0;
+          if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+            std::fprintf(stderr, "puro_fp8: no CTA pair of the GEMM kernel fits on this device\n");
+            v = PURO_ERR_LAUNCH;
+            return true;
+          }
+          v = clusters;  // > 0
+        }
         return true;
       }))
     return PURO_ERR_CUDA;
-  if (prep != PURO_OK) return prep;
-  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, args);
-  cudaError_t e = cudaGetLastError();
+  if (prep < 0) return prep;
+  cudaError_t e;
+  int grid;
+  if constexpr (PAIR) {
+    const int64_t clusters = tiles < prep ? tiles : prep;
+    grid = static_cast<int>(2 * clusters);
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  } else {
+    grid = static_cast<int>(tiles < sms ? tiles : sms);
+    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, args);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, kern);
     std::fprintf(stderr,
-                 "puro_fp8: GEMM launch (grid %d, %d threads, %d B smem): %s "
+                 "puro_fp8: GEMM launch (grid %d, %d threads, %d B smem, %s): %s "
                  "[kernel: %d regs, max %d threads/block, max dyn smem %d]\n",
-                 grid, THREADS, SMEM_BYTES, cudaGetErrorString(e), fa.numRegs,
-                 fa.maxThreadsPerBlock, fa.maxDynamicSharedSizeBytes);
+                 grid, THREADS, SMEM_BYTES, PAIR ? "CTA pairs" : "single CTAs", cudaGetErrorString(e),
+                 fa.numRegs, fa.maxThreadsPerBlock, fa.maxDynamicSharedSizeBytes);
     return PURO_ERR_LAUNCH;
   }
   return PURO_OK;
+}
+
+template <int LAYOUT, bool ACC32>
+int launch_layout(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
+                  cudaStream_t stream) {
+  return use_pair(args.M) ? launch_kernel<LAYOUT, ACC32, true>(Aq, Bq, Cout, args, sms, stream)
+                          : launch_kernel<LAYOUT, ACC32, false>(Aq, Bq, Cout, args, sms, stream);
 }
 
 }  // namespace

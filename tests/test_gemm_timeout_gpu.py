@@ -12,7 +12,9 @@ out. The test checks, in a child process whose wait limit is 20 ms:
 * the status word is clear again after that read;
 * with the hook off, the same GEMM on the same context runs clean and gives the exact
   result of an exact-integer case, so the context and the library stay usable.
-Both promotion shapes are covered: fprop (32x32b TMEM loads) and wgrad (16x256b).
+Both promotion shapes are covered, fprop (32x32b TMEM loads) and wgrad (16x256b), on a
+single-CTA tile (M = 128) and on one CTA pair's tile (M = 256: the withheld hand-back is
+owed to the leader's barrier by both CTAs, and each CTA gives up on its own bounded waits).
 """
 
 import os
@@ -55,10 +57,11 @@ import numpy as np
 import torch
 lib = ctypes.CDLL(sys.argv[1])
 layout = int(sys.argv[2])
+M = int(sys.argv[3])
 p, i64 = ctypes.c_void_p, ctypes.c_int64
 lib.puro_fp8_gemm_blockwise.argtypes = [p, p, p, p, p, i64, i64, i64, ctypes.c_int, p, ctypes.c_size_t, p]
 lib.puro_fp8_sync_status.argtypes = [p]
-M, N, K = 128, 256, 1024          # one 128 x 256 tile, 8 K blocks
+N, K = 256, 1024                  # one output tile (128 x 256, or a CTA pair's 256 x 256), 8 K blocks
 rng = np.random.default_rng(1)
 codes = np.array([0x00, 0x38, 0xB8, 0x40, 0xC0], dtype=np.uint8)    # 0, +-1, +-2
 aq = codes[rng.integers(0, 5, size=(M, K))]
@@ -89,11 +92,12 @@ print("RESULT", *out, int(exact), flush=True)
 """
 
 
+@pytest.mark.parametrize("m", [128, 256], ids=["single_cta", "cta_pair"])
 @pytest.mark.parametrize("layout", [0, 2], ids=["fprop", "wgrad"])
-def test_gemm_wait_gives_up_reports_timeout_and_context_survives(layout):
+def test_gemm_wait_gives_up_reports_timeout_and_context_survives(layout, m):
     _build()
     env = dict(os.environ, PURO_WAIT_TIMEOUT_MS="20")
-    r = subprocess.run([sys.executable, "-c", CHILD, LIB, str(layout)], capture_output=True, text=True,
+    r = subprocess.run([sys.executable, "-c", CHILD, LIB, str(layout), str(m)], capture_output=True, text=True,
                        env=env, timeout=300)
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("RESULT")]
     assert r.returncode == 0 and lines, r.stdout + r.stderr
