@@ -59,7 +59,8 @@ def _args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--config", default="5",
                    help="workload: 1 small outlier GEMM, 2 one layer's forward linears, 3 its backward, "
-                        "4 the LM head, 5 the full 28-layer step (default), or 'all' for 1-4 then 5")
+                        "4 the LM head, 5 the full 28-layer step (default), 'all' for 1-4 then 5, or "
+                        "'fused' for the fused epilogue quantisation against GEMM + separate quantiser")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions of configs 1-4")
     return p.parse_args()
 
@@ -591,6 +592,10 @@ def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.config == "fused":
+        from bench_configs import run_fused_comparison
+        run_fused_comparison(args)
         return
     if args.config in ("1", "2", "3", "4", "all"):
         from bench_configs import run_config

@@ -265,3 +265,61 @@ def run_config(c, args):
     print(json.dumps(line), flush=True)
     del ops, flush
     torch.cuda.empty_cache()
+
+
+def run_fused_comparison(args):
+    """fprop and dgrad of one Qwen3-1.7B-shaped block at 8192 tokens, each timed two ways:
+    the GEMM followed by a separate 1x128 quantisation of its BF16 output (the input of the
+    next linear), and puro_fp8_gemm_blockwise_quant, which writes both from one launch.
+    Same operands, L2 flushed before every repetition, median over repetitions."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    T = 8192
+    fwd = wl.layer_forward(4, T, dev, layer=0)
+    grads = wl.layer_grads(4, T, dev, layer=0)
+    flush = torch.empty(512 * 2 ** 20 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    cases = []
+    for (name, x, w), (_, dy) in zip(fwd, grads):
+        xq, xs = pf.quantize_1x128(x)
+        wq, wqt, ws = pf.quantize_128x128(w)
+        dyq, dys = pf.quantize_1x128(dy)
+        cases.append((f"{name} fprop", "fprop", (xq, xs, wq, ws)))
+        cases.append((f"{name} dgrad", "dgrad", (dyq, dys, wqt, ws)))
+    rows = []
+    for label, layout, ops in cases:
+        m, n = ops[0].shape[0], ops[2].shape[0]
+        c = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        cq = torch.empty((m, n), dtype=torch.uint8, device=dev)
+        cs = torch.empty((n // 128, m), dtype=torch.float32, device=dev)
+        lay = {"fprop": pf.PURO_FPROP, "dgrad": pf.PURO_DGRAD}[layout]
+
+        def separate(st):
+            pf.puro_fp8_gemm_blockwise(*ops, c, lay, None, st)
+            pf.puro_fp8_quantize_1x128(c, cq, cs, st)
+
+        def fused(st):
+            pf.puro_fp8_gemm_blockwise_quant(*ops, c, cq, cs, lay, st)
+
+        t = {"separate": [], "fused": []}
+        for rep in range(args.warmup + args.reps):
+            for kind, fn in (("separate", separate), ("fused", fused)):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn(stream)
+                e1.record(stream)
+                e1.synchronize()
+                if rep >= args.warmup:
+                    t[kind].append(e0.elapsed_time(e1))
+        sep, fus = statistics.median(t["separate"]), statistics.median(t["fused"])
+        rows.append({"op": label, "M": m, "N": n, "K": ops[0].shape[1], "separate_us": round(sep * 1e3, 1),
+                     "fused_us": round(fus * 1e3, 1), "saved_pct": round(100 * (1 - fus / sep), 1)})
+        del c, cq, cs
+    pf.puro_fp8_sync_status()
+    tot_sep = sum(r["separate_us"] for r in rows)
+    tot_fus = sum(r["fused_us"] for r in rows)
+    print(json.dumps({"comparison": "GEMM + separate 1x128 quantiser of its output vs the fused epilogue",
+                      "workload": "fprop and dgrad of one Qwen3-1.7B-shaped block at 8192 tokens, seed 4",
+                      "l2": "flushed before every repetition", "reps": args.reps,
+                      "total_separate_us": round(tot_sep, 1), "total_fused_us": round(tot_fus, 1),
+                      "saved_pct": round(100 * (1 - tot_fus / tot_sep), 1), "ops": rows}), flush=True)

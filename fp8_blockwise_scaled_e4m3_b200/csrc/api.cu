@@ -100,6 +100,23 @@ int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *B
   return puro::launch_gemm_blockwise(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
 }
 
+int puro_fp8_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                                  const float *Bs, uint16_t *C, uint8_t *Cq, float *Cs, int64_t M,
+                                  int64_t N, int64_t K, int layout, puro_stream_t stream) {
+  if (Aq == nullptr || As == nullptr || Bq == nullptr || Bs == nullptr || C == nullptr ||
+      Cq == nullptr || Cs == nullptr)
+    return PURO_ERR_NULL;
+  if (layout != PURO_FPROP && layout != PURO_DGRAD) return PURO_ERR_LAYOUT;
+  if (M < 1 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0) return PURO_ERR_SHAPE;
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
+  if (!tiles_fit(M, 128, N, 256)) return PURO_ERR_SHAPE;
+  if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16) || !aligned(Cq, 16) || !aligned(As, 4) ||
+      !aligned(Bs, 4) || !aligned(Cs, 4))
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_gemm_blockwise_quant(Aq, As, Bq, Bs, C, Cq, Cs, M, N, K, layout, stream);
+}
+
 int puro_fp8_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                                 const float *Bs, float *C, int64_t M, int64_t N, int64_t K,
                                 puro_stream_t stream) {

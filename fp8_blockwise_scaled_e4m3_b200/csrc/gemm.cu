@@ -46,6 +46,7 @@
 #include "host_cache.h"
 #include "ptx.cuh"
 #include "quant.h"
+#include "quant_math.cuh"
 
 namespace puro {
 namespace {
@@ -87,7 +88,7 @@ struct Cfg {
   static constexpr int WCOLS = TN / 2;             // columns per promotion warp
   static constexpr int B_ROWS = PAIR ? TN / 2 : TN;  // rows of B this CTA stages
   static constexpr int B_BYTES = B_ROWS * BK;
-  static constexpr int STAGES = PAIR ? 4 : (TN == 256 ? 3 : 5);
+  static constexpr int STAGES = PAIR ? (TN == 128 ? 6 : 4) : (TN == 256 ? 3 : 5);
   // Scale-ring slot, KPS K blocks: KPS x 128 row scales of A, then KPS x SB_STRIDE
   // scales of B (TN column scales for wgrad, one per 128-column block otherwise).
   static constexpr int SB_STRIDE = LAYOUT == PURO_WGRAD ? TN : 4;
@@ -111,9 +112,11 @@ struct Cfg {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
-// Every layout uses 256-wide tiles (two TMEM buffers): measured faster than 128-wide
-// tiles with four buffers, for wgrad too once its promotion reads the 16x256b shape.
-template <int LAYOUT>
+// Tile widths: 128 x 256 for single CTAs and 256 x 256 for CTA pairs, in every layout (two
+// 256-column TMEM buffers). Measured on B200 and set aside: 128-wide tiles with four
+// buffers, 25-30% slower for single CTAs (shared-memory bandwidth) and 12-17% slower as
+// 256 x 128 pair tiles (MMA issue rate and shared-memory bandwidth).
+template <int LAYOUT, bool PAIR>
 struct TileFor {
   static constexpr int TN = 256;
 };
@@ -128,6 +131,8 @@ struct GemmArgs {
   int vec_b;  // wgrad: Bs rows are 16-byte aligned (Bs aligned; N % 8 == 0 always)
   unsigned long long timeout_ns;
   int *status;
+  uint8_t *Cq;  // QOUT: 1x128 codes of the BF16 output along N, [M, N] dense
+  float *Cs;    // QOUT: their scales, [N/128, M]
 };
 
 __device__ int g_status;  // non-zero: a bounded wait gave up since the last read
@@ -165,7 +170,11 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 
 // ACC32: instead of storing BF16, add the FP32 result into an FP32 C (main-gradient
 // accumulation of wgrad) with TMA reduce-add.
-template <int LAYOUT, int TN, bool ACC32, bool PAIR>
+// QOUT (fprop/dgrad): the epilogue also quantises the BF16 output row-wise, 1x128 along N:
+// a promotion thread holds one output row x 128 columns, exactly one group, so the group's
+// amax, scale and codes come from the thread's own registers (the same arithmetic as the
+// separate 1x128 quantiser, applied to the same BF16 values).
+template <int LAYOUT, int TN, bool ACC32, bool PAIR, bool QOUT>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
@@ -297,9 +306,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------ MMA issuers
-    static_assert(NBUF == 2, "one MMA issuer per TMEM buffer");
+    static_assert(NBUF % 2 == 0, "two MMA issuers take alternate K blocks");
     if (lane == 0 && leader) {  // PAIR: the leader issues for both CTAs
-      const uint32_t mine = warp == 1 ? 0u : 1u;  // the buffer, and the parity of its K blocks
+      const uint32_t mine = warp == 1 ? 0u : 1u;  // the parity of this issuer's K blocks
       uint32_t use = 0;                            // K blocks of this CTA so far, both issuers
       bool ok = true;
       for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if ((use & 1u) != mine) continue;
           const int s = static_cast<int>(use % STAGES);
           const uint32_t ph = (use / STAGES) & 1u;
-          const uint32_t b = mine;
+          const uint32_t b = use % NBUF;
           // The stage's operands are normally in long before its TMEM buffer is free, so
           // that wait comes first and its cost overlaps the promotion still draining the
           // buffer.
@@ -438,6 +447,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint64_t acc[WCOLS / 2];
 #pragma unroll
       for (int i = 0; i < WCOLS / 2; ++i) acc[i] = 0;
+      float fq[KPS];  // fprop/dgrad: the slot's factors sA * sB, K block kb's first
 
       for (int kb = 0; kb < kblocks; ++kb, ++use) {
         const uint32_t b = use % NBUF;
@@ -449,8 +459,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         const float *slot = sc_smem + ss * C::SC_SLOT_FLOATS;
-        const float sa = slot[kq * BM + row];
-        const float *sbk = slot + KPS * BM + kq * C::SB_STRIDE;
         const bool slot_done = kq == KPS - 1 || kb == kblocks - 1;
         auto release_slot = [&]() {
           if (slot_done) {
@@ -460,19 +468,30 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         };
         if constexpr (LAYOUT != PURO_WGRAD) {
-          // One scalar factor per thread and K block: partial * (sA * sB).
-          const float sb = sbk[(half * WCOLS) / 128];
-          release_slot();
-          const uint64_t s2 = pack2(sa * sb, sa * sb);
+          // One scalar factor per thread and K block: partial * (sA * sB). All KPS factors
+          // of a slot are read at its first K block (one shared-memory latency per slot,
+          // off the per-K-block chain) and the slot goes back to the loader at once.
+          static_assert(WCOLS == 128 || WCOLS == 64, "fprop/dgrad promotion: 64 or 128 columns per warp");
+          if (kq == 0) {
+            const int sbi = (half * WCOLS) / 128;
+#pragma unroll
+            for (int q = 0; q < KPS; ++q) fq[q] = slot[q * BM + row] * slot[KPS * BM + q * C::SB_STRIDE + sbi];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sempty_bar(ss));
+            if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
+          }
+          const uint64_t s2 = pack2(fq[0], fq[0]);
+#pragma unroll
+          for (int q = 0; q + 1 < KPS; ++q) fq[q] = fq[q + 1];
           if (!mbar_wait(tfull_bar(b), (use / NBUF) & 1u, tmo, abort)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
           const uint32_t taddr = tmem + lane_base + b * BN + half * WCOLS;
-          // 64-column TMEM loads, one wait each; the buffer goes back to the MMA warp
-          // once the last chunk is in registers. (Double-buffered 32-column loads, with
-          // the next chunk in flight while one is added, measured 1-2% slower.)
+          // 64-column TMEM loads, one wait each; the buffer goes back to the MMA issuer once
+          // the last chunk is in registers, before that chunk's FMAs. (With 32-column loads,
+          // each chunk's FMAs overlapping the next chunk's load, it measured 1-2% slower.)
 #pragma unroll
           for (int c = 0; c < WCOLS / 64; ++c) {
             uint32_t r[64];
@@ -610,6 +629,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
       if constexpr (LAYOUT != PURO_WGRAD) {
         // thread = row `lane`, columns in order
+        uint32_t w[WCOLS / 2];  // the row's BF16 pairs
 #pragma unroll
         for (int j = 0; j < WCOLS / 8; ++j) {
           float v[8];
@@ -617,12 +637,46 @@ __global__ void __launch_bounds__(THREADS, 1)
           unpack2(acc[4 * j + 1], v[2], v[3]);
           unpack2(acc[4 * j + 2], v[4], v[5]);
           unpack2(acc[4 * j + 3], v[6], v[7]);
+          w[4 * j] = bf16x2_bits(v[0], v[1]);
+          w[4 * j + 1] = bf16x2_bits(v[2], v[3]);
+          w[4 * j + 2] = bf16x2_bits(v[4], v[5]);
+          w[4 * j + 3] = bf16x2_bits(v[6], v[7]);
           const uint32_t addr =
               stg + (j >> 3) * STG_BOX_BYTES + lane * 128 + (((j & 7) ^ (lane & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                       "r"(bf16x2_bits(v[0], v[1])), "r"(bf16x2_bits(v[2], v[3])),
-                       "r"(bf16x2_bits(v[4], v[5])), "r"(bf16x2_bits(v[6], v[7]))
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[4 * j]),
+                       "r"(w[4 * j + 1]), "r"(w[4 * j + 2]), "r"(w[4 * j + 3])
                        : "memory");
+        }
+        if constexpr (QOUT) {
+          static_assert(WCOLS == 128, "one 1x128 group per thread");
+          const int grow = m_first + row;
+          if (grow < args.M && n_base < args.N) {
+            // amax over the 128 BF16 values (exact), in four independent chains
+            uint32_t m4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int i = 0; i < WCOLS / 2; ++i) m4[i & 3] = bf16x2_absmax(m4[i & 3], w[i]);
+            const float amax =
+                bf16x2_absmax_to_f32(bf16x2_absmax(bf16x2_absmax(m4[0], m4[1]), bf16x2_absmax(m4[2], m4[3])));
+            float sq;
+            BlockDivider dq;
+            bool fast;
+            block_scale_fast(amax, sq, dq, fast);
+            if (!fast) block_scale(amax, sq, dq);  // tiny, infinite or NaN amax
+            const uint64_t nr2 = pack2(-dq.r, -dq.r), s2q = pack2(dq.s, dq.s);
+            uint8_t *qrow = args.Cq + static_cast<int64_t>(grow) * args.N + n_base;
+#pragma unroll
+            for (int k = 0; k < WCOLS / 16; ++k) {
+              uint32_t q[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t)
+                q[t] = fast ? block_codes4_fast(w[8 * k + 2 * t], w[8 * k + 2 * t + 1], nr2, s2q)
+                            : block_codes4(w[8 * k + 2 * t], w[8 * k + 2 * t + 1], dq);
+              asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(qrow + 16 * k), "r"(q[0]),
+                           "r"(q[1]), "r"(q[2]), "r"(q[3])
+                           : "memory");
+            }
+            args.Cs[static_cast<int64_t>(n_base / 128) * args.M + grow] = sq;
+          }
         }
       } else {
         // 16x256b ownership: acc[8x + j] is row g + 8x, columns 8j + c, 8j + c + 1; one
@@ -740,10 +794,10 @@ bool use_pair(int64_t M) {
   return M > BM;
 }
 
-template <int LAYOUT, bool ACC32, bool PAIR>
+template <int LAYOUT, bool ACC32, bool PAIR, bool QOUT>
 int launch_kernel(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
                   cudaStream_t stream) {
-  constexpr int TN = TileFor<LAYOUT>::TN;
+  constexpr int TN = TileFor<LAYOUT, PAIR>::TN;
   using CF = Cfg<LAYOUT, TN, PAIR>;
   constexpr int SMEM_BYTES = CF::SMEM_BYTES;
   const int64_t M = args.M, N = args.N, K = args.K;
@@ -761,7 +815,7 @@ int launch_kernel(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs arg
   args.num_m = static_cast<int>((M + tile_rows - 1) / tile_rows);
   args.num_n = static_cast<int>((N + TN - 1) / TN);
   const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
-  auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32, PAIR>;
+  auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32, PAIR, QOUT>;
   // Once per device: the register split inside the kernel assumes exactly LAUNCH_REGS per
   // thread at launch (with any other count the promotion warps' setmaxnreg.inc could wait
   // forever), the kernel needs its dynamic shared memory opted in, and a pair kernel's
@@ -845,11 +899,11 @@ int launch_kernel(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs arg
   return PURO_OK;
 }
 
-template <int LAYOUT, bool ACC32>
+template <int LAYOUT, bool ACC32, bool QOUT = false>
 int launch_layout(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
                   cudaStream_t stream) {
-  return use_pair(args.M) ? launch_kernel<LAYOUT, ACC32, true>(Aq, Bq, Cout, args, sms, stream)
-                          : launch_kernel<LAYOUT, ACC32, false>(Aq, Bq, Cout, args, sms, stream);
+  return use_pair(args.M) ? launch_kernel<LAYOUT, ACC32, true, QOUT>(Aq, Bq, Cout, args, sms, stream)
+                          : launch_kernel<LAYOUT, ACC32, false, QOUT>(Aq, Bq, Cout, args, sms, stream);
 }
 
 }  // namespace
@@ -892,6 +946,22 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
     case PURO_FPROP: return launch_layout<PURO_FPROP, false>(Aq, Bq, C, args, sms, stream);
     case PURO_DGRAD: return launch_layout<PURO_DGRAD, false>(Aq, Bq, C, args, sms, stream);
     case PURO_WGRAD: return launch_layout<PURO_WGRAD, false>(Aq, Bq, C, args, sms, stream);
+    default: return PURO_ERR_LAYOUT;
+  }
+}
+
+int launch_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                                const float *Bs, uint16_t *C, uint8_t *Cq, float *Cs, int64_t M,
+                                int64_t N, int64_t K, int layout, cudaStream_t stream) {
+  GemmArgs args;
+  int sms = 0;
+  if (int e = gemm_args(As, Bs, M, N, K, args, sms)) return e;
+  args.C = C;
+  args.Cq = Cq;
+  args.Cs = Cs;
+  switch (layout) {
+    case PURO_FPROP: return launch_layout<PURO_FPROP, false, true>(Aq, Bq, C, args, sms, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD, false, true>(Aq, Bq, C, args, sms, stream);
     default: return PURO_ERR_LAYOUT;
   }
 }

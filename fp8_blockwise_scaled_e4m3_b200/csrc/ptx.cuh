@@ -51,6 +51,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is suspended
+// until it completes or about `hint_ns` pass, instead of returning at once to poll again
+// (a polling thread takes issue slots from the warps that share its SM sub-partition).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// As mbar_wait below, but each poll may suspend the thread for up to `hint_ns`.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                                const volatile int *abort, uint32_t hint_ns) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
+    if ((it & 15u) == 0) {  // each poll may have slept: look at the clock more often
+      if (abort != nullptr && *abort) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0)
+        t0 = now;
+      else if (now - t0 > timeout_ns)
+        return false;
+    }
+  }
+  return false;
+}
+
 // Waits for the phase of parity `parity` to complete. Gives up, returning false, when
 // `*abort` becomes non-zero (another warp of the CTA gave up; `abort` may be null) or
 // after `timeout_ns` of wall time; an iteration cap backs the timer up. Never spins
@@ -295,6 +328,20 @@ __device__ __forceinline__ void tmem_ld_64cols(uint32_t taddr, uint32_t (&r)[64]
       : "r"(taddr)
       : "memory");
 }
+// 32 lanes x 32 consecutive FP32 columns: thread i of the warp gets row (lane base + i).
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
 // tcgen05.wait::ld that also names the registers of the load(s) it waits for, so the
 // compiler cannot schedule a use of them above the wait.
 __device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[64]) {

@@ -24,6 +24,12 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                           uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
                           cudaStream_t stream);
 
+// fprop / dgrad whose epilogue also writes the 1x128 quantisation of the BF16 output along
+// N: codes Cq [M, N] and scales Cs [N/128, M].
+int launch_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                                const float *Bs, uint16_t *C, uint8_t *Cq, float *Cs, int64_t M,
+                                int64_t N, int64_t K, int layout, cudaStream_t stream);
+
 // wgrad with FP32 accumulation: C[M, N] (FP32) += the wgrad product.
 int launch_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                               const float *Bs, float *C, int64_t M, int64_t N, int64_t K,

@@ -41,6 +41,7 @@ def _load():
         "puro_fp8_gemm_blockwise": [_p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p,
                                     ctypes.c_size_t, _p],
         "puro_fp8_gemm_wgrad_acc_f32": [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p],
+        "puro_fp8_gemm_blockwise_quant": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p],
         "puro_fp8_sync_status": [_p],
     }
     for name, args in sig.items():
@@ -184,6 +185,39 @@ def puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, workspace=None, stream=No
         st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_gemm_blockwise(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
                                             layout, _ptr(workspace), ws_bytes, st), "puro_fp8_gemm_blockwise", st)
+
+
+def puro_fp8_gemm_blockwise_quant(Aq, As, Bq, Bs, C, Cq, Cs, layout, stream=None):
+    """fprop / dgrad into C (bf16 [M, N]) plus the 1x128 quantisation of C along N: Cq
+    (uint8 [M, N]) and Cs (float32 [N/128, M]); see the C declaration."""
+    layout = int(LAYOUTS.get(layout, layout))
+    if layout not in (PURO_FPROP, PURO_DGRAD):
+        raise ValueError(f"layout must be fprop or dgrad, got {layout}")
+    bs_shape = {PURO_FPROP: lambda n, k: ((n + 127) // 128, k // 128),
+                PURO_DGRAD: lambda n, k: (k // 128, (n + 127) // 128)}[layout]
+    M, N, K = _gemm_shapes(Aq, As, Bq, Bs, C, bs_shape)
+    _shape(Cq, (M, N), "Cq"); _shape(Cs, (N // 128, M), "Cs")
+    _need(Aq, torch.uint8, "Aq"); _need(Bq, torch.uint8, "Bq"); _need(C, torch.bfloat16, "C")
+    _need(As, torch.float32, "As"); _need(Bs, torch.float32, "Bs")
+    _need(Cq, torch.uint8, "Cq"); _need(Cs, torch.float32, "Cs")
+    for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C"), (Cq, "Cq"), (Cs, "Cs")):
+        _dense(t, n)
+    with torch.cuda.device(Aq.device):
+        st = _stream(stream)  # the current stream of the tensors' device
+        _check(_lib.puro_fp8_gemm_blockwise_quant(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), _ptr(Cq),
+                                                  _ptr(Cs), M, N, K, layout, st),
+               "puro_fp8_gemm_blockwise_quant", st)
+
+
+def gemm_quant(Aq, As, Bq, Bs, layout, stream=None):
+    """(C bf16 [M, N], Cq uint8 [M, N], Cs float32 [N/128, M]) = the GEMM and its output's
+    1x128 quantisation from one launch (see puro_fp8_gemm_blockwise_quant)."""
+    M, N = Aq.shape[0], Bq.shape[0]
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=Aq.device)
+    Cq = torch.empty((M, N), dtype=torch.uint8, device=Aq.device)
+    Cs = torch.empty((N // 128, M), dtype=torch.float32, device=Aq.device)
+    puro_fp8_gemm_blockwise_quant(Aq, As, Bq, Bs, C, Cq, Cs, layout, stream)
+    return C, Cq, Cs
 
 
 def puro_fp8_gemm_wgrad_acc_f32(Aq, As, Bq, Bs, C, stream=None):

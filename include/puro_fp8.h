@@ -148,6 +148,31 @@ PURO_API int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const u
                             puro_stream_t stream);
 
 /*
+ * fprop or dgrad whose epilogue also quantises its own output for the next GEMM:
+ *     C = the PURO_FPROP / PURO_DGRAD product of puro_fp8_gemm_blockwise (BF16), and
+ *     Cq, Cs = the 1x128 quantisation of that BF16 C along N, exactly what
+ *              puro_fp8_quantize_1x128(C, ...) with ldq = N would write from it.
+ * Source: "Lever 2: use blockwise FP8 from step zero" -- tensors are converted to FP8 only
+ * for the GEMM that consumes them, in groups of 128 along its reduction dimension. When
+ * the output feeds another linear layer as its input, that dimension is this GEMM's N,
+ * and each thread of the epilogue already holds one output row x 128 columns: the group's
+ * amax, scale and codes are formed from the BF16 values in its registers, so the BF16
+ * output is not read back by a separate quantiser pass.
+ *
+ *   Aq, As, Bq, Bs, M, N, K, layout   as for puro_fp8_gemm_blockwise (PURO_FPROP or
+ *                                     PURO_DGRAD only; PURO_ERR_LAYOUT otherwise)
+ *   C   [M, N] BF16, dense            output
+ *   Cq  [M, N] E4M3 codes, dense      output
+ *   Cs  [N/128, M] float, dense       output; Cs[j*M + m] is the scale of C[m, 128j .. +127]
+ * Requires M >= 1, N >= 128, N % 128 == 0, K >= 128, K % 128 == 0; Aq, Bq, C, Cq 16-byte
+ * aligned; As, Bs, Cs 4-byte aligned. Status codes as for puro_fp8_gemm_blockwise.
+ */
+PURO_API int puro_fp8_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                                           const float *Bs, uint16_t *C, uint8_t *Cq, float *Cs,
+                                           int64_t M, int64_t N, int64_t K, int layout,
+                                           puro_stream_t stream);
+
+/*
  * Weight gradient with FP32 accumulation:
  *     C[m, n] += sum_kb sA(kb, m) * sB(kb, n) * sum_{k in kb} A[m, k] B[n, k]
  * the PURO_WGRAD product of puro_fp8_gemm_blockwise (same operands, same FP32 promotion),

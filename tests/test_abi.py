@@ -43,8 +43,8 @@ def exported_symbols(path):
 def test_header_declares_the_entry_points():
     assert declared_functions() == sorted([
         "puro_fp8_quantize_1x128", "puro_fp8_quantize_1x128_transposed", "puro_fp8_quantize_128x128",
-        "puro_fp8_gemm_blockwise", "puro_fp8_gemm_wgrad_acc_f32", "puro_fp8_sync_status",
-        "puro_strerror"])
+        "puro_fp8_gemm_blockwise", "puro_fp8_gemm_wgrad_acc_f32", "puro_fp8_gemm_blockwise_quant",
+        "puro_fp8_sync_status", "puro_strerror"])
 
 
 def test_library_exports_exactly_the_declared_symbols(lib):
@@ -193,3 +193,20 @@ def test_binding_refuses_tensors_of_the_wrong_shape(lib):
     for call, what in cases:
         with pytest.raises(ValueError, match=what):
             call()
+
+
+def test_gemm_quant_rejects_bad_arguments(lib):
+    """The fused-quantisation GEMM: fprop / dgrad only, N a multiple of 128 (the groups run
+    along N), every output present and aligned; all checked before any launch."""
+    f = lib.puro_fp8_gemm_blockwise_quant
+    ops = [A16, A16, A16, A16, A16, A16, A16]
+    assert f(None, *ops[1:], 128, 256, 256, 0, None) == ENULL
+    assert f(*ops[:5], None, A16, 128, 256, 256, 0, None) == ENULL      # Cq
+    assert f(*ops[:6], None, 128, 256, 256, 0, None) == ENULL           # Cs
+    assert f(*ops, 128, 256, 256, 2, None) == ELAYOUT                   # wgrad has no fused form
+    assert f(*ops, 128, 256, 256, 7, None) == ELAYOUT
+    assert f(*ops, 128, 200, 256, 0, None) == ESHAPE                    # N % 128
+    assert f(*ops, 0, 256, 256, 1, None) == ESHAPE
+    assert f(*ops, 128, 256, 200, 0, None) == ESHAPE                    # K % 128
+    assert f(*ops[:5], A16 + 8, A16, 128, 256, 256, 0, None) == EALIGN  # Cq not 16-byte aligned
+    assert f(*ops[:6], A16 + 2, 128, 256, 256, 0, None) == EALIGN       # Cs not 4-byte aligned
