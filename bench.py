@@ -57,10 +57,13 @@ def _args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-group", action="store_true",
+                   help="one wgrad launch per linear instead of one grouped launch per block")
     p.add_argument("--config", default="5",
                    help="workload: 1 small outlier GEMM, 2 one layer's forward linears, 3 its backward, "
                         "4 the LM head, 5 the full 28-layer step (default), 'all' for 1-4 then 5, or "
-                        "'fused' for the fused epilogue quantisation against GEMM + separate quantiser")
+                        "'fused' for the fused epilogue quantisation against GEMM + separate quantiser, "
+                        "'grouped' for one block's four wgrads in one launch against four")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions of configs 1-4")
     return p.parse_args()
 
@@ -188,7 +191,7 @@ class Clocks:
 class Step:
     """All buffers of one micro-step and the sequence of library calls over them."""
 
-    def __init__(self, pf, wl, tokens, layers, device, seed):
+    def __init__(self, pf, wl, tokens, layers, device, seed, group_wgrad=True):
         import torch
         self.pf, self.torch = pf, torch
         T = tokens
@@ -238,9 +241,11 @@ class Step:
             gb += T * n + n * k + 4 * (T * n // 128 + (n // 128) * (k // 128)) + 2 * T * k   # dgrad
             gb += n * T + k * T + 4 * (n + k) * (T // 128) + 2 * n * k                      # wgrad
         self.gemm_bytes = gb
-        self.gemm_launches = 3 * len(self.linears)
+        self.group_wgrad = group_wgrad
+        n_wgrad = len({self.layer_of(i) for i in range(len(self.linears))}) if group_wgrad else len(self.linears)
+        self.gemm_launches = 2 * len(self.linears) + n_wgrad
         self.quant_launches = 3 * len(self.linears)
-        self.launches_per_step = 6 * len(self.linears)
+        self.launches_per_step = self.gemm_launches + self.quant_launches
 
     def run(self, ev=None, stream=None, overlap=False, before_fwd=None, before_bwd=None,
             before_wgrad=None, after_wgrad=None):
@@ -284,8 +289,41 @@ class Step:
                 main.wait_event(w_ready[i])
             pf.puro_fp8_gemm_blockwise(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, None, main); rec("g")
         wgrad_done = {}  # per shape: the last wgrad that read the shape's token-dim operands
+        pending = []     # this layer's linears whose dY is quantised and whose wgrad is not issued
+
+        def issue_wgrads():
+            # One launch for a layer's wgrads (grouped mode), else one per linear.
+            if not pending:
+                return
+            if overlap:
+                side.wait_stream(main)  # every pending dY quantisation is done
+            for i in pending:
+                if before_wgrad is not None:
+                    before_wgrad(i, side)
+            with torch.cuda.stream(side):
+                probs = []
+                for i in pending:
+                    _, x, w, dy, wq, wqt, ws, xqt, xst = self.linears[i]
+                    s = self.scratch[tuple(w.shape)]
+                    probs.append((s["dyqt"], s["dyst"], xqt, xst, s["dw"]))
+                if self.group_wgrad and len(probs) > 1:
+                    pf.puro_fp8_gemm_blockwise_grouped(probs, pf.PURO_WGRAD, side); rec("g")
+                else:
+                    for pr in probs:
+                        pf.puro_fp8_gemm_blockwise(*pr, pf.PURO_WGRAD, None, side); rec("g")
+                if after_wgrad is not None:
+                    for i, pr in zip(pending, probs):
+                        after_wgrad(i, pr[4], side)
+            if overlap:
+                done = side.record_event()
+                for i in pending:
+                    wgrad_done[tuple(self.linears[i][2].shape)] = done
+            pending.clear()
+
         for i in range(len(self.linears) - 1, -1, -1):
             tag, x, w, dy, wq, wqt, ws, xqt, xst = self.linears[i]
+            if pending and self.layer_of(pending[-1]) != self.layer_of(i):
+                issue_wgrads()
             key = tuple(w.shape)
             s = self.scratch[key]
             if before_bwd is not None:
@@ -293,21 +331,17 @@ class Step:
             if overlap and key in wgrad_done:
                 main.wait_event(wgrad_done[key])  # the quantiser below overwrites its dY operands
             pf.puro_fp8_quantize_1x128_transposed(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], main); rec("q")
-            q_ready = main.record_event() if overlap else None
             pf.puro_fp8_gemm_blockwise(s["dyq"], s["dys"], wqt, ws, s["dx"], pf.PURO_DGRAD, None, main); rec("g")
-            if overlap:
-                side.wait_event(q_ready)
-            if before_wgrad is not None:
-                before_wgrad(i, side)
-            with torch.cuda.stream(side):
-                pf.puro_fp8_gemm_blockwise(s["dyqt"], s["dyst"], xqt, xst, s["dw"], pf.PURO_WGRAD, None,
-                                           side); rec("g")
-                if after_wgrad is not None:
-                    after_wgrad(i, s["dw"], side)
-            if overlap:
-                wgrad_done[key] = side.record_event()
+            pending.append(i)
+            if not self.group_wgrad:
+                issue_wgrads()
+        issue_wgrads()
         if overlap:
             main.wait_stream(side)
+
+    def layer_of(self, i):
+        """The block a linear belongs to (its tag's prefix; the LM head is its own)."""
+        return self.linears[i][0].split(".")[0]
 
 
 def _record(torch):
@@ -428,7 +462,7 @@ def run_ours(args):
     device = torch.device("cuda", torch.cuda.current_device())
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
 
-    step = Step(pf, wl, args.tokens, args.layers, device, seed=4 + 1000 * rank)
+    step = Step(pf, wl, args.tokens, args.layers, device, seed=4 + 1000 * rank, group_wgrad=not args.no_group)
     stream = torch.cuda.current_stream()
 
     clocks = Clocks(torch.cuda.current_device())
@@ -593,9 +627,9 @@ def main():
     if args.impl == "reference":
         run_reference(args)
         return
-    if args.config == "fused":
-        from bench_configs import run_fused_comparison
-        run_fused_comparison(args)
+    if args.config in ("fused", "grouped"):
+        import bench_configs
+        {"fused": bench_configs.run_fused_comparison, "grouped": bench_configs.run_grouped_comparison}[args.config](args)
         return
     if args.config in ("1", "2", "3", "4", "all"):
         from bench_configs import run_config

@@ -323,3 +323,49 @@ def run_fused_comparison(args):
                       "l2": "flushed before every repetition", "reps": args.reps,
                       "total_separate_us": round(tot_sep, 1), "total_fused_us": round(tot_fus, 1),
                       "saved_pct": round(100 * (1 - tot_fus / tot_sep), 1), "ops": rows}), flush=True)
+
+
+def run_grouped_comparison(args):
+    """The four weight gradients of one Qwen3-1.7B-shaped block at 8192 tokens: four
+    puro_fp8_gemm_blockwise launches against one puro_fp8_gemm_blockwise_grouped launch.
+    Same operands, L2 flushed before every repetition, median over repetitions."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    T = 8192
+    fwd = wl.layer_forward(4, T, dev, layer=0)
+    grads = wl.layer_grads(4, T, dev, layer=0)
+    problems = []
+    flops = 0.0
+    for (name, x, w), (_, dy) in zip(fwd, grads):
+        dyt, dyst = pf.quantize_1x128_transposed(dy)
+        xt, xst = pf.quantize_1x128_transposed(x)
+        problems.append((dyt, dyst, xt, xst, torch.empty(w.shape, dtype=torch.bfloat16, device=dev)))
+        flops += 2.0 * w.shape[0] * w.shape[1] * T
+    flush = torch.empty(512 * 2 ** 20 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def separate(st):
+        for pr in problems:
+            pf.puro_fp8_gemm_blockwise(*pr, pf.PURO_WGRAD, None, st)
+
+    def grouped(st):
+        pf.puro_fp8_gemm_blockwise_grouped(problems, pf.PURO_WGRAD, st)
+
+    t = {"separate": [], "grouped": []}
+    for rep in range(args.warmup + args.reps):
+        for kind, fn in (("separate", separate), ("grouped", grouped)):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(stream)
+            e1.record(stream)
+            e1.synchronize()
+            if rep >= args.warmup:
+                t[kind].append(e0.elapsed_time(e1))
+    pf.puro_fp8_sync_status()
+    sep, grp = statistics.median(t["separate"]), statistics.median(t["grouped"])
+    print(json.dumps({"comparison": "four wgrad launches vs one grouped launch",
+                      "workload": "wgrads of one Qwen3-1.7B-shaped block (QKV, O, gate/up, down) at 8192 tokens, seed 4",
+                      "l2": "flushed before every repetition", "reps": args.reps,
+                      "separate_us": round(sep * 1e3, 1), "grouped_us": round(grp * 1e3, 1),
+                      "separate_tflops": round(flops / sep / 1e9, 1), "grouped_tflops": round(flops / grp / 1e9, 1),
+                      "saved_pct": round(100 * (1 - grp / sep), 1)}), flush=True)

@@ -80,11 +80,9 @@ int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t l
   return puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, S, stream);
 }
 
-int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
-                            const float *Bs, uint16_t *C, int64_t M, int64_t N, int64_t K,
-                            int layout, void *workspace, size_t ws_bytes, puro_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
+// The checks of one GEMM's arguments (every layout); PURO_OK or the status to return.
+int check_gemm(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs, const void *C,
+               int64_t M, int64_t N, int64_t K, int layout) {
   if (Aq == nullptr || As == nullptr || Bq == nullptr || Bs == nullptr || C == nullptr)
     return PURO_ERR_NULL;
   if (layout != PURO_FPROP && layout != PURO_DGRAD && layout != PURO_WGRAD)
@@ -96,8 +94,32 @@ int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *B
   if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16) || !aligned(As, 4) ||
       !aligned(Bs, 4))
     return PURO_ERR_ALIGN;
+  return PURO_OK;
+}
+
+int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
+                            const float *Bs, uint16_t *C, int64_t M, int64_t N, int64_t K,
+                            int layout, void *workspace, size_t ws_bytes, puro_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  if (int e = check_gemm(Aq, As, Bq, Bs, C, M, N, K, layout)) return e;
   if (int d = check_device()) return d;
   return puro::launch_gemm_blockwise(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
+}
+
+int puro_fp8_gemm_blockwise_grouped(const puro_gemm_problem *problems, int count, int layout,
+                                    puro_stream_t stream) {
+  if (problems == nullptr) return PURO_ERR_NULL;
+  if (count < 1 || count > PURO_GROUP_MAX) return PURO_ERR_SHAPE;
+  int64_t tiles = 0;
+  for (int p = 0; p < count; ++p) {
+    const puro_gemm_problem &g = problems[p];
+    if (int e = check_gemm(g.Aq, g.As, g.Bq, g.Bs, g.C, g.M, g.N, g.K, layout)) return e;
+    tiles += ((g.M + 127) / 128) * ((g.N + 255) / 256);
+  }
+  if (tiles > (1ll << 31) - (1ll << 16)) return PURO_ERR_SHAPE;
+  if (int d = check_device()) return d;
+  return puro::launch_gemm_blockwise_grouped(problems, count, layout, stream);
 }
 
 int puro_fp8_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_t *Bq,

@@ -121,6 +121,9 @@ struct TileFor {
   static constexpr int TN = 256;
 };
 
+// One GEMM of a launch. A launch serves up to G of them (the same layout): their tiles are
+// numbered one after the other, problem p owning tiles [tile_begin, tile_begin + num_m *
+// num_n), and the persistent CTAs walk that joint sequence.
 struct GemmArgs {
   const float *As;
   const float *Bs;
@@ -129,11 +132,24 @@ struct GemmArgs {
   int num_m, num_n, kblocks, m_fastest;
   int vec_a;  // As rows are 16-byte aligned (As aligned, M % 4 == 0): 16-byte scale copies
   int vec_b;  // wgrad: Bs rows are 16-byte aligned (Bs aligned; N % 8 == 0 always)
-  unsigned long long timeout_ns;
-  int *status;
   uint8_t *Cq;  // QOUT: 1x128 codes of the BF16 output along N, [M, N] dense
   float *Cs;    // QOUT: their scales, [N/128, M]
+  int tile_begin;
 };
+
+// Kernel parameters: the problems' tensor maps (A, B and C of problem p at index p) and
+// arguments, passed by value as a __grid_constant__ (the TMA unit reads the maps from the
+// parameter space).
+template <int G>
+struct alignas(64) GemmParams {
+  CUtensorMap tmA[G], tmB[G], tmC[G];
+  GemmArgs prob[G];
+  int count;  // problems in use
+  int tiles;  // tiles of all problems
+  unsigned long long timeout_ns;
+  int *status;
+};
+constexpr int GROUP_MAX = 4;  // problems per grouped launch
 
 __device__ int g_status;  // non-zero: a bounded wait gave up since the last read
 
@@ -148,6 +164,10 @@ __device__ int g_test_skip_release;
 #define PURO_SKIP_RELEASE(use) false
 #endif
 
+// Problem p of global tile `tile` and the tile's coordinates within that problem.
+template <int G>
+__device__ __forceinline__ int locate_tile(int tile, const GemmParams<G> &prm, int &mt, int &nt);
+
 __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mt, int &nt) {
   if (a.m_fastest) {
     mt = tile % a.num_m;
@@ -156,6 +176,15 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmArgs &a, int &mt
     nt = tile % a.num_n;
     mt = tile / a.num_n;
   }
+}
+
+template <int G>
+__device__ __forceinline__ int locate_tile(int tile, const GemmParams<G> &prm, int &mt, int &nt) {
+  int p = 0;  // problems are numbered in tile order: count the ones that begin at or before `tile`
+#pragma unroll
+  for (int q = 1; q < G; ++q) p += (q < prm.count && tile >= prm.prob[q].tile_begin) ? 1 : 0;
+  tile_coords(tile - prm.prob[p].tile_begin, prm.prob[p], mt, nt);
+  return p;
 }
 
 __device__ __forceinline__ void raise_abort(volatile int *abort, int *status) {
@@ -174,10 +203,9 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 // a promotion thread holds one output row x 128 columns, exactly one group, so the group's
 // amax, scale and codes come from the thread's own registers (the same arithmetic as the
 // separate 1x128 quantiser, applied to the same BF16 values).
-template <int LAYOUT, int TN, bool ACC32, bool PAIR, bool QOUT>
+template <int LAYOUT, int TN, bool ACC32, bool PAIR, bool QOUT, int G>
 __global__ void __launch_bounds__(THREADS, 1)
-    k_gemm_blockwise(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+    k_gemm_blockwise(const __grid_constant__ GemmParams<G> prm) {
   using C = Cfg<LAYOUT, TN, PAIR>;
   constexpr int BN = C::BN, NBUF = C::NBUF, STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
@@ -229,10 +257,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-    prefetch_tensormap(&tmC);
+  if (warp == 0 && lane < prm.count) {
+    prefetch_tensormap(&prm.tmA[lane]);
+    prefetch_tensormap(&prm.tmB[lane]);
+    prefetch_tensormap(&prm.tmC[lane]);
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -251,9 +279,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
-  const int tiles = args.num_m * args.num_n;
-  const int kblocks = args.kblocks;
-  const uint64_t tmo = args.timeout_ns;
+  const int tiles = prm.tiles;
+  const uint64_t tmo = prm.timeout_ns;
 
   if (warp < EPI_FIRST_WARP) {
     // Each role's code sits inside the branch that set its register limit, so ptxas
@@ -268,7 +295,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
         int mt, nt;
-        tile_coords(tile, args, mt, nt);
+        const int p = locate_tile(tile, prm, mt, nt);
+        const CUtensorMap *tmA = &prm.tmA[p];
+        const CUtensorMap *tmB = &prm.tmB[p];
+        const int kblocks = prm.prob[p].kblocks;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(empty_bar(s), ph ^ 1u, tmo, abort)) {
             ok = false;
@@ -281,13 +311,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             // it never lands in the leader's barrier before the previous phase is over.
             const uint32_t fb = map_to_rank(full_bar(s), 0);
             if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (A_BYTES + B_BYTES));
-            tma_load_2d_pair(sbase + OFF_A + s * A_BYTES, &tmA, fb, kb * BK, row_base(mt));
-            tma_load_2d_pair(sbase + OFF_B + s * B_BYTES, &tmB, fb, kb * BK,
+            tma_load_2d_pair(sbase + OFF_A + s * A_BYTES, tmA, fb, kb * BK, row_base(mt));
+            tma_load_2d_pair(sbase + OFF_B + s * B_BYTES, tmB, fb, kb * BK,
                              nt * BN + static_cast<int>(rank) * C::B_ROWS);
           } else {
             mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
-            tma_load_2d(sbase + OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
-            tma_load_2d(sbase + OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
+            tma_load_2d(sbase + OFF_A + s * A_BYTES, tmA, full_bar(s), kb * BK, mt * BM);
+            tma_load_2d(sbase + OFF_B + s * B_BYTES, tmB, full_bar(s), kb * BK, nt * BN);
           }
           issued |= 1u << s;
           issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
@@ -295,7 +325,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (!ok) {
-        raise_abort(abort, args.status);
+        raise_abort(abort, prm.status);
         // Let every issued tensor load land before the CTA can exit. (A peer's loads are
         // counted on the leader's barriers, which the leader drains; the peer stays alive
         // until then through the cluster barrier at the end of the kernel.)
@@ -312,6 +342,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t use = 0;                            // K blocks of this CTA so far, both issuers
       bool ok = true;
       for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
+        int mt, nt;
+        const int kblocks = prm.prob[locate_tile(tile, prm, mt, nt)].kblocks;
         for (int kb = 0; kb < kblocks; ++kb, ++use) {
           if ((use & 1u) != mine) continue;
           const int s = static_cast<int>(use % STAGES);
@@ -347,7 +379,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (!ok) {
-        raise_abort(abort, args.status);
+        raise_abort(abort, prm.status);
         // arrives once every MMA this thread issued has finished
         if constexpr (PAIR)
           mma_commit_pair(drain_bar(mine));
@@ -359,13 +391,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale loader
     // Scales outside the matrix are zero-filled, so the promotion needs no bounds checks.
-    const int nb_total = (args.N + 127) / 128;
     int ss = 0;
     uint32_t sph = 0;
     bool ok = true;
     for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
       int mt, nt;
-      tile_coords(tile, args, mt, nt);
+      const GemmArgs &args = prm.prob[locate_tile(tile, prm, mt, nt)];
+      const int kblocks = args.kblocks;
+      const int nb_total = (args.N + 127) / 128;
       const int m_first = row_base(mt);
       for (int kb0 = 0; kb0 < kblocks; kb0 += KPS) {
         if (!mbar_wait(sempty_bar(ss), sph ^ 1u, tmo, abort)) {
@@ -422,7 +455,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (++ss == SC_STAGES) ss = 0, sph ^= 1u;
       }
     }
-    if (!ok) raise_abort(abort, args.status);
+    if (!ok) raise_abort(abort, prm.status);
     cp_async_wait_all();  // no copy may land after the CTA has exited
   }
   } else {
@@ -440,10 +473,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     // PAIR: the TMEM buffer goes back to the leader's MMA issuer, which waits for both CTAs
     const uint32_t tempty_target0 = PAIR ? map_to_rank(tempty_bar(0), 0) : tempty_bar(0);
     for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
-      int mt, nt;
-      tile_coords(tile, args, mt, nt);
-      const int n_base = nt * BN + half * WCOLS;  // first column of this warp
-      const int m_first = row_base(mt);
+      int kblocks;
+      {
+        int mt, nt;
+        kblocks = prm.prob[locate_tile(tile, prm, mt, nt)].kblocks;
+      }
       uint64_t acc[WCOLS / 2];
 #pragma unroll
       for (int i = 0; i < WCOLS / 2; ++i) acc[i] = 0;
@@ -579,6 +613,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (!ok) break;
+      // The tile's problem and position, looked up again only now (registers are scarce
+      // during the K loop).
+      int mt, nt;
+      const int p = locate_tile(tile, prm, mt, nt);
+      const GemmArgs &args = prm.prob[p];
+      const CUtensorMap *tmC = &prm.tmC[p];
+      const int m_first = row_base(mt);
+      const int n_base = nt * BN + half * WCOLS;  // first column of this warp
       // Stage this warp's 32 rows x WCOLS columns as BF16 (64-column boxes, 16-byte
       // chunk c of row r at chunk position c ^ (r % 8)) and store them with the TMA unit.
       const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST_WARP) * C::STG_WARP_BYTES;
@@ -620,7 +662,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
               for (int bb = 0; bb < 2; ++bb) {
                 const int col = n_base + 32 * (2 * h + bb);
-                if (col < args.N) tma_reduce_add_2d(&tmC, stg + bb * STG_BOX_BYTES, col, row0);
+                if (col < args.N) tma_reduce_add_2d(tmC, stg + bb * STG_BOX_BYTES, col, row0);
               }
             }
             bulk_commit_group();
@@ -702,14 +744,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int box = 0; box < WCOLS / 64; ++box)
             if (n_base + 64 * box < args.N)
-              tma_store_2d(&tmC, stg + box * STG_BOX_BYTES, n_base + 64 * box, row0);
+              tma_store_2d(tmC, stg + box * STG_BOX_BYTES, n_base + 64 * box, row0);
         }
         bulk_commit_group();
       }
       }  // BF16 store
     }
     if (lane == 0) bulk_wait_group_all();  // stores complete before the CTA exits
-    if (!ok) raise_abort(abort, args.status);
+    if (!ok) raise_abort(abort, prm.status);
   }
 
   tc_fence_before_sync();
@@ -794,28 +836,64 @@ bool use_pair(int64_t M) {
   return M > BM;
 }
 
-template <int LAYOUT, bool ACC32, bool PAIR, bool QOUT>
-int launch_kernel(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
-                  cudaStream_t stream) {
+// One GEMM as the host hands it over: operands, outputs and sizes.
+struct HostProblem {
+  const uint8_t *Aq, *Bq;
+  const float *As, *Bs;
+  void *C;                // BF16 [M, N], or FP32 for ACC32
+  uint8_t *Cq;            // QOUT only
+  float *Cs;              // QOUT only
+  int64_t M, N, K;
+};
+
+template <int LAYOUT, bool ACC32, bool PAIR, bool QOUT, int G>
+int launch_kernel(const HostProblem *probs, int count, int sms, cudaStream_t stream) {
   constexpr int TN = TileFor<LAYOUT, PAIR>::TN;
   using CF = Cfg<LAYOUT, TN, PAIR>;
   constexpr int SMEM_BYTES = CF::SMEM_BYTES;
-  const int64_t M = args.M, N = args.N, K = args.K;
-  CUtensorMap ta, tb, tc;
-  if (!make_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK,
-                CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, CF::B_ROWS, BK,
-                CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !(ACC32 ? make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, N, 32, 32,
-                         CU_TENSOR_MAP_SWIZZLE_128B)
-              : make_map(&tc, Cout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64,
-                         CU_TENSOR_MAP_SWIZZLE_128B)))
-    return PURO_ERR_CUDA;
+  static_assert(sizeof(GemmParams<G>) <= 32000, "kernel parameters");
+  GemmParams<G> prm{};
+  int *status = device_status_ptr();
+  if (status == nullptr) return PURO_ERR_CUDA;
+  prm.count = count;
+  prm.timeout_ns = wait_timeout_ns();
+  prm.status = status;
   const int tile_rows = PAIR ? 2 * BM : BM;
-  args.num_m = static_cast<int>((M + tile_rows - 1) / tile_rows);
-  args.num_n = static_cast<int>((N + TN - 1) / TN);
-  const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
-  auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32, PAIR, QOUT>;
+  int64_t tiles = 0;
+  for (int p = 0; p < count; ++p) {
+    const HostProblem &h = probs[p];
+    if (!make_map(&prm.tmA[p], h.Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.M, h.K, BM, BK,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&prm.tmB[p], h.Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, h.N, h.K, CF::B_ROWS, BK,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !(ACC32 ? make_map(&prm.tmC[p], h.C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, h.M, h.N, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_128B)
+                : make_map(&prm.tmC[p], h.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h.M, h.N, 32, 64,
+                           CU_TENSOR_MAP_SWIZZLE_128B)))
+      return PURO_ERR_CUDA;
+    GemmArgs &a = prm.prob[p];
+    a.As = h.As;
+    a.Bs = h.Bs;
+    a.C = static_cast<uint16_t *>(h.C);
+    a.Cq = h.Cq;
+    a.Cs = h.Cs;
+    a.M = static_cast<int>(h.M);
+    a.N = static_cast<int>(h.N);
+    a.K = static_cast<int>(h.K);
+    a.kblocks = static_cast<int>(h.K / BK);
+    // Walk the smaller operand fastest so that it stays resident in L2 while the larger
+    // one streams through once.
+    a.m_fastest = h.M <= h.N ? 1 : 0;
+    a.vec_a = (reinterpret_cast<uintptr_t>(h.As) % 16 == 0 && h.M % 4 == 0) ? 1 : 0;
+    a.vec_b = (reinterpret_cast<uintptr_t>(h.Bs) % 16 == 0) ? 1 : 0;  // used by wgrad only
+    a.num_m = static_cast<int>((h.M + tile_rows - 1) / tile_rows);
+    a.num_n = static_cast<int>((h.N + TN - 1) / TN);
+    a.tile_begin = static_cast<int>(tiles);
+    tiles += static_cast<int64_t>(a.num_m) * a.num_n;
+  }
+  if (tiles > (1ll << 31) - (1ll << 16)) return PURO_ERR_SHAPE;
+  prm.tiles = static_cast<int>(tiles);
+  auto kern = k_gemm_blockwise<LAYOUT, TN, ACC32, PAIR, QOUT, G>;
   // Once per device: the register split inside the kernel assumes exactly LAUNCH_REGS per
   // thread at launch (with any other count the promotion warps' setmaxnreg.inc could wait
   // forever), the kernel needs its dynamic shared memory opted in, and a pair kernel's
@@ -879,11 +957,11 @@ int launch_kernel(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs arg
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args);
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
     if (e == cudaSuccess) e = cudaGetLastError();
   } else {
     grid = static_cast<int>(tiles < sms ? tiles : sms);
-    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, args);
+    kern<<<grid, THREADS, SMEM_BYTES, stream>>>(prm);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) {
@@ -899,38 +977,22 @@ int launch_kernel(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs arg
   return PURO_OK;
 }
 
+// Single problems (G = 1) and groups of up to GROUP_MAX, on CTA pairs unless some problem
+// has at most 128 output rows.
 template <int LAYOUT, bool ACC32, bool QOUT = false>
-int launch_layout(const uint8_t *Aq, const uint8_t *Bq, void *Cout, GemmArgs args, int sms,
-                  cudaStream_t stream) {
-  return use_pair(args.M) ? launch_kernel<LAYOUT, ACC32, true, QOUT>(Aq, Bq, Cout, args, sms, stream)
-                          : launch_kernel<LAYOUT, ACC32, false, QOUT>(Aq, Bq, Cout, args, sms, stream);
-}
-
-}  // namespace
-
-namespace {
-
-// Kernel arguments common to every launch; returns PURO_OK or an error status.
-int gemm_args(const float *As, const float *Bs, int64_t M, int64_t N, int64_t K, GemmArgs &args,
-              int &sms) {
+int launch_layout(const HostProblem *probs, int count, cudaStream_t stream) {
+  int sms = 0;
   if (!sm_count(sms)) return PURO_ERR_CUDA;
-  int *status = device_status_ptr();
-  if (status == nullptr) return PURO_ERR_CUDA;
-  args = GemmArgs{};
-  args.As = As;
-  args.Bs = Bs;
-  args.M = static_cast<int>(M);
-  args.N = static_cast<int>(N);
-  args.K = static_cast<int>(K);
-  args.kblocks = static_cast<int>(K / BK);
-  // Walk the smaller operand fastest so that it stays resident in L2 while the larger
-  // one streams through once.
-  args.m_fastest = M <= N ? 1 : 0;
-  args.vec_a = (reinterpret_cast<uintptr_t>(As) % 16 == 0 && M % 4 == 0) ? 1 : 0;
-  args.vec_b = (reinterpret_cast<uintptr_t>(Bs) % 16 == 0) ? 1 : 0;  // used by wgrad only
-  args.timeout_ns = wait_timeout_ns();
-  args.status = status;
-  return PURO_OK;
+  bool pair = true;
+  for (int p = 0; p < count; ++p) pair = pair && use_pair(probs[p].M);
+  if (count == 1)
+    return pair ? launch_kernel<LAYOUT, ACC32, true, QOUT, 1>(probs, 1, sms, stream)
+                : launch_kernel<LAYOUT, ACC32, false, QOUT, 1>(probs, 1, sms, stream);
+  if constexpr (!ACC32 && !QOUT) {
+    return pair ? launch_kernel<LAYOUT, false, true, false, GROUP_MAX>(probs, count, sms, stream)
+                : launch_kernel<LAYOUT, false, false, false, GROUP_MAX>(probs, count, sms, stream);
+  }
+  return PURO_ERR_LAYOUT;
 }
 
 }  // namespace
@@ -938,14 +1000,33 @@ int gemm_args(const float *As, const float *Bs, int64_t M, int64_t N, int64_t K,
 int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs,
                           uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
                           cudaStream_t stream) {
-  GemmArgs args;
-  int sms = 0;
-  if (int e = gemm_args(As, Bs, M, N, K, args, sms)) return e;
-  args.C = C;
+  const HostProblem h{Aq, Bq, As, Bs, C, nullptr, nullptr, M, N, K};
   switch (layout) {
-    case PURO_FPROP: return launch_layout<PURO_FPROP, false>(Aq, Bq, C, args, sms, stream);
-    case PURO_DGRAD: return launch_layout<PURO_DGRAD, false>(Aq, Bq, C, args, sms, stream);
-    case PURO_WGRAD: return launch_layout<PURO_WGRAD, false>(Aq, Bq, C, args, sms, stream);
+    case PURO_FPROP: return launch_layout<PURO_FPROP, false>(&h, 1, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD, false>(&h, 1, stream);
+    case PURO_WGRAD: return launch_layout<PURO_WGRAD, false>(&h, 1, stream);
+    default: return PURO_ERR_LAYOUT;
+  }
+}
+
+int launch_gemm_blockwise_grouped(const GroupedProblem *problems, int count, int layout,
+                                  cudaStream_t stream) {
+  if (count < 1 || count > GROUP_MAX) return PURO_ERR_SHAPE;
+  HostProblem h[GROUP_MAX];
+  for (int p = 0; p < count; ++p)
+    h[p] = HostProblem{problems[p].Aq, problems[p].Bq, problems[p].As, problems[p].Bs, problems[p].C,
+                       nullptr, nullptr, problems[p].M, problems[p].N, problems[p].K};
+  // The longest tiles (most K blocks) first, so the shorter ones fill the last wave.
+  for (int a = 1; a < count; ++a)
+    for (int b = a; b > 0 && h[b].K > h[b - 1].K; --b) {
+      const HostProblem t = h[b];
+      h[b] = h[b - 1];
+      h[b - 1] = t;
+    }
+  switch (layout) {
+    case PURO_FPROP: return launch_layout<PURO_FPROP, false>(h, count, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD, false>(h, count, stream);
+    case PURO_WGRAD: return launch_layout<PURO_WGRAD, false>(h, count, stream);
     default: return PURO_ERR_LAYOUT;
   }
 }
@@ -953,15 +1034,10 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
 int launch_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                                 const float *Bs, uint16_t *C, uint8_t *Cq, float *Cs, int64_t M,
                                 int64_t N, int64_t K, int layout, cudaStream_t stream) {
-  GemmArgs args;
-  int sms = 0;
-  if (int e = gemm_args(As, Bs, M, N, K, args, sms)) return e;
-  args.C = C;
-  args.Cq = Cq;
-  args.Cs = Cs;
+  const HostProblem h{Aq, Bq, As, Bs, C, Cq, Cs, M, N, K};
   switch (layout) {
-    case PURO_FPROP: return launch_layout<PURO_FPROP, false, true>(Aq, Bq, C, args, sms, stream);
-    case PURO_DGRAD: return launch_layout<PURO_DGRAD, false, true>(Aq, Bq, C, args, sms, stream);
+    case PURO_FPROP: return launch_layout<PURO_FPROP, false, true>(&h, 1, stream);
+    case PURO_DGRAD: return launch_layout<PURO_DGRAD, false, true>(&h, 1, stream);
     default: return PURO_ERR_LAYOUT;
   }
 }
@@ -969,10 +1045,8 @@ int launch_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_
 int launch_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                               const float *Bs, float *C, int64_t M, int64_t N, int64_t K,
                               cudaStream_t stream) {
-  GemmArgs args;
-  int sms = 0;
-  if (int e = gemm_args(As, Bs, M, N, K, args, sms)) return e;
-  return launch_layout<PURO_WGRAD, true>(Aq, Bq, C, args, sms, stream);
+  const HostProblem h{Aq, Bq, As, Bs, C, nullptr, nullptr, M, N, K};
+  return launch_layout<PURO_WGRAD, true>(&h, 1, stream);
 }
 
 int read_and_clear_device_status(cudaStream_t stream, int *status_out) {

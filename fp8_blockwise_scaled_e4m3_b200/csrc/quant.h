@@ -6,6 +6,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include "../../include/puro_fp8.h"
+
 namespace puro {
 
 // Quantiser launchers; return 0 or a negative puro_status.
@@ -23,6 +25,11 @@ int read_and_clear_quant_status(cudaStream_t stream, int *status_out);
 int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq, const float *Bs,
                           uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
                           cudaStream_t stream);
+
+// Up to 8 GEMMs of one layout in one persistent launch (see puro_fp8_gemm_blockwise_grouped).
+using GroupedProblem = puro_gemm_problem;
+int launch_gemm_blockwise_grouped(const GroupedProblem *problems, int count, int layout,
+                                  cudaStream_t stream);
 
 // fprop / dgrad whose epilogue also writes the 1x128 quantisation of the BF16 output along
 // N: codes Cq [M, N] and scales Cs [N/128, M].

@@ -23,6 +23,15 @@ _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
 
 
+GROUP_MAX = 4  # PURO_GROUP_MAX
+
+
+class GemmProblem(ctypes.Structure):
+    """puro_gemm_problem: one GEMM of a grouped launch."""
+    _fields_ = [("Aq", _p), ("As", _p), ("Bq", _p), ("Bs", _p), ("C", _p),
+                ("M", _i64), ("N", _i64), ("K", _i64)]
+
+
 class PuroError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -42,6 +51,7 @@ def _load():
                                     ctypes.c_size_t, _p],
         "puro_fp8_gemm_wgrad_acc_f32": [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p],
         "puro_fp8_gemm_blockwise_quant": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p],
+        "puro_fp8_gemm_blockwise_grouped": [_p, ctypes.c_int, ctypes.c_int, _p],
         "puro_fp8_sync_status": [_p],
     }
     for name, args in sig.items():
@@ -185,6 +195,34 @@ def puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, workspace=None, stream=No
         st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_gemm_blockwise(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K,
                                             layout, _ptr(workspace), ws_bytes, st), "puro_fp8_gemm_blockwise", st)
+
+
+def puro_fp8_gemm_blockwise_grouped(problems, layout, stream=None):
+    """problems: sequence of (Aq, As, Bq, Bs, C) tensor tuples, each checked as for
+    puro_fp8_gemm_blockwise; all run in one launch (see the C declaration)."""
+    layout = int(LAYOUTS.get(layout, layout))
+    if layout not in (PURO_FPROP, PURO_DGRAD, PURO_WGRAD):
+        raise ValueError(f"unknown layout {layout}")
+    if not 1 <= len(problems) <= GROUP_MAX:
+        raise ValueError(f"1 to {GROUP_MAX} problems per grouped launch, got {len(problems)}")
+    bs_shape = {PURO_FPROP: lambda n, k: ((n + 127) // 128, k // 128),
+                PURO_DGRAD: lambda n, k: (k // 128, (n + 127) // 128),
+                PURO_WGRAD: lambda n, k: (k // 128, n)}[layout]
+    arr = (GemmProblem * len(problems))()
+    dev = problems[0][0].device
+    for i, (Aq, As, Bq, Bs, C) in enumerate(problems):
+        M, N, K = _gemm_shapes(Aq, As, Bq, Bs, C, bs_shape)
+        _need(Aq, torch.uint8, "Aq"); _need(Bq, torch.uint8, "Bq"); _need(C, torch.bfloat16, "C")
+        _need(As, torch.float32, "As"); _need(Bs, torch.float32, "Bs")
+        for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C")):
+            _dense(t, n)
+            if t.device != dev:
+                raise ValueError("all problems of a group must be on one device")
+        arr[i] = GemmProblem(Aq.data_ptr(), As.data_ptr(), Bq.data_ptr(), Bs.data_ptr(), C.data_ptr(), M, N, K)
+    with torch.cuda.device(dev):
+        st = _stream(stream)  # the current stream of the tensors' device
+        _check(_lib.puro_fp8_gemm_blockwise_grouped(ctypes.cast(arr, _p), len(problems), layout, st),
+               "puro_fp8_gemm_blockwise_grouped", st)
 
 
 def puro_fp8_gemm_blockwise_quant(Aq, As, Bq, Bs, C, Cq, Cs, layout, stream=None):

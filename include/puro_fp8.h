@@ -147,6 +147,38 @@ PURO_API int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const u
                             int layout, void *workspace, size_t ws_bytes,
                             puro_stream_t stream);
 
+/* One GEMM of a grouped launch: the operands and output of a puro_fp8_gemm_blockwise call. */
+typedef struct {
+  const uint8_t *Aq; /* [M, K] codes            */
+  const float *As;   /* [K/128, M] scales        */
+  const uint8_t *Bq; /* [N, K] codes            */
+  const float *Bs;   /* scales, layout-dependent */
+  uint16_t *C;       /* [M, N] BF16 output       */
+  int64_t M, N, K;
+} puro_gemm_problem;
+
+/* Largest number of problems in one puro_fp8_gemm_blockwise_grouped call. */
+enum { PURO_GROUP_MAX = 4 };
+
+/*
+ * 1 to PURO_GROUP_MAX independent GEMMs of the same layout in one persistent launch: each
+ * problem computes exactly what puro_fp8_gemm_blockwise with its arguments computes (bit for
+ * bit: same tiles, same order of additions). Source: "Lever 2: use blockwise FP8 from step
+ * zero" (the linear-layer GEMMs in FP8). A layer's weight gradients need only their own dY
+ * and X, so they can share one launch: the CTAs walk the problems' tiles as one sequence
+ * (the problems with the most K blocks first), and the tiles of one problem fill the SMs
+ * another problem's last wave leaves idle.
+ *
+ *   problems  host array of `count` descriptors (read during the call, not kept); every
+ *             problem obeys the requirements of puro_fp8_gemm_blockwise
+ *   count     1 .. PURO_GROUP_MAX
+ *   layout    PURO_FPROP, PURO_DGRAD or PURO_WGRAD, for every problem
+ * Outputs of different problems must not overlap. Status codes as for
+ * puro_fp8_gemm_blockwise; PURO_ERR_SHAPE also for a count outside 1 .. PURO_GROUP_MAX.
+ */
+PURO_API int puro_fp8_gemm_blockwise_grouped(const puro_gemm_problem *problems, int count, int layout,
+                                             puro_stream_t stream);
+
 /*
  * fprop or dgrad whose epilogue also quantises its own output for the next GEMM:
  *     C = the PURO_FPROP / PURO_DGRAD product of puro_fp8_gemm_blockwise (BF16), and

@@ -44,7 +44,7 @@ def test_header_declares_the_entry_points():
     assert declared_functions() == sorted([
         "puro_fp8_quantize_1x128", "puro_fp8_quantize_1x128_transposed", "puro_fp8_quantize_128x128",
         "puro_fp8_gemm_blockwise", "puro_fp8_gemm_wgrad_acc_f32", "puro_fp8_gemm_blockwise_quant",
-        "puro_fp8_sync_status", "puro_strerror"])
+        "puro_fp8_gemm_blockwise_grouped", "puro_fp8_sync_status", "puro_strerror"])
 
 
 def test_library_exports_exactly_the_declared_symbols(lib):
@@ -210,3 +210,23 @@ def test_gemm_quant_rejects_bad_arguments(lib):
     assert f(*ops, 128, 256, 200, 0, None) == ESHAPE                    # K % 128
     assert f(*ops[:5], A16 + 8, A16, 128, 256, 256, 0, None) == EALIGN  # Cq not 16-byte aligned
     assert f(*ops[:6], A16 + 2, 128, 256, 256, 0, None) == EALIGN       # Cs not 4-byte aligned
+
+
+def test_gemm_grouped_rejects_bad_arguments(lib):
+    """The grouped GEMM checks the count, the layout and every problem as the single call
+    does, before anything is launched; one bad problem rejects the whole group."""
+    from fp8_blockwise_scaled_e4m3_b200.puro_fp8 import GROUP_MAX, GemmProblem
+    f = lib.puro_fp8_gemm_blockwise_grouped
+    good = GemmProblem(A16, A16, A16, A16, A16, 128, 256, 256)
+    arr = (GemmProblem * (GROUP_MAX + 1))(*([good] * (GROUP_MAX + 1)))
+    ptr = ctypes.cast(arr, ctypes.c_void_p)
+    assert f(None, 2, 0, None) == ENULL
+    assert f(ptr, 0, 0, None) == ESHAPE
+    assert f(ptr, GROUP_MAX + 1, 0, None) == ESHAPE
+    assert f(ptr, 2, 3, None) == ELAYOUT
+    arr[1] = GemmProblem(A16, A16, A16, A16, A16, 128, 250, 256)     # N % 8
+    assert f(ptr, 2, 0, None) == ESHAPE
+    arr[1] = GemmProblem(A16, A16, None, A16, A16, 128, 256, 256)    # Bq
+    assert f(ptr, 2, 2, None) == ENULL
+    arr[1] = GemmProblem(A16, A16, A16, A16, A16 + 8, 128, 256, 256)  # C not 16-byte aligned
+    assert f(ptr, 2, 1, None) == EALIGN
