@@ -34,6 +34,9 @@ Modules
                 closed forms and PyTorch's own float8_e4m3fn conversion.
 ``quant``       the 1x128, transposed 1x128 and 128x128 quantisers, pinned by
                 invariants, hand-worked fixtures and special cases.
+``mx``          the power-of-two (UE8M0) scale mode of the same groups (scale rounded up
+                to a power of two, stored as an exponent byte), pinned by its exponent
+                rule in exact rationals, a hand-worked group and nearest-value checks.
 ``gemm``        the FP64 reference contraction for the fprop / dgrad / wgrad operand
                 layouts, pinned by exact rational brute force and an exact-integer case.
 ``accounting``  parameter and FLOP accounting (C = 6ND), pinned by the numbers the
