@@ -35,49 +35,40 @@ int check_device() {
   return v;
 }
 
-}  // namespace
-
-extern "C" {
-
-int puro_fp8_quantize_1x128(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
-                            int64_t ldq, float *S, puro_stream_t stream) {
+// Argument checks of the quantisers (both scale modes); `sa` is the scales' alignment.
+int check_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, const uint8_t *Xq, int64_t ldq,
+               const void *S, uintptr_t sa) {
   if (X == nullptr || Xq == nullptr || S == nullptr) return PURO_ERR_NULL;
   if (R < 1 || C < 128 || C % 128 != 0 || ldx < C || ldq < C) return PURO_ERR_SHAPE;
   if (R > (1ll << 31) - 1 || C / 128 > 65535 || !tiles_fit(R, 128, C, 128)) return PURO_ERR_SHAPE;
-  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(S, 4) || ldx % 8 != 0 || ldq % 16 != 0)
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(S, sa) || ldx % 8 != 0 || ldq % 16 != 0)
     return PURO_ERR_ALIGN;
-  if (int d = check_device()) return d;
-  return puro::launch_quant_rows(X, R, C, ldx, Xq, ldq, S, stream);
+  return check_device();
 }
 
-int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, int64_t C, int64_t ldx,
-                                       uint8_t *XqT, float *ST, uint8_t *Xq, float *S,
-                                       puro_stream_t stream) {
+int check_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, const uint8_t *XqT, const void *ST,
+               const uint8_t *Xq, const void *S, uintptr_t sa) {
   if (X == nullptr || XqT == nullptr || ST == nullptr) return PURO_ERR_NULL;
   if ((Xq == nullptr) != (S == nullptr)) return PURO_ERR_NULL;
   if (T < 128 || T % 128 != 0 || C < 8 || C % 8 != 0 || ldx < C) return PURO_ERR_SHAPE;
   if (Xq != nullptr && C % 128 != 0) return PURO_ERR_SHAPE;
   if (T / 128 > 65535 || (C + 127) / 128 > (1ll << 31) - 1 || !tiles_fit(T, 128, C, 128))
     return PURO_ERR_SHAPE;
-  if (!aligned(X, 16) || !aligned(XqT, 16) || !aligned(ST, 4) || ldx % 8 != 0)
-    return PURO_ERR_ALIGN;
-  if (Xq != nullptr && (!aligned(Xq, 16) || !aligned(S, 4))) return PURO_ERR_ALIGN;
-  if (int d = check_device()) return d;
-  return puro::launch_quant_cols(X, T, C, ldx, XqT, ST, Xq, S, stream);
+  if (!aligned(X, 16) || !aligned(XqT, 16) || !aligned(ST, sa) || ldx % 8 != 0) return PURO_ERR_ALIGN;
+  if (Xq != nullptr && (!aligned(Xq, 16) || !aligned(S, sa))) return PURO_ERR_ALIGN;
+  return check_device();
 }
 
-int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
-                              uint8_t *WqT, float *S, puro_stream_t stream) {
+int check_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, const uint8_t *Wq,
+                 const uint8_t *WqT, const void *S, uintptr_t sa) {
   if (W == nullptr || Wq == nullptr || S == nullptr) return PURO_ERR_NULL;
   if (R < 1 || C < 128 || C % 128 != 0 || ldw < C) return PURO_ERR_SHAPE;
   if ((R + 127) / 128 > 65535 || C / 128 > (1ll << 31) - 1 || !tiles_fit(R, 128, C, 128))
     return PURO_ERR_SHAPE;
   if (WqT != nullptr && R % 16 != 0) return PURO_ERR_SHAPE;
-  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(S, 4) || ldw % 8 != 0)
-    return PURO_ERR_ALIGN;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(S, sa) || ldw % 8 != 0) return PURO_ERR_ALIGN;
   if (WqT != nullptr && !aligned(WqT, 16)) return PURO_ERR_ALIGN;
-  if (int d = check_device()) return d;
-  return puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, S, stream);
+  return check_device();
 }
 
 // The checks of one GEMM's arguments (every layout); PURO_OK or the status to return.
@@ -97,6 +88,48 @@ int check_gemm(const uint8_t *Aq, const float *As, const uint8_t *Bq, const floa
   return PURO_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int puro_fp8_quantize_1x128(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                            int64_t ldq, float *S, puro_stream_t stream) {
+  if (int e = check_rows(X, R, C, ldx, Xq, ldq, S, 4)) return e;
+  return puro::launch_quant_rows(X, R, C, ldx, Xq, ldq, S, stream);
+}
+
+int puro_fp8_quantize_1x128_pow2(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                                 int64_t ldq, uint8_t *S, puro_stream_t stream) {
+  if (int e = check_rows(X, R, C, ldx, Xq, ldq, S, 1)) return e;
+  return puro::launch_quant_rows(X, R, C, ldx, Xq, ldq, nullptr, stream, S);
+}
+
+int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, int64_t C, int64_t ldx,
+                                       uint8_t *XqT, float *ST, uint8_t *Xq, float *S,
+                                       puro_stream_t stream) {
+  if (int e = check_cols(X, T, C, ldx, XqT, ST, Xq, S, 4)) return e;
+  return puro::launch_quant_cols(X, T, C, ldx, XqT, ST, Xq, S, stream);
+}
+
+int puro_fp8_quantize_1x128_transposed_pow2(const uint16_t *X, int64_t T, int64_t C, int64_t ldx,
+                                            uint8_t *XqT, uint8_t *ST, uint8_t *Xq, uint8_t *S,
+                                            puro_stream_t stream) {
+  if (int e = check_cols(X, T, C, ldx, XqT, ST, Xq, S, 1)) return e;
+  return puro::launch_quant_cols(X, T, C, ldx, XqT, nullptr, Xq, nullptr, stream, ST, S);
+}
+
+int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
+                              uint8_t *WqT, float *S, puro_stream_t stream) {
+  if (int e = check_weight(W, R, C, ldw, Wq, WqT, S, 4)) return e;
+  return puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, S, stream);
+}
+
+int puro_fp8_quantize_128x128_pow2(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
+                                   uint8_t *WqT, uint8_t *S, puro_stream_t stream) {
+  if (int e = check_weight(W, R, C, ldw, Wq, WqT, S, 1)) return e;
+  return puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, nullptr, stream, S);
+}
+
 int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                             const float *Bs, uint16_t *C, int64_t M, int64_t N, int64_t K,
                             int layout, void *workspace, size_t ws_bytes, puro_stream_t stream) {
@@ -105,6 +138,19 @@ int puro_fp8_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *B
   if (int e = check_gemm(Aq, As, Bq, Bs, C, M, N, K, layout)) return e;
   if (int d = check_device()) return d;
   return puro::launch_gemm_blockwise(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
+}
+
+int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs,
+                     uint16_t *C, int64_t M, int64_t N, int64_t K, int layout, puro_stream_t stream) {
+  if (Aq == nullptr || As == nullptr || Bq == nullptr || Bs == nullptr || C == nullptr)
+    return PURO_ERR_NULL;
+  if (layout != PURO_FPROP && layout != PURO_DGRAD && layout != PURO_WGRAD) return PURO_ERR_LAYOUT;
+  if (M < 1 || N < 8 || N % 8 != 0 || K < 128 || K % 128 != 0) return PURO_ERR_SHAPE;
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
+  if (!tiles_fit(M, 128, N, 256)) return PURO_ERR_SHAPE;
+  if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16)) return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_gemm_mx(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
 }
 
 int puro_fp8_gemm_blockwise_grouped(const puro_gemm_problem *problems, int count, int layout,
@@ -157,10 +203,11 @@ int puro_fp8_sync_status(puro_stream_t stream) {
   // The status words are per device and collect timeouts from kernels on every stream:
   // join the whole device first so that none is missed.
   if (cudaDeviceSynchronize() != cudaSuccess) return PURO_ERR_CUDA;
-  int gemm = 0, quant = 0;
+  int gemm = 0, quant = 0, mx = 0;
   if (int e = puro::read_and_clear_device_status(stream, &gemm)) return e;
   if (int e = puro::read_and_clear_quant_status(stream, &quant)) return e;
-  return (gemm | quant) != 0 ? PURO_ERR_TIMEOUT : PURO_OK;
+  if (int e = puro::read_and_clear_mx_status(stream, &mx)) return e;
+  return (gemm | quant | mx) != 0 ? PURO_ERR_TIMEOUT : PURO_OK;
 }
 
 const char *puro_strerror(int status) {

@@ -1,0 +1,495 @@
+// Blockwise-FP8 GEMM with power-of-two (UE8M0) scales on the tensor cores' block-scaled MMA
+// (tcgen05.mma.kind::mxf8f6f4.block_scale), sm_100a.
+//
+// The groups are the method's ("Paper walkthrough: Puro-2B ...", section "Lever 2: use
+// blockwise FP8 from step zero": 1x128 along K for activations and gradients, 128x128
+// weight blocks); the scales are the power-of-two mode's bytes (2^(byte - 127)). A power of
+// two is applied exactly by the tensor core, which takes one scale per row of A and per
+// column of B for every 32 elements of K and accumulates the whole K in FP32 in TMEM, so
+// no promotion runs on the CUDA cores: the tile's accumulator is read once, at its end.
+//
+// One CTA per SM, 128 x 256 tiles, 512 threads in four warpgroups:
+//   warp 0       TMA producer: A and B K blocks (128 wide) into a 3-stage ring
+//   warp 1       MMA issuer and TMEM owner: per K block 4 block-scaled MMAs (K = 32 each)
+//                into the tile's accumulator
+//   warps 4..11  epilogue: at a tile's end each reads its 32 rows x 128 columns of the
+//                accumulator, hands it back to the MMA issuer, then rounds to BF16 into
+//                swizzled shared memory and stores with the TMA unit
+//   warps 12..15 scale writers, one per TMEM lane quadrant: for every K block they write
+//                its scale factors into a ring slot of TMEM columns. The MMA reads the
+//                factor of A row m from lane m, column m / 32, and that of B column n from
+//                lane 32q + n % 32, column n / 32, in the lane quadrant q of the row it
+//                computes; each quadrant therefore holds its 32 rows' A factors (4
+//                columns) and all 256 columns' B factors (8 columns). A 32-bit cell holds
+//                the factors of four K sub-blocks; one scale covers all 128 of K here, so
+//                its byte is written four times.
+// TMEM: accumulator columns 0..255; ring slot i: A factors at 256 + 16i (4 columns), B
+// factors at 260 + 16i (8 columns). Every mbarrier wait is bounded; a wait that gives up
+// sets the abort flag and the device status word, and the CTA drains and exits.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+
+#include "../../include/puro_fp8.h"
+#include "host_cache.h"
+#include "ptx.cuh"
+#include "quant.h"
+
+namespace puro {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int STAGES = 3;
+constexpr int SF_SLOTS = 4;
+constexpr int THREADS = 512;
+constexpr int EPI_FIRST = 4, EPI_WARPS = 8, SFW_FIRST = 12;
+constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK;
+constexpr int STG_BOX_BYTES = 32 * 128;               // 32 rows x 64 BF16, 128B-swizzled
+constexpr int STG_WARP_BYTES = 2 * STG_BOX_BYTES;     // 128 columns per epilogue warp
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
+// full/empty per stage, sf_full/sf_empty per slot, tfull, tempty, drain
+constexpr int N_BARS = 2 * STAGES + 2 * SF_SLOTS + 3;
+constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_SLOT_COLS = 16;
+constexpr int LAUNCH_REGS = 128;   // 65536 / 512
+constexpr int REGS_SMALL = 56;     // warpgroups 0 and 3
+constexpr int REGS_EPI = 200;      // warpgroups 1 and 2
+static_assert(128 * REGS_SMALL * 2 + 256 * REGS_EPI == THREADS * LAUNCH_REGS, "register split");
+
+// Block-scaled instruction descriptor: E4M3 A and B, K-major, FP32 accumulate, UE8M0 scale
+// factors, M x N; sf_a / sf_b pick the byte (K sub-block) of the scale-factor cells.
+__host__ __device__ constexpr uint32_t idesc_mx(int m, int n, uint32_t sf_a, uint32_t sf_b) {
+  return (sf_b << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(m >> 4) << 24) | (sf_a << 29);
+}
+
+__device__ __forceinline__ void mma_mx(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                       uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, const uint32_t (&v)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+struct MxArgs {
+  const uint8_t *As;  // UE8M0 [K/128, M]
+  const uint8_t *Bs;  // UE8M0, layout-dependent (see the C declaration)
+  int M, N, K;
+  int num_m, num_n, kblocks, m_fastest;
+  unsigned long long timeout_ns;
+  int *status;
+};
+
+__device__ int g_mx_status;  // non-zero: a bounded wait gave up since the last read
+
+__device__ __forceinline__ void mx_tile_coords(int tile, const MxArgs &a, int &mt, int &nt) {
+  if (a.m_fastest) {
+    mt = tile % a.num_m;
+    nt = tile / a.num_m;
+  } else {
+    nt = tile % a.num_n;
+    mt = tile / a.num_n;
+  }
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits_mx(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmC, const MxArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + OFF_BAR;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto sf_full_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + i); };
+  auto sf_empty_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + SF_SLOTS + i); };
+  const uint32_t tfull_bar = bar0 + 8u * (2 * STAGES + 2 * SF_SLOTS);
+  const uint32_t tempty_bar = tfull_bar + 8u;
+  const uint32_t drain_bar = tfull_bar + 16u;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < SF_SLOTS; ++i) {
+      mbar_init(sf_full_bar(i), 4);   // the four scale-writer warps
+      mbar_init(sf_empty_bar(i), 1);  // the MMA commit
+    }
+    mbar_init(tfull_bar, 1);
+    mbar_init(tempty_bar, EPI_WARPS);
+    mbar_init(drain_bar, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+  const int tiles = args.num_m * args.num_n;
+  const int kblocks = args.kblocks;
+  const uint64_t tmo = args.timeout_ns;
+
+  if (warp < EPI_FIRST) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_SMALL));
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        int mt, nt;
+        mx_tile_coords(tile, args, mt, nt);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty_bar(s), ph ^ 1u, tmo, abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+          tma_load_2d(sbase + OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
+          tma_load_2d(sbase + OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
+          issued |= 1u << s;
+          issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) s = 0, ph ^= 1u;
+        }
+      }
+      if (!ok) {
+        *abort = 1;
+        atomicOr(args.status, 1);
+        for (int i = 0; i < STAGES; ++i)
+          if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      int s = 0, slot = 0;
+      uint32_t ph = 0, sph = 0, it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++it) {
+        if (!mbar_wait(tempty_bar, (it & 1u) ^ 1u, tmo, abort)) {  // the accumulator is free
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full_bar(s), ph, tmo, abort) || !mbar_wait(sf_full_bar(slot), sph, tmo, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = sbase + OFF_A + s * A_BYTES, b_addr = sbase + OFF_B + s * B_BYTES;
+          const uint32_t sfa = tmem + SF_COL + SF_SLOT_COLS * slot, sfb = sfa + 4;
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_mx(tmem + ACC_COL, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k),
+                   idesc_mx(BM, BN, k, k), sfa, sfb, (kb > 0 || k > 0) ? 1u : 0u);
+          mma_commit(empty_bar(s));
+          mma_commit(sf_empty_bar(slot));
+          if (++s == STAGES) s = 0, ph ^= 1u;
+          if (++slot == SF_SLOTS) slot = 0, sph ^= 1u;
+        }
+        if (ok) mma_commit(tfull_bar);
+      }
+      if (!ok) {
+        *abort = 1;
+        atomicOr(args.status, 1);
+        mma_commit(drain_bar);
+        mbar_wait(drain_bar, 0, tmo, nullptr);
+      }
+    }
+  } else if (warp >= SFW_FIRST) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_SMALL));
+    // ------------------------------------------------------------------ scale writers
+    const uint32_t lane_field = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int nb_total = (args.N + 127) / 128;
+    // the factors of (tile, kb), each byte repeated in the four bytes of its cell
+    auto fetch = [&](int tile, int kb, uint32_t (&wa)[4], uint32_t (&wb)[8]) {
+      int mt, nt;
+      mx_tile_coords(tile, args, mt, nt);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int m = mt * BM + 32 * g + lane;
+        const uint32_t b = m < args.M ? __ldg(args.As + static_cast<int64_t>(kb) * args.M + m) : 127u;
+        wa[g] = b * 0x01010101u;
+      }
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const int n = nt * BN + 32 * g + lane;
+        uint32_t b = 127u;
+        if (n < args.N) {
+          if (LAYOUT == PURO_FPROP)
+            b = __ldg(args.Bs + static_cast<int64_t>(n >> 7) * kblocks + kb);
+          else if (LAYOUT == PURO_DGRAD)
+            b = __ldg(args.Bs + static_cast<int64_t>(kb) * nb_total + (n >> 7));
+          else
+            b = __ldg(args.Bs + static_cast<int64_t>(kb) * args.N + n);
+        }
+        wb[g] = b * 0x01010101u;
+      }
+    };
+    int slot = 0;
+    uint32_t sph = 0;
+    bool ok = true;
+    int tile = blockIdx.x, kb = 0;
+    uint32_t wa[4], wb[8];
+    if (tile < tiles) fetch(tile, 0, wa, wb);
+    while (ok && tile < tiles) {
+      int ntile = tile, nkb = kb + 1;
+      if (nkb == kblocks) nkb = 0, ntile += gridDim.x;
+      uint32_t na[4], nb[8];
+      if (ntile < tiles) fetch(ntile, nkb, na, nb);  // in flight while this slot is written
+      if (!mbar_wait(sf_empty_bar(slot), sph ^ 1u, tmo, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      tmem_st_x4(tmem + lane_field + SF_COL + SF_SLOT_COLS * slot, wa);
+      tmem_st_x8(tmem + lane_field + SF_COL + SF_SLOT_COLS * slot + 4, wb);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sf_full_bar(slot));
+      if (++slot == SF_SLOTS) slot = 0, sph ^= 1u;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) wa[g] = na[g];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) wb[g] = nb[g];
+      tile = ntile;
+      kb = nkb;
+    }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      atomicOr(args.status, 1);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_EPI));
+    // ------------------------------------------------------------------ epilogue
+    const int quad = warp & 3, half = (warp - EPI_FIRST) >> 2;
+    const uint32_t taddr = tmem + ACC_COL + (static_cast<uint32_t>(quad * 32) << 16) + half * 128;
+    const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST) * STG_WARP_BYTES;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+      int mt, nt;
+      mx_tile_coords(tile, args, mt, nt);
+      if (!mbar_wait(tfull_bar, it & 1u, tmo, abort)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      uint32_t r0[64], r1[64];
+      tmem_ld_64cols(taddr, r0);
+      tmem_ld_64cols(taddr + 64, r1);
+      tmem_wait_ld_dep(r0);
+      tmem_wait_ld_dep(r1);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar);  // the MMA may start the next tile
+      if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores left the staging
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t *r = j < 8 ? r0 : r1;
+        const int jj = j & 7;
+        const uint32_t addr = stg + (j >> 3) * STG_BOX_BYTES + lane * 128 + (((jj) ^ (lane & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                     "r"(bf16x2_bits_mx(__uint_as_float(r[8 * jj]), __uint_as_float(r[8 * jj + 1]))),
+                     "r"(bf16x2_bits_mx(__uint_as_float(r[8 * jj + 2]), __uint_as_float(r[8 * jj + 3]))),
+                     "r"(bf16x2_bits_mx(__uint_as_float(r[8 * jj + 4]), __uint_as_float(r[8 * jj + 5]))),
+                     "r"(bf16x2_bits_mx(__uint_as_float(r[8 * jj + 6]), __uint_as_float(r[8 * jj + 7])))
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int row0 = mt * BM + quad * 32, col0 = nt * BN + half * 128;
+        if (row0 < args.M) {
+          if (col0 < args.N) tma_store_2d(&tmC, stg, col0, row0);
+          if (col0 + 64 < args.N) tma_store_2d(&tmC, stg + STG_BOX_BYTES, col0 + 64, row0);
+        }
+        bulk_commit_group();
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();
+    if (!ok && lane == 0) {
+      *abort = 1;
+      atomicOr(args.status, 1);
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn mx_encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+bool mx_map(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem, uint64_t rows,
+            uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+  EncodeTiledFn fn = mx_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+unsigned long long mx_timeout_ns() {
+  static unsigned long long ns = [] {
+    const char *e = std::getenv("PURO_WAIT_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 2000;
+    if (ms < 1) ms = 1;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return ns;
+}
+
+template <int LAYOUT>
+int launch_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs, uint16_t *C,
+              int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  int sms = 0;
+  if (!sm_count(sms)) return PURO_ERR_CUDA;
+  static PerDevice<int *> status_addr;
+  MxArgs args{};
+  if (!status_addr.get(args.status, [](int, int *&v) {
+        return cudaGetSymbolAddress(reinterpret_cast<void **>(&v), g_mx_status) == cudaSuccess;
+      }))
+    return PURO_ERR_CUDA;
+  CUtensorMap ta, tb, tc;
+  if (!mx_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK) ||
+      !mx_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, BN, BK) ||
+      !mx_map(&tc, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64))
+    return PURO_ERR_CUDA;
+  args.As = As;
+  args.Bs = Bs;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.kblocks = static_cast<int>(K / BK);
+  args.num_m = static_cast<int>((M + BM - 1) / BM);
+  args.num_n = static_cast<int>((N + BN - 1) / BN);
+  args.m_fastest = M <= N ? 1 : 0;
+  args.timeout_ns = mx_timeout_ns();
+  const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  auto kern = k_gemm_mx<LAYOUT>;
+  // Once per device: the register split assumes exactly LAUNCH_REGS per thread at launch
+  // (otherwise the epilogue's setmaxnreg.inc could wait forever); shared memory opt-in.
+  static PerDevice<int> prepared;
+  int prep = PURO_ERR_CUDA;
+  if (!prepared.get(prep, [&](int, int &v) {
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return false;
+        if (fa.numRegs != LAUNCH_REGS) {
+          std::fprintf(stderr, "puro_fp8: MX GEMM kernel built with %d registers (expected %d); not launched\n",
+                       fa.numRegs, LAUNCH_REGS);
+          v = PURO_ERR_LAUNCH;
+          return true;
+        }
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+          return false;
+        v = PURO_OK;
+        return true;
+      }))
+    return PURO_ERR_CUDA;
+  if (prep != PURO_OK) return prep;
+  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, args);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "puro_fp8: MX GEMM launch (grid %d): %s\n", grid, cudaGetErrorString(e));
+    return PURO_ERR_LAUNCH;
+  }
+  return PURO_OK;
+}
+
+}  // namespace
+
+int launch_gemm_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs, uint16_t *C,
+                   int64_t M, int64_t N, int64_t K, int layout, cudaStream_t stream) {
+  switch (layout) {
+    case PURO_FPROP: return launch_mx<PURO_FPROP>(Aq, As, Bq, Bs, C, M, N, K, stream);
+    case PURO_DGRAD: return launch_mx<PURO_DGRAD>(Aq, As, Bq, Bs, C, M, N, K, stream);
+    case PURO_WGRAD: return launch_mx<PURO_WGRAD>(Aq, As, Bq, Bs, C, M, N, K, stream);
+    default: return PURO_ERR_LAYOUT;
+  }
+}
+
+int read_and_clear_mx_status(cudaStream_t stream, int *status_out) {
+  int host = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&host, g_mx_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemcpyToSymbolAsync(g_mx_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  *status_out = host;
+  return PURO_OK;
+}
+
+}  // namespace puro

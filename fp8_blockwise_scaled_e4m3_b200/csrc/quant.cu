@@ -67,6 +67,8 @@ struct QArgs {
   float *s;          // S of the row-wise groups, or of the weight blocks
   float *st;         // ST of the transposed groups (Q_COLS, Q_DUAL)
   int write_t;       // Q_WEIGHT: also write WqT through the transposed store
+  uint8_t *sb;       // P2: UE8M0 scale bytes in place of s
+  uint8_t *stb;      // P2: UE8M0 scale bytes in place of st
   int tiles_r, tiles_c;
   unsigned long long timeout_ns;
   int *status;
@@ -154,7 +156,9 @@ __device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[TG],
   }
 }
 
-template <int MODE>
+// P2: power-of-two scales (UE8M0 bytes) instead of the method's FP32 amax / 448; the codes
+// then come out of the same fast path exactly as x * 2^-e (see pow2_scale).
+template <int MODE, bool P2>
 __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
     k_quant_tiles(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
                   const QArgs args) {
@@ -241,9 +245,14 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
       float amax = warp_max[0];
 #pragma unroll
       for (int k = 1; k < NT / 32; ++k) amax = fmaxf(amax, warp_max[k]);
-      float sblk;
-      block_scale(amax, sblk, wdiv);
-      if (tid == 0) args.s[static_cast<int64_t>(tr) * args.tiles_c + tc] = sblk;
+      if constexpr (P2) {
+        const uint32_t byte = pow2_scale(amax, wdiv);
+        if (tid == 0) args.sb[static_cast<int64_t>(tr) * args.tiles_c + tc] = static_cast<uint8_t>(byte);
+      } else {
+        float sblk;
+        block_scale(amax, sblk, wdiv);
+        if (tid == 0) args.s[static_cast<int64_t>(tr) * args.tiles_c + tc] = sblk;
+      }
     }
 
     // ---------------------------------------------------------------- row-wise codes
@@ -260,6 +269,7 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
         v1[p] = row_chunk(stage, rg + RSTEP * p, 1, j8);
       }
       float srow[NP], amax[NP];
+      uint32_t brow[NP];  // P2: scale bytes
       BlockDivider div[NP];
       bool ok = true;
       if (kRows) {
@@ -272,9 +282,12 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
           for (int p = 0; p < NP; ++p) m[p] = bf16x2_absmax(m[p], __shfl_xor_sync(0xffffffffu, m[p], o));
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          bool okp;
+          bool okp = true;
           amax[p] = bf16x2_absmax_to_f32(m[p]);
-          block_scale_fast(amax[p], srow[p], div[p], okp);
+          if constexpr (P2)
+            brow[p] = pow2_scale(amax[p], div[p]);
+          else
+            block_scale_fast(amax[p], srow[p], div[p], okp);
           ok = ok && okp;
         }
       } else {
@@ -293,7 +306,7 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
       } else {
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          if (kRows) block_scale(amax[p], srow[p], div[p]);
+          if constexpr (kRows && !P2) block_scale(amax[p], srow[p], div[p]);
           q0[p] = codes8(v0[p], div[p]);
           q1[p] = codes8(v1[p], div[p]);
         }
@@ -305,7 +318,12 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
           uint8_t *qrow = args.q + row * args.ldq + c0 + 8 * j8;
           *reinterpret_cast<uint2 *>(qrow) = q0[p];
           *reinterpret_cast<uint2 *>(qrow + 64) = q1[p];
-          if (kRows && j8 == 0) args.s[(c0 / kTile) * args.R + row] = srow[p];
+          if (kRows && j8 == 0) {
+            if constexpr (P2)
+              args.sb[(c0 / kTile) * args.R + row] = static_cast<uint8_t>(brow[p]);
+            else
+              args.s[(c0 / kTile) * args.R + row] = srow[p];
+          }
         }
       }
     }
@@ -337,18 +355,30 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
             a1 = fmaxf(a1, part[k][2 * cp + 1]);
           }
           float s0, s1;
-          bool ok0, ok1;
-          block_scale_fast(a0, s0, d0, ok0);
-          block_scale_fast(a1, s1, d1, ok1);
-          if (!ok0) block_scale(a0, s0, d0);
-          if (!ok1) block_scale(a1, s1, d1);
+          bool ok0 = true, ok1 = true;
+          uint32_t b0 = 0, b1 = 0;
+          if constexpr (P2) {
+            b0 = pow2_scale(a0, d0);
+            b1 = pow2_scale(a1, d1);
+          } else {
+            block_scale_fast(a0, s0, d0, ok0);
+            block_scale_fast(a1, s1, d1, ok1);
+            if (!ok0) block_scale(a0, s0, d0);
+            if (!ok1) block_scale(a1, s1, d1);
+          }
           ok = ok0 && ok1;
           col_div[2 * cp] = make_float2(d0.s, d0.fast ? d0.r : -1.0f);
           col_div[2 * cp + 1] = make_float2(d1.s, d1.fast ? d1.r : -1.0f);
           const int64_t c = c0 + 2 * cp;
-          float *strow = args.st + static_cast<int64_t>(tr) * args.C;
-          if (c < args.C) strow[c] = s0;
-          if (c + 1 < args.C) strow[c + 1] = s1;
+          if constexpr (P2) {
+            uint8_t *strow = args.stb + static_cast<int64_t>(tr) * args.C;
+            if (c < args.C) strow[c] = static_cast<uint8_t>(b0);
+            if (c + 1 < args.C) strow[c + 1] = static_cast<uint8_t>(b1);
+          } else {
+            float *strow = args.st + static_cast<int64_t>(tr) * args.C;
+            if (c < args.C) strow[c] = s0;
+            if (c + 1 < args.C) strow[c + 1] = s1;
+          }
         }
         tile_fast = __syncthreads_and(ok);
         const float2 e0 = col_div[2 * cp], e1 = col_div[2 * cp + 1];
@@ -429,7 +459,7 @@ unsigned long long wait_timeout_ns() {
   return ns;
 }
 
-template <int MODE>
+template <int MODE, bool P2>
 int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *qt, QArgs args,
                  cudaStream_t stream) {
   int sms = 0;
@@ -456,7 +486,7 @@ int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *
   args.timeout_ns = wait_timeout_ns();
   const int64_t tiles = static_cast<int64_t>(args.tiles_r) * args.tiles_c;
   const int grid = static_cast<int>(tiles < kCtasPerSm * sms ? tiles : kCtasPerSm * sms);
-  auto kern = k_quant_tiles<MODE>;
+  auto kern = k_quant_tiles<MODE, P2>;
   static PerDevice<bool> smem_opt_in;  // dynamic shared memory opted in once per device
   bool done = false;
   if (!smem_opt_in.get(done, [&](int, bool &v) {
@@ -478,35 +508,44 @@ int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *
 
 // ------------------------------------------------------------------ launchers
 int launch_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
-                      int64_t ldq, float *S, cudaStream_t stream) {
+                      int64_t ldq, float *S, cudaStream_t stream, uint8_t *Sb) {
   QArgs a{};
   a.q = Xq;
   a.ldq = ldq;
   a.s = S;
-  return launch_tiles<Q_ROWS>(X, R, C, ldx, nullptr, a, stream);
+  a.sb = Sb;
+  return Sb != nullptr ? launch_tiles<Q_ROWS, true>(X, R, C, ldx, nullptr, a, stream)
+                       : launch_tiles<Q_ROWS, false>(X, R, C, ldx, nullptr, a, stream);
 }
 
 int launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint8_t *XqT,
-                      float *ST, uint8_t *Xq, float *S, cudaStream_t stream) {
+                      float *ST, uint8_t *Xq, float *S, cudaStream_t stream, uint8_t *STb, uint8_t *Sb) {
   QArgs a{};
   a.st = ST;
+  a.stb = STb;
+  const bool p2 = STb != nullptr;
   if (Xq != nullptr) {
     a.q = Xq;
     a.ldq = C;
     a.s = S;
-    return launch_tiles<Q_DUAL>(X, T, C, ldx, XqT, a, stream);
+    a.sb = Sb;
+    return p2 ? launch_tiles<Q_DUAL, true>(X, T, C, ldx, XqT, a, stream)
+              : launch_tiles<Q_DUAL, false>(X, T, C, ldx, XqT, a, stream);
   }
-  return launch_tiles<Q_COLS>(X, T, C, ldx, XqT, a, stream);
+  return p2 ? launch_tiles<Q_COLS, true>(X, T, C, ldx, XqT, a, stream)
+            : launch_tiles<Q_COLS, false>(X, T, C, ldx, XqT, a, stream);
 }
 
 int launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
-                        uint8_t *WqT, float *S, cudaStream_t stream) {
+                        uint8_t *WqT, float *S, cudaStream_t stream, uint8_t *Sb) {
   QArgs a{};
   a.q = Wq;
   a.ldq = C;
   a.s = S;
+  a.sb = Sb;
   a.write_t = WqT != nullptr;
-  return launch_tiles<Q_WEIGHT>(W, R, C, ldw, WqT, a, stream);
+  return Sb != nullptr ? launch_tiles<Q_WEIGHT, true>(W, R, C, ldw, WqT, a, stream)
+                       : launch_tiles<Q_WEIGHT, false>(W, R, C, ldw, WqT, a, stream);
 }
 
 int read_and_clear_quant_status(cudaStream_t stream, int *status_out) {

@@ -10,13 +10,15 @@
 
 namespace puro {
 
-// Quantiser launchers; return 0 or a negative puro_status.
+// Quantiser launchers; return 0 or a negative puro_status. With the byte pointers set (Sb,
+// STb) the scales are the power-of-two (UE8M0) mode's bytes and the float pointers unused.
 int launch_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
-                      int64_t ldq, float *S, cudaStream_t stream);
+                      int64_t ldq, float *S, cudaStream_t stream, uint8_t *Sb = nullptr);
 int launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint8_t *XqT,
-                      float *ST, uint8_t *Xq, float *S, cudaStream_t stream);
+                      float *ST, uint8_t *Xq, float *S, cudaStream_t stream, uint8_t *STb = nullptr,
+                      uint8_t *Sb = nullptr);
 int launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
-                        uint8_t *WqT, float *S, cudaStream_t stream);
+                        uint8_t *WqT, float *S, cudaStream_t stream, uint8_t *Sb = nullptr);
 
 // Reads and clears the quantisers' device status word (after a stream sync).
 int read_and_clear_quant_status(cudaStream_t stream, int *status_out);
@@ -41,6 +43,11 @@ int launch_gemm_blockwise_quant(const uint8_t *Aq, const float *As, const uint8_
 int launch_gemm_wgrad_acc_f32(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                               const float *Bs, float *C, int64_t M, int64_t N, int64_t K,
                               cudaStream_t stream);
+
+// Blockwise GEMM with power-of-two scale bytes on the block-scaled MMA; and its status word.
+int launch_gemm_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs, uint16_t *C,
+                   int64_t M, int64_t N, int64_t K, int layout, cudaStream_t stream);
+int read_and_clear_mx_status(cudaStream_t stream, int *status_out);
 
 // Reads and clears the device status word of the GEMM kernels (after a stream sync).
 int read_and_clear_device_status(cudaStream_t stream, int *status_out);

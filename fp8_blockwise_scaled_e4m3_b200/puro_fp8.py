@@ -52,6 +52,10 @@ def _load():
         "puro_fp8_gemm_wgrad_acc_f32": [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p],
         "puro_fp8_gemm_blockwise_quant": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p],
         "puro_fp8_gemm_blockwise_grouped": [_p, ctypes.c_int, ctypes.c_int, _p],
+        "puro_fp8_quantize_1x128_pow2": [_p, _i64, _i64, _i64, _p, _i64, _p, _p],
+        "puro_fp8_mx_gemm": [_p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p],
+        "puro_fp8_quantize_1x128_transposed_pow2": [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
+        "puro_fp8_quantize_128x128_pow2": [_p, _i64, _i64, _i64, _p, _p, _p, _p],
         "puro_fp8_sync_status": [_p],
     }
     for name, args in sig.items():
@@ -197,6 +201,75 @@ def puro_fp8_gemm_blockwise(Aq, As, Bq, Bs, C, layout, workspace=None, stream=No
                                             layout, _ptr(workspace), ws_bytes, st), "puro_fp8_gemm_blockwise", st)
 
 
+def puro_fp8_quantize_1x128_pow2(X, Xq, S, stream=None):
+    """As puro_fp8_quantize_1x128, power-of-two scales as bytes: S uint8 [C/128, R]."""
+    R, C = _matrix(X, "X")
+    _shape(Xq, (R, C), "Xq"); _shape(S, (C // 128, R), "S")
+    _need(X, torch.bfloat16, "X"); _need(Xq, torch.uint8, "Xq"); _need(S, torch.uint8, "S")
+    _dense(S, "S")
+    with torch.cuda.device(X.device):
+        st = _stream(stream)  # the current stream of the tensors' device
+        _check(_lib.puro_fp8_quantize_1x128_pow2(_ptr(X), R, C, X.stride(0), _ptr(Xq), Xq.stride(0), _ptr(S), st),
+               "puro_fp8_quantize_1x128_pow2", st)
+
+
+def puro_fp8_quantize_1x128_transposed_pow2(X, XqT, ST, Xq=None, S=None, stream=None):
+    """As puro_fp8_quantize_1x128_transposed, power-of-two scales as bytes."""
+    T, C = _matrix(X, "X")
+    _shape(XqT, (C, T), "XqT"); _shape(ST, (T // 128, C), "ST")
+    _shape(Xq, (T, C), "Xq"); _shape(S, (C // 128, T), "S")
+    _need(X, torch.bfloat16, "X"); _need(XqT, torch.uint8, "XqT"); _need(ST, torch.uint8, "ST")
+    _need(Xq, torch.uint8, "Xq"); _need(S, torch.uint8, "S")
+    for t, n in ((XqT, "XqT"), (ST, "ST"), (Xq, "Xq"), (S, "S")):
+        _dense(t, n)
+    with torch.cuda.device(X.device):
+        st = _stream(stream)  # the current stream of the tensors' device
+        _check(_lib.puro_fp8_quantize_1x128_transposed_pow2(_ptr(X), T, C, X.stride(0), _ptr(XqT), _ptr(ST),
+                                                            _ptr(Xq), _ptr(S), st),
+               "puro_fp8_quantize_1x128_transposed_pow2", st)
+
+
+def puro_fp8_quantize_128x128_pow2(W, Wq, WqT, S, stream=None):
+    """As puro_fp8_quantize_128x128, power-of-two scales as bytes: S uint8 [ceil(R/128), C/128]."""
+    R, C = _matrix(W, "W")
+    _shape(Wq, (R, C), "Wq"); _shape(WqT, (C, R), "WqT"); _shape(S, ((R + 127) // 128, C // 128), "S")
+    _need(W, torch.bfloat16, "W"); _need(Wq, torch.uint8, "Wq"); _need(WqT, torch.uint8, "WqT")
+    _need(S, torch.uint8, "S")
+    for t, n in ((Wq, "Wq"), (WqT, "WqT"), (S, "S")):
+        _dense(t, n)
+    with torch.cuda.device(W.device):
+        st = _stream(stream)  # the current stream of the tensors' device
+        _check(_lib.puro_fp8_quantize_128x128_pow2(_ptr(W), R, C, W.stride(0), _ptr(Wq), _ptr(WqT), _ptr(S), st),
+               "puro_fp8_quantize_128x128_pow2", st)
+
+
+def puro_fp8_mx_gemm(Aq, As, Bq, Bs, C, layout, stream=None):
+    """The block-scaled GEMM of power-of-two scale bytes (see the C declaration): As, Bs uint8
+    laid out as the float scales of puro_fp8_gemm_blockwise for the same layout."""
+    layout = int(LAYOUTS.get(layout, layout))
+    if layout not in (PURO_FPROP, PURO_DGRAD, PURO_WGRAD):
+        raise ValueError(f"unknown layout {layout}")
+    bs_shape = {PURO_FPROP: lambda n, k: ((n + 127) // 128, k // 128),
+                PURO_DGRAD: lambda n, k: (k // 128, (n + 127) // 128),
+                PURO_WGRAD: lambda n, k: (k // 128, n)}[layout]
+    M, N, K = _gemm_shapes(Aq, As, Bq, Bs, C, bs_shape)
+    _need(Aq, torch.uint8, "Aq"); _need(Bq, torch.uint8, "Bq"); _need(C, torch.bfloat16, "C")
+    _need(As, torch.uint8, "As"); _need(Bs, torch.uint8, "Bs")
+    for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs"), (C, "C")):
+        _dense(t, n)
+    with torch.cuda.device(Aq.device):
+        st = _stream(stream)  # the current stream of the tensors' device
+        _check(_lib.puro_fp8_mx_gemm(_ptr(Aq), _ptr(As), _ptr(Bq), _ptr(Bs), _ptr(C), M, N, K, layout, st),
+               "puro_fp8_mx_gemm", st)
+
+
+def mx_gemm(Aq, As, Bq, Bs, layout, stream=None):
+    """C [M, N] bf16 from the block-scaled GEMM (allocating helper)."""
+    C = torch.empty((Aq.shape[0], Bq.shape[0]), dtype=torch.bfloat16, device=Aq.device)
+    puro_fp8_mx_gemm(Aq, As, Bq, Bs, C, layout, stream)
+    return C
+
+
 def puro_fp8_gemm_blockwise_grouped(problems, layout, stream=None):
     """problems: sequence of (Aq, As, Bq, Bs, C) tensor tuples, each checked as for
     puro_fp8_gemm_blockwise; all run in one launch (see the C declaration)."""
@@ -306,6 +379,38 @@ def quantize_128x128(W, transposed=True, stream=None):
     WqT = torch.empty((C, R), dtype=torch.uint8, device=W.device) if transposed else None
     S = torch.empty(((R + 127) // 128, C // 128), dtype=torch.float32, device=W.device)
     puro_fp8_quantize_128x128(W, Wq, WqT, S, stream)
+    return Wq, WqT, S
+
+
+def quantize_1x128_pow2(X, stream=None):
+    """X [R, C] bf16 -> (Xq [R, C], UE8M0 bytes [C/128, R])."""
+    R, C = X.shape
+    Xq = torch.empty((R, C), dtype=torch.uint8, device=X.device)
+    S = torch.empty((C // 128, R), dtype=torch.uint8, device=X.device)
+    puro_fp8_quantize_1x128_pow2(X, Xq, S, stream)
+    return Xq, S
+
+
+def quantize_1x128_transposed_pow2(X, dual=False, stream=None):
+    """X [T, C] bf16 -> (XqT [C, T], bytes [T/128, C]) and, if dual, also (Xq, bytes) row-wise."""
+    T, C = X.shape
+    XqT = torch.empty((C, T), dtype=torch.uint8, device=X.device)
+    ST = torch.empty((T // 128, C), dtype=torch.uint8, device=X.device)
+    Xq = S = None
+    if dual:
+        Xq = torch.empty((T, C), dtype=torch.uint8, device=X.device)
+        S = torch.empty((C // 128, T), dtype=torch.uint8, device=X.device)
+    puro_fp8_quantize_1x128_transposed_pow2(X, XqT, ST, Xq, S, stream)
+    return (XqT, ST, Xq, S) if dual else (XqT, ST)
+
+
+def quantize_128x128_pow2(W, transposed=True, stream=None):
+    """W [R, C] bf16 -> (Wq, WqT or None, bytes [ceil(R/128), C/128])."""
+    R, C = W.shape
+    Wq = torch.empty((R, C), dtype=torch.uint8, device=W.device)
+    WqT = torch.empty((C, R), dtype=torch.uint8, device=W.device) if transposed else None
+    S = torch.empty(((R + 127) // 128, C // 128), dtype=torch.uint8, device=W.device)
+    puro_fp8_quantize_128x128_pow2(W, Wq, WqT, S, stream)
     return Wq, WqT, S
 
 

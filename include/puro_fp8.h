@@ -125,6 +125,48 @@ PURO_API int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, 
                               uint8_t *Wq, uint8_t *WqT, float *S, puro_stream_t stream);
 
 /*
+ * Power-of-two (UE8M0) scale mode of the three quantisers above: the same groups, codes
+ * written the same way, but each group's scale is the method's amax / 448 rounded up to a
+ * power of two, stored as one byte. Source: "Lever 2: use blockwise FP8 from step zero"
+ * (FP8 with local scales per group of 128 / 128x128 block); the pages give no scale
+ * formula, and this mode is the variant whose scales the tensor cores' block-scaled FP8
+ * MMAs (puro_fp8_mx_gemm) apply themselves:
+ *     e    = the smallest integer with 448 * 2^e >= amax, clamped to [-127, 127]
+ *            (an all-zero group: -127)
+ *     byte = e + 127                     (UE8M0)
+ *     code = E4M3_RNE(x * 2^-e)          (exact scaling; nothing saturates)
+ * Arguments, layouts and requirements as for puro_fp8_quantize_1x128,
+ * puro_fp8_quantize_1x128_transposed and puro_fp8_quantize_128x128, with every scale
+ * array (S, ST) holding bytes instead of floats (no alignment requirement).
+ */
+PURO_API int puro_fp8_quantize_1x128_pow2(const uint16_t *X, int64_t R, int64_t C, int64_t ldx,
+                                          uint8_t *Xq, int64_t ldq, uint8_t *S, puro_stream_t stream);
+PURO_API int puro_fp8_quantize_1x128_transposed_pow2(const uint16_t *X, int64_t T, int64_t C, int64_t ldx,
+                                                     uint8_t *XqT, uint8_t *ST, uint8_t *Xq, uint8_t *S,
+                                                     puro_stream_t stream);
+PURO_API int puro_fp8_quantize_128x128_pow2(const uint16_t *W, int64_t R, int64_t C, int64_t ldw,
+                                            uint8_t *Wq, uint8_t *WqT, uint8_t *S, puro_stream_t stream);
+
+/*
+ * Blockwise-FP8 GEMM with power-of-two scales, on the tensor cores' block-scaled MMA:
+ *     C[m, n] = sum_kb 2^(sA(kb, m) - 127) * 2^(sB(kb, n) - 127) * sum_{k in kb} A[m, k] B[n, k]
+ * The operands are the power-of-two quantisers' output (puro_fp8_quantize_*_pow2); the
+ * tensor core applies each power-of-two factor exactly and accumulates all of K in FP32,
+ * so no scale promotion runs on the CUDA cores. Source: "Lever 2: use blockwise FP8 from
+ * step zero" (the linear-layer GEMMs in FP8 with local scales), in the power-of-two scale
+ * mode described above.
+ *
+ *   Aq  [M, K] E4M3 codes, dense      As [K/128, M] UE8M0 bytes
+ *   Bq  [N, K] E4M3 codes, dense      Bs bytes, laid out as the float Bs of
+ *                                     puro_fp8_gemm_blockwise for the same layout
+ *   C   [M, N] BF16, dense            output (round to nearest even)
+ * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, Bq, C 16-byte aligned.
+ * Status codes as for puro_fp8_gemm_blockwise.
+ */
+PURO_API int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs,
+                              uint16_t *C, int64_t M, int64_t N, int64_t K, int layout, puro_stream_t stream);
+
+/*
  * Blockwise-FP8 GEMM  C[m, n] = sum_kb sA(kb, m) * sB(kb, n) * sum_{k in kb} A[m, k] B[n, k]
  * with an FP32 tensor-core partial per 128-wide K block, FP32 promotion and BF16 output.
  * Source: "Lever 2: use blockwise FP8 from step zero" (the linear-layer GEMMs in FP8

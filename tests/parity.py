@@ -16,6 +16,7 @@ import numpy as np
 import torch
 
 from oracle import gemm as ogemm
+from oracle import mx as omx
 from oracle import quant as oquant
 from fp8_blockwise_scaled_e4m3_b200 import workloads as wl
 
@@ -52,8 +53,32 @@ def oracle_rows_1x128(x_bits_rows):
     return oquant.quant_1x128(x_bits_rows)
 
 
-def oracle_gemm_sampled(layout, a_bf16, b_bf16, rows, nblocks):
-    """Oracle C[rows, n] for n in the 128-wide column blocks `nblocks`, from BF16 inputs.
+class _Pow2Quant:
+    """The power-of-two scale quantisers of oracle.mx, with their bytes turned into the float
+    scales 2^(byte - 127) so that oracle.gemm applies unchanged."""
+
+    @staticmethod
+    def quant_1x128(x):
+        q, b = omx.quant_1x128_pow2(x)
+        return q, omx.scales_from_ue8m0(b)
+
+    @staticmethod
+    def quant_1x128_transposed(x):
+        q, b = omx.quant_1x128_transposed_pow2(x)
+        return q, omx.scales_from_ue8m0(b)
+
+    @staticmethod
+    def quant_128x128(w):
+        q, qt, b = omx.quant_128x128_pow2(w)
+        return q, qt, omx.scales_from_ue8m0(b)
+
+
+QUANTISERS = {"fp32": oquant, "pow2": _Pow2Quant}
+
+
+def oracle_gemm_sampled(layout, a_bf16, b_bf16, rows, nblocks, scales="fp32"):
+    """Oracle C[rows, n] for n in the 128-wide column blocks `nblocks`, from BF16 inputs,
+    quantised with FP32 scales (oracle.quant) or power-of-two scales (oracle.mx).
 
     fprop: a = X [T, K_in],  b = W [N_out, K_in]   -> C = X W^T      [T, N_out]
     dgrad: a = dY [T, N_out], b = W [N_out, K_in]  -> C = dY W       [T, K_in]
@@ -61,6 +86,7 @@ def oracle_gemm_sampled(layout, a_bf16, b_bf16, rows, nblocks):
     Returns (c_ref [len(rows), len(cols)], cols, a_norm, b_norm).
     """
     rows = np.asarray(rows)
+    oquant = QUANTISERS[scales]
     if layout == "fprop":
         a_rows = host_bits(a_bf16[torch.as_tensor(rows, device=a_bf16.device)])
         aq, a_s = oquant.quant_1x128(a_rows)

@@ -44,7 +44,9 @@ def test_header_declares_the_entry_points():
     assert declared_functions() == sorted([
         "puro_fp8_quantize_1x128", "puro_fp8_quantize_1x128_transposed", "puro_fp8_quantize_128x128",
         "puro_fp8_gemm_blockwise", "puro_fp8_gemm_wgrad_acc_f32", "puro_fp8_gemm_blockwise_quant",
-        "puro_fp8_gemm_blockwise_grouped", "puro_fp8_sync_status", "puro_strerror"])
+        "puro_fp8_gemm_blockwise_grouped", "puro_fp8_quantize_1x128_pow2",
+        "puro_fp8_quantize_1x128_transposed_pow2", "puro_fp8_quantize_128x128_pow2", "puro_fp8_mx_gemm",
+        "puro_fp8_sync_status", "puro_strerror"])
 
 
 def test_library_exports_exactly_the_declared_symbols(lib):
@@ -230,3 +232,28 @@ def test_gemm_grouped_rejects_bad_arguments(lib):
     assert f(ptr, 2, 2, None) == ENULL
     arr[1] = GemmProblem(A16, A16, A16, A16, A16 + 8, 128, 256, 256)  # C not 16-byte aligned
     assert f(ptr, 2, 1, None) == EALIGN
+
+
+def test_pow2_quantisers_reject_bad_arguments(lib):
+    """The power-of-two scale mode checks its arguments like the FP32-scale quantisers; byte
+    scales need no alignment."""
+    q = lib.puro_fp8_quantize_1x128_pow2
+    assert q(None, 4, 128, 128, A16, 128, A16, None) == ENULL
+    assert q(A16, 4, 100, 128, A16, 128, A16, None) == ESHAPE
+    assert q(A16 + 2, 4, 128, 128, A16, 128, A16, None) == EALIGN
+    qt = lib.puro_fp8_quantize_1x128_transposed_pow2
+    assert qt(A16, 100, 64, 64, A16, A16, None, None, None) == ESHAPE        # T % 128
+    assert qt(A16, 256, 64, 64, A16, A16, A16, None, None) == ENULL          # Xq without S
+    qw = lib.puro_fp8_quantize_128x128_pow2
+    assert qw(A16, 100, 256, 256, A16, A16, A16, None) == ESHAPE             # WqT needs R % 16
+    assert qw(A16, 128, 256, 256, A16 + 4, None, A16, None) == EALIGN
+
+
+def test_mx_gemm_rejects_bad_arguments(lib):
+    f = lib.puro_fp8_mx_gemm
+    ops = [A16, A16, A16, A16, A16]
+    assert f(None, *ops[1:], 128, 256, 256, 0, None) == ENULL
+    assert f(*ops, 128, 256, 256, 5, None) == ELAYOUT
+    assert f(*ops, 128, 250, 256, 0, None) == ESHAPE
+    assert f(*ops, 128, 256, 200, 2, None) == ESHAPE
+    assert f(*ops[:4], A16 + 2, 128, 256, 256, 1, None) == EALIGN
