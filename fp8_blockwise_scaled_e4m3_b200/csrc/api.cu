@@ -149,6 +149,7 @@ int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, co
   if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
   if (!tiles_fit(M, 128, N, 256)) return PURO_ERR_SHAPE;
   if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(C, 16)) return PURO_ERR_ALIGN;
+  if (layout == PURO_WGRAD && !aligned(Bs, 8)) return PURO_ERR_ALIGN;
   if (int d = check_device()) return d;
   return puro::launch_gemm_mx(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
 }

@@ -16,13 +16,14 @@
 //                accumulator, hands it back to the MMA issuer, then rounds to BF16 into
 //                swizzled shared memory and stores with the TMA unit
 //   warps 12..15 scale writers, one per TMEM lane quadrant: for every K block they write
-//                its scale factors into a ring slot of TMEM columns. The MMA reads the
-//                factor of A row m from lane m, column m / 32, and that of B column n from
-//                lane 32q + n % 32, column n / 32, in the lane quadrant q of the row it
-//                computes; each quadrant therefore holds its 32 rows' A factors (4
-//                columns) and all 256 columns' B factors (8 columns). A 32-bit cell holds
-//                the factors of four K sub-blocks; one scale covers all 128 of K here, so
-//                its byte is written four times.
+//                its scale factors into a ring slot of TMEM columns, loading them from
+//                global memory as many K blocks ahead as the ring has slots. The MMA reads
+//                the factor of A row m from lane m, column m / 32, and that of B column n
+//                from lane 32q + n % 32, column n / 32, in the lane quadrant q of the row it
+//                computes; each quadrant therefore holds its 32 rows' A factors (written
+//                into all 4 A columns of its lanes) and all 256 columns' B factors (8
+//                columns). A 32-bit cell holds the factors of four K sub-blocks; one scale
+//                covers all 128 of K here, so its byte is written four times.
 // TMEM: accumulator columns 0..255; ring slot i: A factors at 256 + 16i (4 columns), B
 // factors at 260 + 16i (8 columns). Every mbarrier wait is bounded; a wait that gives up
 // sets the abort flag and the device status word, and the CTA drains and exits.
@@ -242,62 +243,97 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp >= SFW_FIRST) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_SMALL));
     // ------------------------------------------------------------------ scale writers
-    const uint32_t lane_field = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // Loads run SF_SLOTS K blocks ahead of the stores, in a register ring of raw loaded
+    // values (3 registers per K block), so their latency is hidden behind the MMAs.
+    const int quad = warp & 3;
+    const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
     const int nb_total = (args.N + 127) / 128;
-    // the factors of (tile, kb), each byte repeated in the four bytes of its cell
-    auto fetch = [&](int tile, int kb, uint32_t (&wa)[4], uint32_t (&wb)[8]) {
+    // raw values of one K block: this lane's A byte (row 32 quad + lane of the tile) and
+    // two words for B (wgrad: bytes 8 lane .. 8 lane + 7 of the tile's 256 columns;
+    // fprop/dgrad: the bytes of the tile's two 128-column blocks)
+    auto fetch = [&](int tile, int kb, uint32_t &ra, uint32_t &rb0, uint32_t &rb1) {
       int mt, nt;
       mx_tile_coords(tile, args, mt, nt);
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int m = mt * BM + 32 * g + lane;
-        const uint32_t b = m < args.M ? __ldg(args.As + static_cast<int64_t>(kb) * args.M + m) : 127u;
-        wa[g] = b * 0x01010101u;
-      }
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const int n = nt * BN + 32 * g + lane;
-        uint32_t b = 127u;
-        if (n < args.N) {
-          if (LAYOUT == PURO_FPROP)
-            b = __ldg(args.Bs + static_cast<int64_t>(n >> 7) * kblocks + kb);
-          else if (LAYOUT == PURO_DGRAD)
-            b = __ldg(args.Bs + static_cast<int64_t>(kb) * nb_total + (n >> 7));
-          else
-            b = __ldg(args.Bs + static_cast<int64_t>(kb) * args.N + n);
+      const int m = mt * BM + 32 * quad + lane;
+      ra = m < args.M ? __ldg(args.As + static_cast<int64_t>(kb) * args.M + m) : 127u;
+      if (LAYOUT == PURO_WGRAD) {
+        const int n0 = nt * BN + 8 * lane;  // N % 8 == 0: the 8 bytes exist or none do
+        if (n0 < args.N) {
+          const uint2 w = __ldg(reinterpret_cast<const uint2 *>(args.Bs + static_cast<int64_t>(kb) * args.N + n0));
+          rb0 = w.x;
+          rb1 = w.y;
+        } else {
+          rb0 = rb1 = 0x7F7F7F7Fu;
         }
-        wb[g] = b * 0x01010101u;
+      } else {
+        const int j0 = 2 * nt, j1 = 2 * nt + 1;
+        auto at = [&](int j) -> uint32_t {
+          if (j >= nb_total) return 127u;
+          return LAYOUT == PURO_FPROP ? __ldg(args.Bs + static_cast<int64_t>(j) * kblocks + kb)
+                                      : __ldg(args.Bs + static_cast<int64_t>(kb) * nb_total + j);
+        };
+        rb0 = at(j0);
+        rb1 = at(j1);
       }
     };
-    int slot = 0;
+    // TMEM cells of one K block from its raw values; each byte is repeated in the four
+    // bytes of its cell (one cell serves the four K sub-blocks of the 128-wide block)
+    auto store = [&](uint32_t slot, uint32_t ra, uint32_t rb0, uint32_t rb1) {
+      uint32_t ca[4], cb[8];
+      const uint32_t a = (ra & 0xFFu) * 0x01010101u;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) ca[g] = a;
+      if (LAYOUT == PURO_WGRAD) {
+        // column n = 32 g + lane: byte lane & 7 of the words held by lane 4 g + lane / 8
+        const uint32_t sel = ((lane & 3u) * 8u), hi = lane & 4u;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int src = 4 * g + (lane >> 3);
+          const uint32_t w0 = __shfl_sync(0xffffffffu, rb0, src), w1 = __shfl_sync(0xffffffffu, rb1, src);
+          cb[g] = (((hi ? w1 : w0) >> sel) & 0xFFu) * 0x01010101u;
+        }
+      } else {
+        const uint32_t c0 = (rb0 & 0xFFu) * 0x01010101u, c1 = (rb1 & 0xFFu) * 0x01010101u;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) cb[g] = g < 4 ? c0 : c1;
+      }
+      tmem_st_x4(tmem + lane_field + SF_COL + SF_SLOT_COLS * slot, ca);
+      tmem_st_x8(tmem + lane_field + SF_COL + SF_SLOT_COLS * slot + 4, cb);
+    };
+    auto advance = [&](int &tile, int &kb) {
+      if (++kb == kblocks) kb = 0, tile += gridDim.x;
+    };
+    uint32_t ra[SF_SLOTS], rb0[SF_SLOTS], rb1[SF_SLOTS];
+    int ft = blockIdx.x, fk = 0;  // the next K block to fetch
+#pragma unroll
+    for (int d = 0; d < SF_SLOTS; ++d) {
+      if (ft < tiles) fetch(ft, fk, ra[d], rb0[d], rb1[d]);
+      advance(ft, fk);
+    }
     uint32_t sph = 0;
     bool ok = true;
-    int tile = blockIdx.x, kb = 0;
-    uint32_t wa[4], wb[8];
-    if (tile < tiles) fetch(tile, 0, wa, wb);
-    while (ok && tile < tiles) {
-      int ntile = tile, nkb = kb + 1;
-      if (nkb == kblocks) nkb = 0, ntile += gridDim.x;
-      uint32_t na[4], nb[8];
-      if (ntile < tiles) fetch(ntile, nkb, na, nb);  // in flight while this slot is written
-      if (!mbar_wait(sf_empty_bar(slot), sph ^ 1u, tmo, abort)) {
-        ok = false;
-        break;
+    int ct = blockIdx.x, ck = 0;  // the next K block to store
+    while (ok && ct < tiles) {
+#pragma unroll
+      for (int d = 0; d < SF_SLOTS; ++d) {  // ring slot d holds the K block fetched into set d
+        if (ct < tiles) {
+          // warp-uniform outcome: the stores and shuffles below need the whole warp
+          if (!__all_sync(0xffffffffu, mbar_wait(sf_empty_bar(d), sph ^ 1u, tmo, abort))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          store(d, ra[d], rb0[d], rb1[d]);
+          if (ft < tiles) fetch(ft, fk, ra[d], rb0[d], rb1[d]);
+          advance(ft, fk);
+          tmem_wait_st();
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sf_full_bar(d));
+          advance(ct, ck);
+        }
       }
-      tc_fence_after_sync();
-      tmem_st_x4(tmem + lane_field + SF_COL + SF_SLOT_COLS * slot, wa);
-      tmem_st_x8(tmem + lane_field + SF_COL + SF_SLOT_COLS * slot + 4, wb);
-      tmem_wait_st();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sf_full_bar(slot));
-      if (++slot == SF_SLOTS) slot = 0, sph ^= 1u;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) wa[g] = na[g];
-#pragma unroll
-      for (int g = 0; g < 8; ++g) wb[g] = nb[g];
-      tile = ntile;
-      kb = nkb;
+      sph ^= 1u;
     }
     if (!ok && lane == 0) {
       *abort = 1;

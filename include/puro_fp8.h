@@ -160,8 +160,8 @@ PURO_API int puro_fp8_quantize_128x128_pow2(const uint16_t *W, int64_t R, int64_
  *   Bq  [N, K] E4M3 codes, dense      Bs bytes, laid out as the float Bs of
  *                                     puro_fp8_gemm_blockwise for the same layout
  *   C   [M, N] BF16, dense            output (round to nearest even)
- * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, Bq, C 16-byte aligned.
- * Status codes as for puro_fp8_gemm_blockwise.
+ * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, Bq, C 16-byte aligned;
+ * for PURO_WGRAD also Bs 8-byte aligned. Status codes as for puro_fp8_gemm_blockwise.
  */
 PURO_API int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs,
                               uint16_t *C, int64_t M, int64_t N, int64_t K, int layout, puro_stream_t stream);

@@ -257,3 +257,4 @@ def test_mx_gemm_rejects_bad_arguments(lib):
     assert f(*ops, 128, 250, 256, 0, None) == ESHAPE
     assert f(*ops, 128, 256, 200, 2, None) == ESHAPE
     assert f(*ops[:4], A16 + 2, 128, 256, 256, 1, None) == EALIGN
+    assert f(*ops[:3], A16 + 4, A16, 128, 256, 256, 2, None) == EALIGN   # wgrad Bs 8-byte aligned
