@@ -63,7 +63,8 @@ def _args():
                    help="workload: 1 small outlier GEMM, 2 one layer's forward linears, 3 its backward, "
                         "4 the LM head, 5 the full 28-layer step (default), 'all' for 1-4 then 5, or "
                         "'fused' for the fused epilogue quantisation against GEMM + separate quantiser, "
-                        "'grouped' for one block's four wgrads in one launch against four")
+                        "'grouped' for one block's four wgrads in one launch against four, "
+                        "'scales' for the full step with FP32 scales against power-of-two scales")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions of configs 1-4")
     return p.parse_args()
 
@@ -189,11 +190,28 @@ class Clocks:
 # ------------------------------------------------------------------ the GPU step
 
 class Step:
-    """All buffers of one micro-step and the sequence of library calls over them."""
+    """All buffers of one micro-step and the sequence of library calls over them.
 
-    def __init__(self, pf, wl, tokens, layers, device, seed, group_wgrad=True):
+    scales="fp32": the method's scales (amax / 448 as FP32) and the blockwise GEMM;
+    scales="pow2": the power-of-two (UE8M0 byte) quantisers and the block-scaled GEMM
+    (one wgrad launch per linear: that GEMM has no grouped launch)."""
+
+    def __init__(self, pf, wl, tokens, layers, device, seed, group_wgrad=True, scales="fp32"):
         import torch
         self.pf, self.torch = pf, torch
+        if scales not in ("fp32", "pow2"):
+            raise ValueError(scales)
+        self.scales = scales
+        pow2 = scales == "pow2"
+        self._qw = pf.puro_fp8_quantize_128x128_pow2 if pow2 else pf.puro_fp8_quantize_128x128
+        self._qt = pf.puro_fp8_quantize_1x128_transposed_pow2 if pow2 else pf.puro_fp8_quantize_1x128_transposed
+        if pow2:
+            self._gemm = lambda a, sa, b, sb, c, lay, st: pf.puro_fp8_mx_gemm(a, sa, b, sb, c, lay, st)
+            group_wgrad = False
+        else:
+            self._gemm = lambda a, sa, b, sb, c, lay, st: pf.puro_fp8_gemm_blockwise(a, sa, b, sb, c, lay, None, st)
+        # grouped launches: one per block for its wgrads, one per 64 weights for the weights
+        self.group_weights = group_wgrad and not pow2
         T = tokens
         self.tokens = T
         self.linears = []  # (tag, X, W, dY, wq, wqt, ws, xqt, xst) in forward order
@@ -206,22 +224,24 @@ class Step:
         self.linears.append(["lm_head", h, w_head, dl])
         torch.cuda.synchronize()
         self.scratch = {}
-        u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
+        u8, bf = torch.uint8, torch.bfloat16
+        sdt = torch.uint8 if pow2 else torch.float32   # the scales' type
+        sb = 1 if pow2 else 4                          # bytes per scale
         for lin in self.linears:
             _, x, w, dy = lin
             n, k = w.shape
             lin += [torch.empty((n, k), dtype=u8, device=device),           # Wq
                     torch.empty((k, n), dtype=u8, device=device),           # WqT
-                    torch.empty(((n + 127) // 128, k // 128), dtype=f32, device=device),  # Ws
+                    torch.empty(((n + 127) // 128, k // 128), dtype=sdt, device=device),  # Ws
                     # X's codes along the tokens, made in the forward, used by wgrad
                     torch.empty((k, T), dtype=u8, device=device),           # XqT
-                    torch.empty((T // 128, k), dtype=f32, device=device)]   # XsT
+                    torch.empty((T // 128, k), dtype=sdt, device=device)]   # XsT
             if (n, k) not in self.scratch:
                 e = lambda *s, dt=u8: torch.empty(s, dtype=dt, device=device)
                 self.scratch[(n, k)] = dict(
-                    xq=e(T, k), xs=e(k // 128, T, dt=f32),
-                    dyq=e(T, n), dys=e(n // 128, T, dt=f32),
-                    dyqt=e(n, T), dyst=e(T // 128, n, dt=f32),
+                    xq=e(T, k), xs=e(k // 128, T, dt=sdt),
+                    dyq=e(T, n), dys=e(n // 128, T, dt=sdt),
+                    dyqt=e(n, T), dyst=e(T // 128, n, dt=sdt),
                     y=e(T, n, dt=bf), dx=e(T, k, dt=bf), dw=e(n, k, dt=bf))
         self.side = torch.cuda.Stream(device=device)  # weight quantisers and wgrad (overlap mode)
         self.gemm_flops = sum(3 * 2 * T * lin[2].shape[0] * lin[2].shape[1] for lin in self.linears)
@@ -229,22 +249,23 @@ class Step:
         qb = 0
         for _, x, w, dy, *_ in self.linears:
             n, k = w.shape
-            qb += T * k * (2 + 2) + 4 * (T * (k // 128) + (T // 128) * k)  # X dual
-            qb += n * k * (2 + 2) + 4 * (n // 128) * (k // 128)         # W + WqT
-            qb += T * n * (2 + 2) + 4 * (T * (n // 128) + (T // 128) * n)  # dY dual
+            qb += T * k * (2 + 2) + sb * (T * (k // 128) + (T // 128) * k)  # X dual
+            qb += n * k * (2 + 2) + sb * (n // 128) * (k // 128)         # W + WqT
+            qb += T * n * (2 + 2) + sb * (T * (n // 128) + (T // 128) * n)  # dY dual
         self.quant_bytes = qb
-        # algorithmic GEMM bytes: FP8 operands and FP32 scales read once, BF16 output written
+        # algorithmic GEMM bytes: FP8 operands and scales read once, BF16 output written
         gb = 0
         for _, x, w, dy, *_ in self.linears:
             n, k = w.shape
-            gb += T * k + n * k + 4 * (T * k // 128 + (n // 128) * (k // 128)) + 2 * T * n   # fprop
-            gb += T * n + n * k + 4 * (T * n // 128 + (n // 128) * (k // 128)) + 2 * T * k   # dgrad
-            gb += n * T + k * T + 4 * (n + k) * (T // 128) + 2 * n * k                      # wgrad
+            gb += T * k + n * k + sb * (T * k // 128 + (n // 128) * (k // 128)) + 2 * T * n   # fprop
+            gb += T * n + n * k + sb * (T * n // 128 + (n // 128) * (k // 128)) + 2 * T * k   # dgrad
+            gb += n * T + k * T + sb * (n + k) * (T // 128) + 2 * n * k                      # wgrad
         self.gemm_bytes = gb
         self.group_wgrad = group_wgrad
         n_wgrad = len({self.layer_of(i) for i in range(len(self.linears))}) if group_wgrad else len(self.linears)
         self.gemm_launches = 2 * len(self.linears) + n_wgrad
-        self.quant_launches = 3 * len(self.linears)
+        n_wquant = -(-len(self.linears) // 64) if self.group_weights else len(self.linears)
+        self.quant_launches = 2 * len(self.linears) + n_wquant
         self.launches_per_step = self.gemm_launches + self.quant_launches
 
     def run(self, ev=None, stream=None, overlap=False, before_fwd=None, before_bwd=None,
@@ -275,19 +296,26 @@ class Step:
             side.wait_stream(main)  # the previous step is done with every buffer
         w_ready = []
         with torch.cuda.stream(side):
-            for i, (tag, x, w, dy, wq, wqt, ws, xqt, xst) in enumerate(self.linears):
-                if before_fwd is not None:
-                    before_fwd(i, side)
-                pf.puro_fp8_quantize_128x128(w, wq, wqt, ws, side); rec("q")
-                w_ready.append(side.record_event() if overlap else None)
+            if self.group_weights and before_fwd is None:
+                # every weight is known before the forward: one grouped launch per 64 weights
+                pf.puro_fp8_quantize_128x128_grouped([lin[2:3] + lin[4:7] for lin in self.linears], side)
+                for _ in range(-(-len(self.linears) // 64)):
+                    rec("q")
+                w_ready = [side.record_event() if overlap else None] * len(self.linears)
+            else:  # per weight, each as soon as its inputs are there (the e2e run's copies)
+                for i, (tag, x, w, dy, wq, wqt, ws, xqt, xst) in enumerate(self.linears):
+                    if before_fwd is not None:
+                        before_fwd(i, side)
+                    self._qw(w, wq, wqt, ws, side); rec("q")
+                    w_ready.append(side.record_event() if overlap else None)
         for i, (tag, x, w, dy, wq, wqt, ws, xqt, xst) in enumerate(self.linears):
             if before_fwd is not None and overlap:
                 before_fwd(i, main)
             s = self.scratch[tuple(w.shape)]
-            pf.puro_fp8_quantize_1x128_transposed(x, xqt, xst, s["xq"], s["xs"], main); rec("q")
+            self._qt(x, xqt, xst, s["xq"], s["xs"], main); rec("q")
             if overlap:
                 main.wait_event(w_ready[i])
-            pf.puro_fp8_gemm_blockwise(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, None, main); rec("g")
+            self._gemm(s["xq"], s["xs"], wq, ws, s["y"], pf.PURO_FPROP, main); rec("g")
         wgrad_done = {}  # per shape: the last wgrad that read the shape's token-dim operands
         pending = []     # this layer's linears whose dY is quantised and whose wgrad is not issued
 
@@ -310,7 +338,7 @@ class Step:
                     pf.puro_fp8_gemm_blockwise_grouped(probs, pf.PURO_WGRAD, side); rec("g")
                 else:
                     for pr in probs:
-                        pf.puro_fp8_gemm_blockwise(*pr, pf.PURO_WGRAD, None, side); rec("g")
+                        self._gemm(*pr, pf.PURO_WGRAD, side); rec("g")
                 if after_wgrad is not None:
                     for i, pr in zip(pending, probs):
                         after_wgrad(i, pr[4], side)
@@ -330,8 +358,8 @@ class Step:
                 before_bwd(i, main)
             if overlap and key in wgrad_done:
                 main.wait_event(wgrad_done[key])  # the quantiser below overwrites its dY operands
-            pf.puro_fp8_quantize_1x128_transposed(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], main); rec("q")
-            pf.puro_fp8_gemm_blockwise(s["dyq"], s["dys"], wqt, ws, s["dx"], pf.PURO_DGRAD, None, main); rec("g")
+            self._qt(dy, s["dyqt"], s["dyst"], s["dyq"], s["dys"], main); rec("q")
+            self._gemm(s["dyq"], s["dys"], wqt, ws, s["dx"], pf.PURO_DGRAD, main); rec("g")
             pending.append(i)
             if not self.group_wgrad:
                 issue_wgrads()
@@ -627,9 +655,10 @@ def main():
     if args.impl == "reference":
         run_reference(args)
         return
-    if args.config in ("fused", "grouped"):
+    if args.config in ("fused", "grouped", "scales"):
         import bench_configs
-        {"fused": bench_configs.run_fused_comparison, "grouped": bench_configs.run_grouped_comparison}[args.config](args)
+        {"fused": bench_configs.run_fused_comparison, "grouped": bench_configs.run_grouped_comparison,
+         "scales": bench_configs.run_scales_comparison}[args.config](args)
         return
     if args.config in ("1", "2", "3", "4", "all"):
         from bench_configs import run_config

@@ -15,8 +15,9 @@ the full 28-layer micro-step, is bench.py's default line):
      logits, dlogits (both directions), dgrad, wgrad.
 
 Inputs are the seeded synthetic tensors of `workloads.py` (configuration c uses seed c - 1),
-resident in HBM. Every repetition first writes a 512 MB buffer, so no operand is left in
-the 126 MB L2 from the previous repetition; each launch is bracketed by CUDA events on the
+resident in HBM. Every repetition first writes a 512 MB buffer and reads it back, so no
+operand is left in the 126 MB L2 from the previous repetition and no dirty line is left for
+the timed kernels to write back; each launch is bracketed by CUDA events on the
 stream it runs on, and the median over repetitions is reported. The CPU oracle runs the
 same calls (on a bounded sample for the LM head) on the host cores beside it.
 """
@@ -34,6 +35,15 @@ from fp8_blockwise_scaled_e4m3_b200 import workloads as wl
 NOMINAL_HBM_GBS = 8000.0
 T4096 = 4096
 
+
+
+def flush_l2(buf):
+    """Evict the previous repetition's operands from the 126 MB L2: write a 512 MB buffer,
+    then read it back, so that L2 is left holding clean lines. (After the write alone it
+    would hold dirty lines, whose write-back to HBM would be charged to the next timed
+    kernel.)"""
+    buf.fill_(1.0)
+    return buf.sum()
 
 def _qbytes_rows(r, c):      # 1x128 row-wise: BF16 read, codes, scales
     return r * c * 3 + 4 * r * (c // 128)
@@ -208,7 +218,7 @@ def run_config(c, args):
         if rep == args.warmup:
             pf.puro_fp8_sync_status()
             t_begin = time.time()
-        flush.zero_()   # evicts the previous repetition's operands from L2
+        flush_l2(flush)
         evs = [torch.cuda.Event(enable_timing=True)]
         evs[0].record(stream)
         for op in ops:
@@ -234,7 +244,7 @@ def run_config(c, args):
     line = {"metric": METRIC, "n_gpus": 1, "steps": args.reps, "warmup": args.warmup,
             "dtype": "e4m3", "data": "synthetic", "scaling": "weak", "vs_baseline": None,
             "config": {"workload": desc, "config_index": c,
-                       "l2": "flushed before every repetition (512 MB write)"},
+                       "l2": "flushed before every repetition (512 MB written, then read back)"},
             "ms_per_step": round(ms_whole, 4), "gpu_launches": len(ops) * args.reps, "clocks": clk}
     if c == 1:
         line.update({"value": round(ms_whole * 1e3, 2), "unit": "us", "higher_is_better": False,
@@ -303,7 +313,7 @@ def run_fused_comparison(args):
         t = {"separate": [], "fused": []}
         for rep in range(args.warmup + args.reps):
             for kind, fn in (("separate", separate), ("fused", fused)):
-                flush.zero_()
+                flush_l2(flush)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 fn(stream)
@@ -320,7 +330,7 @@ def run_fused_comparison(args):
     tot_fus = sum(r["fused_us"] for r in rows)
     print(json.dumps({"comparison": "GEMM + separate 1x128 quantiser of its output vs the fused epilogue",
                       "workload": "fprop and dgrad of one Qwen3-1.7B-shaped block at 8192 tokens, seed 4",
-                      "l2": "flushed before every repetition", "reps": args.reps,
+                      "l2": "flushed before every repetition (512 MB written, then read back)", "reps": args.reps,
                       "total_separate_us": round(tot_sep, 1), "total_fused_us": round(tot_fus, 1),
                       "saved_pct": round(100 * (1 - tot_fus / tot_sep), 1), "ops": rows}), flush=True)
 
@@ -353,7 +363,7 @@ def run_grouped_comparison(args):
     t = {"separate": [], "grouped": []}
     for rep in range(args.warmup + args.reps):
         for kind, fn in (("separate", separate), ("grouped", grouped)):
-            flush.zero_()
+            flush_l2(flush)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn(stream)
@@ -365,7 +375,54 @@ def run_grouped_comparison(args):
     sep, grp = statistics.median(t["separate"]), statistics.median(t["grouped"])
     print(json.dumps({"comparison": "four wgrad launches vs one grouped launch",
                       "workload": "wgrads of one Qwen3-1.7B-shaped block (QKV, O, gate/up, down) at 8192 tokens, seed 4",
-                      "l2": "flushed before every repetition", "reps": args.reps,
+                      "l2": "flushed before every repetition (512 MB written, then read back)", "reps": args.reps,
                       "separate_us": round(sep * 1e3, 1), "grouped_us": round(grp * 1e3, 1),
                       "separate_tflops": round(flops / sep / 1e9, 1), "grouped_tflops": round(flops / grp / 1e9, 1),
                       "saved_pct": round(100 * (1 - grp / sep), 1)}), flush=True)
+
+
+def run_scales_comparison(args):
+    """The full micro-step (28 Qwen3-1.7B-shaped layers and the LM head at 8192 tokens,
+    fprop + dgrad + wgrad) in both scale modes, one after the other on the same seeded
+    inputs: the method's FP32 scales (amax / 448) with the blockwise GEMM, and power-of-two
+    UE8M0 scales with the block-scaled GEMM. Each mode: args.warmup untimed steps, then
+    `steps` steps between two CUDA events (inputs larger than L2), then one pass with an
+    event after every launch for the GEMM / quantiser split."""
+    from bench import Step
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    steps = max(1, min(args.steps, 10))
+    out = {}
+    for mode in ("fp32", "pow2"):
+        step = Step(pf, wl, args.tokens, args.layers, dev, seed=4, scales=mode)
+        for _ in range(args.warmup):
+            step.run(stream=stream, overlap=True)
+        pf.puro_fp8_sync_status()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step.run(stream=stream, overlap=True)
+        e1.record(stream)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        events = [("start", torch.cuda.Event(enable_timing=True))]
+        events[0][1].record(stream)
+        step.run(ev=events, stream=stream)
+        events[-1][1].synchronize()
+        pf.puro_fp8_sync_status()
+        t = {"g": 0.0, "q": 0.0}
+        for (_, a), (kind, b) in zip(events[:-1], events[1:]):
+            t[kind] += a.elapsed_time(b)
+        out[mode] = {"ms_per_step": round(ms, 3), "tflops": round(step.gemm_flops / (ms * 1e-3) / 1e12, 1),
+                     "gemm_ms": round(t["g"], 3), "gemm_tflops": round(step.gemm_flops / (t["g"] * 1e-3) / 1e12, 1),
+                     "quant_ms": round(t["q"], 3), "quant_gbs": round(step.quant_bytes / (t["q"] * 1e-3) / 1e9, 1),
+                     "launches": step.launches_per_step}
+        del step
+        torch.cuda.empty_cache()
+    print(json.dumps({"comparison": "full step, FP32 scales + blockwise GEMM vs power-of-two scales + "
+                                    "block-scaled GEMM",
+                      "workload": f"qwen3-1.7b-linear-stack-{args.layers}L+lm_head fwd+dgrad+wgrad, "
+                                  f"{args.tokens} tokens, seed 4",
+                      "steps": steps, "warmup": args.warmup, **out,
+                      "pow2_speedup": round(out["fp32"]["ms_per_step"] / out["pow2"]["ms_per_step"], 3)}),
+          flush=True)

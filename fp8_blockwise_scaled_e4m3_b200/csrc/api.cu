@@ -60,7 +60,7 @@ int check_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, const uint8
 }
 
 int check_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, const uint8_t *Wq,
-                 const uint8_t *WqT, const void *S, uintptr_t sa) {
+                 const uint8_t *WqT, const void *S, uintptr_t sa, bool device = true) {
   if (W == nullptr || Wq == nullptr || S == nullptr) return PURO_ERR_NULL;
   if (R < 1 || C < 128 || C % 128 != 0 || ldw < C) return PURO_ERR_SHAPE;
   if ((R + 127) / 128 > 65535 || C / 128 > (1ll << 31) - 1 || !tiles_fit(R, 128, C, 128))
@@ -68,7 +68,7 @@ int check_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, const uin
   if (WqT != nullptr && R % 16 != 0) return PURO_ERR_SHAPE;
   if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(S, sa) || ldw % 8 != 0) return PURO_ERR_ALIGN;
   if (WqT != nullptr && !aligned(WqT, 16)) return PURO_ERR_ALIGN;
-  return check_device();
+  return device ? check_device() : PURO_OK;
 }
 
 // The checks of one GEMM's arguments (every layout); PURO_OK or the status to return.
@@ -122,6 +122,20 @@ int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t l
                               uint8_t *WqT, float *S, puro_stream_t stream) {
   if (int e = check_weight(W, R, C, ldw, Wq, WqT, S, 4)) return e;
   return puro::launch_quant_weight(W, R, C, ldw, Wq, WqT, S, stream);
+}
+
+int puro_fp8_quantize_128x128_grouped(const puro_weight_problem *problems, int count, puro_stream_t stream) {
+  if (problems == nullptr) return PURO_ERR_NULL;
+  if (count < 1) return PURO_ERR_SHAPE;
+  int64_t tiles = 0;  // the joint tile numbering of a launch is 32-bit
+  for (int p = 0; p < count; ++p) {
+    const puro_weight_problem &w = problems[p];
+    if (int e = check_weight(w.W, w.R, w.C, w.ldw, w.Wq, w.WqT, w.S, 4, false)) return e;
+    tiles += ((w.R + 127) / 128) * (w.C / 128);
+    if (tiles > (1ll << 31) - 1) return PURO_ERR_SHAPE;
+  }
+  if (int d = check_device()) return d;
+  return puro::launch_quant_weight_grouped(problems, count, stream);
 }
 
 int puro_fp8_quantize_128x128_pow2(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,

@@ -70,9 +70,36 @@ struct QArgs {
   uint8_t *sb;       // P2: UE8M0 scale bytes in place of s
   uint8_t *stb;      // P2: UE8M0 scale bytes in place of st
   int tiles_r, tiles_c;
+  int tile_begin;    // first tile of this problem in the launch's joint tile sequence
   unsigned long long timeout_ns;
   int *status;
 };
+
+// Kernel parameters: G problems of the same mode (G = 1 for the single-tensor entry
+// points), their tensor maps and arguments passed by value as a __grid_constant__ (the
+// TMA unit reads the maps from the parameter space). Problem p owns tiles
+// [args[p].tile_begin, args[p].tile_begin + tiles_r * tiles_c) of the joint sequence.
+template <int G>
+struct alignas(64) QParams {
+  CUtensorMap tmX[G];
+  CUtensorMap tmT[G];
+  QArgs args[G];
+  int count;
+  int tiles;
+};
+constexpr int QGROUP_MAX = 64;  // weights per grouped launch (parameter space: 32 KB)
+static_assert(sizeof(QParams<QGROUP_MAX>) <= 32000, "kernel parameter space");
+
+// The problem that owns `tile`, searched forward from p (a CTA's tiles only increase).
+template <int G>
+__device__ __forceinline__ int problem_of(const QParams<G> &prm, int p, int tile) {
+  if constexpr (G == 1) {
+    return 0;
+  } else {
+    while (p + 1 < prm.count && tile >= prm.args[p + 1].tile_begin) ++p;
+    return p;
+  }
+}
 
 __device__ int g_quant_status;  // non-zero: a bounded wait gave up since the last read
 
@@ -158,10 +185,9 @@ __device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[TG],
 
 // P2: power-of-two scales (UE8M0 bytes) instead of the method's FP32 amax / 448; the codes
 // then come out of the same fast path exactly as x * 2^-e (see pow2_scale).
-template <int MODE, bool P2>
+template <int MODE, bool P2, int G>
 __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
-    k_quant_tiles(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
-                  const QArgs args) {
+    k_quant_tiles(const __grid_constant__ QParams<G> prm) {
   constexpr bool kRows = MODE == Q_ROWS || MODE == Q_DUAL;
   constexpr bool kCols = MODE == Q_COLS || MODE == Q_DUAL;
   constexpr bool kWeight = MODE == Q_WEIGHT;
@@ -183,29 +209,40 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int tiles = args.tiles_r * args.tiles_c;
-  const bool write_t = kCols || (kWeight && args.write_t);
+  const int tiles = prm.tiles;
+  const unsigned long long timeout_ns = prm.args[0].timeout_ns;
+  int *const status = prm.args[0].status;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
     *fail = 0;
     fence_barrier_init();
-    prefetch_tensormap(&tmX);
-    if (write_t) prefetch_tensormap(&tmT);
+    const int p0 = problem_of(prm, 0, blockIdx.x < tiles ? blockIdx.x : 0);
+    prefetch_tensormap(&prm.tmX[p0]);
+    if (kCols || (kWeight && prm.args[p0].write_t)) prefetch_tensormap(&prm.tmT[p0]);
   }
   __syncthreads();
 
   // Tile i of this CTA is global tile blockIdx.x + i * gridDim.x; stage i % kStages.
+  int p_issue = 0;  // thread 0: the problem of the last tile it issued
   auto issue = [&](int i) {
     const int tile = blockIdx.x + i * gridDim.x;
     if (tile >= tiles) return;
-    const int tr = tile / args.tiles_c, tc = tile % args.tiles_c;
+    const int p = problem_of(prm, p_issue, tile);
+    if (p != p_issue) {
+      prefetch_tensormap(&prm.tmX[p]);
+      if (kCols || (kWeight && prm.args[p].write_t)) prefetch_tensormap(&prm.tmT[p]);
+      p_issue = p;
+    }
+    const QArgs &a = prm.args[p];
+    const int lt = tile - a.tile_begin;
+    const int tr = lt / a.tiles_c, tc = lt % a.tiles_c;
     const int s = i % kStages;
     const uint32_t bar = bar0 + 8 * s;
     const uint32_t dst = sbase + s * kStageBytes;
     mbar_arrive_expect_tx(bar, kStageBytes);
-    tma_load_2d(dst, &tmX, bar, tc * kTile, tr * kTile);
-    tma_load_2d(dst + kBoxBytes, &tmX, bar, tc * kTile + 64, tr * kTile);
+    tma_load_2d(dst, &prm.tmX[p], bar, tc * kTile, tr * kTile);
+    tma_load_2d(dst + kBoxBytes, &prm.tmX[p], bar, tc * kTile + 64, tr * kTile);
   };
   if (tid == 0)
     for (int i = 0; i < kStages; ++i) issue(i);
@@ -213,17 +250,23 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
   const int rg = tid >> 3, j8 = tid & 7;   // row group and its lane in the row phase
   const int cp = tid & 63, g = tid >> 6;
   int i = 0;
+  int prob = 0;           // the problem of the current tile
+  bool any_t = false;     // thread 0: a transposed store was issued
   for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++i) {
     const int s = i % kStages;
-    const int tr = tile / args.tiles_c, tc = tile % args.tiles_c;
+    prob = problem_of(prm, prob, tile);
+    const QArgs &args = prm.args[prob];
+    const bool write_t = kCols || (kWeight && args.write_t);
+    const int lt = tile - args.tile_begin;
+    const int tr = lt / args.tiles_c, tc = lt % args.tiles_c;
     const int64_t r0 = static_cast<int64_t>(tr) * kTile;
     const int64_t c0 = static_cast<int64_t>(tc) * kTile;
     const uint8_t *stage = smem + s * kStageBytes;
-    const bool waited = mbar_wait(bar0 + 8 * s, (i / kStages) & 1, args.timeout_ns, fail);
+    const bool waited = mbar_wait(bar0 + 8 * s, (i / kStages) & 1, timeout_ns, fail);
     if (__syncthreads_or(!waited)) {
       if (tid == 0) {
         *fail = 1;
-        atomicOr(args.status, 1);
+        atomicOr(status, 1);
       }
       break;
     }
@@ -394,21 +437,22 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
     __syncthreads();  // the stage and (if any) the code tile are complete
     if (tid == 0) {
       if (write_t) {
-        tma_store_2d(&tmT, sbase + kOffCodes, static_cast<int32_t>(r0), static_cast<int32_t>(c0));
+        tma_store_2d(&prm.tmT[prob], sbase + kOffCodes, static_cast<int32_t>(r0), static_cast<int32_t>(c0));
         bulk_commit_group();
+        any_t = true;
       }
       issue(i + kStages);  // refill the stage just consumed
     }
   }
 
   if (tid == 0) {
-    if (write_t) bulk_wait_group_all();
+    if (any_t) bulk_wait_group_all();
     if (*fail) {
       // Let every load still in flight land before the CTA exits (bounded).
       for (int k = 0; k < kStages; ++k) {
         const int ii = i + k;
         if (blockIdx.x + ii * gridDim.x < tiles)
-          mbar_wait(bar0 + 8 * (ii % kStages), (ii / kStages) & 1, args.timeout_ns, nullptr);
+          mbar_wait(bar0 + 8 * (ii % kStages), (ii / kStages) & 1, timeout_ns, nullptr);
       }
     }
   }
@@ -459,23 +503,14 @@ unsigned long long wait_timeout_ns() {
   return ns;
 }
 
-template <int MODE, bool P2>
-int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *qt, QArgs args,
-                 cudaStream_t stream) {
-  int sms = 0;
-  if (!sm_count(sms)) return PURO_ERR_CUDA;
-  static PerDevice<int *> status_addr;  // g_quant_status on this device, looked up once
-  if (!status_addr.get(args.status, [](int, int *&v) {
-        return cudaGetSymbolAddress(reinterpret_cast<void **>(&v), g_quant_status) == cudaSuccess;
-      }))
-    return PURO_ERR_CUDA;
-  CUtensorMap tmX, tmT;
-  if (!make_map(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, C, ldx, kTile, 64))
-    return PURO_ERR_CUDA;
+// Fills the tensor maps and the sizes of one problem; the caller's args carry the outputs.
+template <int MODE>
+bool set_problem(CUtensorMap &tmX, CUtensorMap &tmT, QArgs &args, const uint16_t *X, int64_t R, int64_t C,
+                 int64_t ldx, uint8_t *qt) {
+  if (!make_map(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, C, ldx, kTile, 64)) return false;
   if (qt != nullptr) {
     // the transposed codes [C, R]: one box of 128 rows (tile columns) x 128 bytes
-    if (!make_map(&tmT, qt, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, C, R, R, kTile, kTile))
-      return PURO_ERR_CUDA;
+    if (!make_map(&tmT, qt, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, C, R, R, kTile, kTile)) return false;
   } else {
     tmT = tmX;  // unused
   }
@@ -484,9 +519,23 @@ int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *
   args.tiles_r = static_cast<int>((R + kTile - 1) / kTile);
   args.tiles_c = static_cast<int>((C + kTile - 1) / kTile);
   args.timeout_ns = wait_timeout_ns();
-  const int64_t tiles = static_cast<int64_t>(args.tiles_r) * args.tiles_c;
-  const int grid = static_cast<int>(tiles < kCtasPerSm * sms ? tiles : kCtasPerSm * sms);
-  auto kern = k_quant_tiles<MODE, P2>;
+  return true;
+}
+
+// Launches k_quant_tiles<MODE, P2, G> over prm (its problems, count and tiles filled in).
+template <int MODE, bool P2, int G>
+int launch_params(QParams<G> &prm, cudaStream_t stream) {
+  int sms = 0;
+  if (!sm_count(sms)) return PURO_ERR_CUDA;
+  static PerDevice<int *> status_addr;  // g_quant_status on this device, looked up once
+  int *st = nullptr;
+  if (!status_addr.get(st, [](int, int *&v) {
+        return cudaGetSymbolAddress(reinterpret_cast<void **>(&v), g_quant_status) == cudaSuccess;
+      }))
+    return PURO_ERR_CUDA;
+  for (int p = 0; p < prm.count; ++p) prm.args[p].status = st;
+  const int grid = prm.tiles < kCtasPerSm * sms ? prm.tiles : kCtasPerSm * sms;
+  auto kern = k_quant_tiles<MODE, P2, G>;
   static PerDevice<bool> smem_opt_in;  // dynamic shared memory opted in once per device
   bool done = false;
   if (!smem_opt_in.get(done, [&](int, bool &v) {
@@ -495,13 +544,25 @@ int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *
         return v;
       }))
     return PURO_ERR_CUDA;
-  kern<<<grid, Threads<MODE>::value, kSmemBytes, stream>>>(tmX, tmT, args);
+  kern<<<grid, Threads<MODE>::value, kSmemBytes, stream>>>(prm);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     std::fprintf(stderr, "puro_fp8: quantiser launch: %s\n", cudaGetErrorString(e));
     return PURO_ERR_LAUNCH;
   }
   return PURO_OK;
+}
+
+template <int MODE, bool P2>
+int launch_tiles(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *qt, QArgs args,
+                 cudaStream_t stream) {
+  QParams<1> prm;
+  prm.args[0] = args;
+  if (!set_problem<MODE>(prm.tmX[0], prm.tmT[0], prm.args[0], X, R, C, ldx, qt)) return PURO_ERR_CUDA;
+  prm.args[0].tile_begin = 0;
+  prm.count = 1;
+  prm.tiles = prm.args[0].tiles_r * prm.args[0].tiles_c;
+  return launch_params<MODE, P2, 1>(prm, stream);
 }
 
 }  // namespace
@@ -546,6 +607,32 @@ int launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, ui
   a.write_t = WqT != nullptr;
   return Sb != nullptr ? launch_tiles<Q_WEIGHT, true>(W, R, C, ldw, WqT, a, stream)
                        : launch_tiles<Q_WEIGHT, false>(W, R, C, ldw, WqT, a, stream);
+}
+
+int launch_quant_weight_grouped(const WeightProblem *probs, int count, cudaStream_t stream) {
+  // Up to QGROUP_MAX weights per launch; the parameter block lives on the host stack only
+  // until the launch has copied it.
+  static thread_local QParams<QGROUP_MAX> prm;
+  for (int first = 0; first < count; first += QGROUP_MAX) {
+    const int n = count - first < QGROUP_MAX ? count - first : QGROUP_MAX;
+    int tiles = 0;
+    for (int k = 0; k < n; ++k) {
+      const WeightProblem &w = probs[first + k];
+      QArgs a{};
+      a.q = w.Wq;
+      a.ldq = w.C;
+      a.s = w.S;
+      a.write_t = w.WqT != nullptr;
+      if (!set_problem<Q_WEIGHT>(prm.tmX[k], prm.tmT[k], a, w.W, w.R, w.C, w.ldw, w.WqT)) return PURO_ERR_CUDA;
+      a.tile_begin = tiles;
+      tiles += a.tiles_r * a.tiles_c;
+      prm.args[k] = a;
+    }
+    prm.count = n;
+    prm.tiles = tiles;
+    if (int e = launch_params<Q_WEIGHT, false, QGROUP_MAX>(prm, stream)) return e;
+  }
+  return PURO_OK;
 }
 
 int read_and_clear_quant_status(cudaStream_t stream, int *status_out) {

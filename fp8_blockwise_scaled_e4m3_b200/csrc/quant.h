@@ -20,6 +20,10 @@ int launch_quant_cols(const uint16_t *X, int64_t T, int64_t C, int64_t ldx, uint
 int launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, uint8_t *Wq,
                         uint8_t *WqT, float *S, cudaStream_t stream, uint8_t *Sb = nullptr);
 
+// Many weights' 128x128 quantisations in persistent launches of up to 64 weights each.
+using WeightProblem = puro_weight_problem;
+int launch_quant_weight_grouped(const WeightProblem *problems, int count, cudaStream_t stream);
+
 // Reads and clears the quantisers' device status word (after a stream sync).
 int read_and_clear_quant_status(cudaStream_t stream, int *status_out);
 
@@ -28,7 +32,8 @@ int launch_gemm_blockwise(const uint8_t *Aq, const float *As, const uint8_t *Bq,
                           uint16_t *C, int64_t M, int64_t N, int64_t K, int layout,
                           cudaStream_t stream);
 
-// Up to 8 GEMMs of one layout in one persistent launch (see puro_fp8_gemm_blockwise_grouped).
+// Up to PURO_GROUP_MAX GEMMs of one layout in one persistent launch (see
+// puro_fp8_gemm_blockwise_grouped).
 using GroupedProblem = puro_gemm_problem;
 int launch_gemm_blockwise_grouped(const GroupedProblem *problems, int count, int layout,
                                   cudaStream_t stream);

@@ -32,6 +32,12 @@ class GemmProblem(ctypes.Structure):
                 ("M", _i64), ("N", _i64), ("K", _i64)]
 
 
+class WeightProblem(ctypes.Structure):
+    """puro_weight_problem: one weight of a grouped 128x128 quantisation."""
+    _fields_ = [("W", _p), ("R", _i64), ("C", _i64), ("ldw", _i64),
+                ("Wq", _p), ("WqT", _p), ("S", _p)]
+
+
 class PuroError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -52,6 +58,7 @@ def _load():
         "puro_fp8_gemm_wgrad_acc_f32": [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p],
         "puro_fp8_gemm_blockwise_quant": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p],
         "puro_fp8_gemm_blockwise_grouped": [_p, ctypes.c_int, ctypes.c_int, _p],
+        "puro_fp8_quantize_128x128_grouped": [_p, ctypes.c_int, _p],
         "puro_fp8_quantize_1x128_pow2": [_p, _i64, _i64, _i64, _p, _i64, _p, _p],
         "puro_fp8_mx_gemm": [_p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p],
         "puro_fp8_quantize_1x128_transposed_pow2": [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
@@ -172,6 +179,30 @@ def puro_fp8_quantize_128x128(W, Wq, WqT, S, stream=None):
         st = _stream(stream)  # the current stream of the tensors' device
         _check(_lib.puro_fp8_quantize_128x128(_ptr(W), R, C, W.stride(0), _ptr(Wq), _ptr(WqT), _ptr(S),
                                               st), "puro_fp8_quantize_128x128", st)
+
+
+def puro_fp8_quantize_128x128_grouped(problems, stream=None):
+    """problems: sequence of (W, Wq, WqT or None, S) tensor tuples, each checked as for
+    puro_fp8_quantize_128x128; quantised in one launch per 64 weights (see the C declaration)."""
+    if len(problems) < 1:
+        raise ValueError("at least one weight")
+    arr = (WeightProblem * len(problems))()
+    dev = problems[0][0].device
+    for i, (W, Wq, WqT, S) in enumerate(problems):
+        R, C = _matrix(W, "W")
+        _shape(Wq, (R, C), "Wq"); _shape(WqT, (C, R), "WqT"); _shape(S, ((R + 127) // 128, C // 128), "S")
+        _need(W, torch.bfloat16, "W"); _need(Wq, torch.uint8, "Wq"); _need(WqT, torch.uint8, "WqT")
+        _need(S, torch.float32, "S")
+        for t, n in ((W, "W"), (Wq, "Wq"), (WqT, "WqT"), (S, "S")):
+            if t is not None and t.device != dev:
+                raise ValueError("all weights of a group must be on one device")
+            if n != "W":
+                _dense(t, n)
+        arr[i] = WeightProblem(W.data_ptr(), R, C, W.stride(0), Wq.data_ptr(), _ptr(WqT), S.data_ptr())
+    with torch.cuda.device(dev):
+        st = _stream(stream)  # the current stream of the tensors' device
+        _check(_lib.puro_fp8_quantize_128x128_grouped(ctypes.cast(arr, _p), len(problems), st),
+               "puro_fp8_quantize_128x128_grouped", st)
 
 
 def _gemm_shapes(Aq, As, Bq, Bs, C, bs_shape):

@@ -124,6 +124,32 @@ PURO_API int puro_fp8_quantize_1x128_transposed(const uint16_t *X, int64_t T, in
 PURO_API int puro_fp8_quantize_128x128(const uint16_t *W, int64_t R, int64_t C, int64_t ldw,
                               uint8_t *Wq, uint8_t *WqT, float *S, puro_stream_t stream);
 
+/* One weight of puro_fp8_quantize_128x128_grouped: the arguments of
+ * puro_fp8_quantize_128x128 for it. */
+typedef struct {
+  const uint16_t *W; /* [R, C] BF16, row stride ldw       */
+  int64_t R, C, ldw;
+  uint8_t *Wq;       /* [R, C] codes, dense               */
+  uint8_t *WqT;      /* [C, R] codes, dense, or NULL      */
+  float *S;          /* [ceil(R/128), C/128] scales       */
+} puro_weight_problem;
+
+/*
+ * The 128x128 quantisation of `count` weights, each exactly what puro_fp8_quantize_128x128
+ * with its arguments writes (bit for bit), in one persistent launch per 64 weights instead of
+ * one launch per weight. Source: "Lever 2: use blockwise FP8 from step zero" -- weights in
+ * 128x128 blocks, converted to FP8 for the GEMMs that consume them. All weights of a model
+ * are known before its forward pass, so a step can quantise them together: the CTAs walk the
+ * weights' tiles as one sequence and one weight's tiles fill the SMs another's last wave
+ * leaves idle. The problem array is read during the call only (the host copies it into the
+ * launches' parameters).
+ * Requires count >= 1 and, for every weight, what puro_fp8_quantize_128x128 requires; the
+ * outputs of different weights must not overlap. Nothing is launched unless every weight
+ * passes the checks. Status codes as for puro_fp8_quantize_128x128.
+ */
+PURO_API int puro_fp8_quantize_128x128_grouped(const puro_weight_problem *problems, int count,
+                                               puro_stream_t stream);
+
 /*
  * Power-of-two (UE8M0) scale mode of the three quantisers above: the same groups, codes
  * written the same way, but each group's scale is the method's amax / 448 rounded up to a

@@ -46,6 +46,7 @@ def test_header_declares_the_entry_points():
         "puro_fp8_gemm_blockwise", "puro_fp8_gemm_wgrad_acc_f32", "puro_fp8_gemm_blockwise_quant",
         "puro_fp8_gemm_blockwise_grouped", "puro_fp8_quantize_1x128_pow2",
         "puro_fp8_quantize_1x128_transposed_pow2", "puro_fp8_quantize_128x128_pow2", "puro_fp8_mx_gemm",
+        "puro_fp8_quantize_128x128_grouped",
         "puro_fp8_sync_status", "puro_strerror"])
 
 
@@ -232,6 +233,28 @@ def test_gemm_grouped_rejects_bad_arguments(lib):
     assert f(ptr, 2, 2, None) == ENULL
     arr[1] = GemmProblem(A16, A16, A16, A16, A16 + 8, 128, 256, 256)  # C not 16-byte aligned
     assert f(ptr, 2, 1, None) == EALIGN
+
+
+def test_quantize_grouped_rejects_bad_arguments(lib):
+    """The grouped weight quantiser checks the count and every weight as the single call
+    does, before anything is launched; one bad weight rejects the whole call."""
+    from fp8_blockwise_scaled_e4m3_b200.puro_fp8 import WeightProblem
+    f = lib.puro_fp8_quantize_128x128_grouped
+    good = WeightProblem(A16, 256, 256, 256, A16, A16, A16)
+    arr = (WeightProblem * 3)(good, good, good)
+    ptr = ctypes.cast(arr, ctypes.c_void_p)
+    assert f(None, 2, None) == ENULL
+    assert f(ptr, 0, None) == ESHAPE
+    arr[2] = WeightProblem(A16, 100, 256, 256, A16, A16, A16)    # WqT needs R % 16
+    assert f(ptr, 3, None) == ESHAPE
+    arr[2] = WeightProblem(A16, 128, 200, 256, A16, None, A16)   # C % 128
+    assert f(ptr, 3, None) == ESHAPE
+    arr[2] = WeightProblem(A16, 128, 256, 256, None, None, A16)  # Wq
+    assert f(ptr, 3, None) == ENULL
+    arr[2] = WeightProblem(A16, 128, 256, 252, A16, None, A16)   # ldw < C
+    assert f(ptr, 3, None) == ESHAPE
+    arr[2] = WeightProblem(A16, 128, 256, 256, A16, None, A16 + 2)  # S not 4-byte aligned
+    assert f(ptr, 3, None) == EALIGN
 
 
 def test_pow2_quantisers_reject_bad_arguments(lib):
