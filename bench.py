@@ -46,6 +46,14 @@ FP8_DENSE_PEAK_TFLOPS = 4500.0  # nominal B200 dense FP8
 WORKLOAD = "qwen3-1.7b-linear-stack-28L+lm_head fwd+dgrad+wgrad, 8192 tokens (2x4096)"
 
 
+def workload_name(args):
+    """WORKLOAD for the default sizes; the same form for a reduced (profiling) step."""
+    if args.layers == 28 and args.tokens == 8192 and not args.no_lm_head:
+        return WORKLOAD
+    head = "" if args.no_lm_head else "+lm_head"
+    return f"qwen3-1.7b-linear-stack-{args.layers}L{head} fwd+dgrad+wgrad, {args.tokens} tokens"
+
+
 def _args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -57,6 +65,8 @@ def _args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-lm-head", action="store_true",
+                   help="leave the LM head out of the step (small profiling cases with --layers)")
     p.add_argument("--no-group", action="store_true",
                    help="one wgrad launch per linear instead of one grouped launch per block")
     p.add_argument("--config", default="5",
@@ -80,10 +90,10 @@ def _peaks():
 
 # ------------------------------------------------------------------ DRAM traffic (ncu)
 
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "dram_traffic_qwen3_28L_lmhead_8192tok.md")
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "dram_traffic_qwen3_1layer_8192tok.md")
 KERNEL_SOURCES = {
-    "gemm": ["gemm.cu", "ptx.cuh"],
-    "quant": ["quant.cu", "quant_math.cuh", "ptx.cuh"],
+    "gemm": ["gemm.cu", "ptx.cuh", "quant_math.cuh", "host_cache.h"],
+    "quant": ["quant.cu", "quant_math.cuh", "ptx.cuh", "host_cache.h"],
 }
 
 
@@ -96,20 +106,21 @@ def sources_sha256(kind):
     return h.hexdigest()
 
 
-def ncu_traffic(kind):
-    """DRAM bytes (read + write) per launch of a kernel family, averaged over one step, as
-    recorded in the committed ncu summary; None if there is none or the family's sources
-    changed since it was captured."""
+def ncu_traffic(kind, algorithmic_bytes_per_launch):
+    """DRAM bytes (read + write) per launch of a kernel family in the step, from the committed
+    ncu summary of one 8192-token layer (the step's own shapes): that capture's DRAM bytes
+    over its algorithmic bytes, times the step's algorithmic bytes per launch. None if there
+    is no summary or the family's sources changed since it was captured."""
     try:
         with open(TRAFFIC_SUMMARY) as f:
             text = f.read()
     except OSError:
         return None
     sha = re.search(rf"^{kind}_sources_sha256: ([0-9a-f]{{64}})$", text, re.M)
-    val = re.search(rf"^{kind}_dram_bytes_per_launch: (\d+)$", text, re.M)
+    val = re.search(rf"^{kind}_dram_over_algorithmic: ([0-9.]+)$", text, re.M)
     if sha is None or val is None or sha.group(1) != sources_sha256(kind):
         return None
-    return int(val.group(1))
+    return round(float(val.group(1)) * algorithmic_bytes_per_launch)
 
 
 # ------------------------------------------------------------------ clocks sampler
@@ -196,7 +207,7 @@ class Step:
     scales="pow2": the power-of-two (UE8M0 byte) quantisers and the block-scaled GEMM
     (one wgrad launch per linear: that GEMM has no grouped launch)."""
 
-    def __init__(self, pf, wl, tokens, layers, device, seed, group_wgrad=True, scales="fp32"):
+    def __init__(self, pf, wl, tokens, layers, device, seed, group_wgrad=True, scales="fp32", lm_head=True):
         import torch
         self.pf, self.torch = pf, torch
         if scales not in ("fp32", "pow2"):
@@ -220,8 +231,9 @@ class Step:
             grads = wl.layer_grads(seed, T, device, layer=l)
             for (name, x, w), (_, dy) in zip(fwd, grads):
                 self.linears.append([f"L{l}.{name}", x, w, dy])
-        h, w_head, dl = wl.lm_head(seed, T, device)
-        self.linears.append(["lm_head", h, w_head, dl])
+        if lm_head:
+            h, w_head, dl = wl.lm_head(seed, T, device)
+            self.linears.append(["lm_head", h, w_head, dl])
         torch.cuda.synchronize()
         self.scratch = {}
         u8, bf = torch.uint8, torch.bfloat16
@@ -490,7 +502,8 @@ def run_ours(args):
     device = torch.device("cuda", torch.cuda.current_device())
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
 
-    step = Step(pf, wl, args.tokens, args.layers, device, seed=4 + 1000 * rank, group_wgrad=not args.no_group)
+    step = Step(pf, wl, args.tokens, args.layers, device, seed=4 + 1000 * rank, group_wgrad=not args.no_group,
+                lm_head=not args.no_lm_head)
     stream = torch.cuda.current_stream()
 
     clocks = Clocks(torch.cuda.current_device())
@@ -542,8 +555,8 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens_per_gpu": args.tokens, "layers": args.layers,
-                   "lm_head": True, "gemm_tflop_per_step": round(step.gemm_flops / 1e12, 4),
+        "config": {"workload": workload_name(args), "tokens_per_gpu": args.tokens, "layers": args.layers,
+                   "lm_head": not args.no_lm_head, "gemm_tflop_per_step": round(step.gemm_flops / 1e12, 4),
                    "quant_gb_per_step": round(step.quant_bytes / 1e9, 3),
                    "l2": "inputs larger than L2: %.1f GB of distinct BF16 inputs read per step" % (
                        sum(t.numel() * 2 for lin in step.linears for t in lin[1:4]) / 1e9),
@@ -554,14 +567,15 @@ def run_ours(args):
                      "frac": round(gemm_tflops / fp8_peak_measured, 4),
                      "peak_note": f"2 x {peak_src} sustained BF16 ({bf16_tf_sus}); "
                                   f"frac of nominal 4.5 PF = {gemm_tflops / FP8_DENSE_PEAK_TFLOPS:.4f}",
-                     "traffic": ncu_traffic("gemm"),
-                     "traffic_unit": "DRAM bytes per launch (ncu, one step, mean over launches)",
+                     "traffic": ncu_traffic("gemm", step.gemm_bytes / step.gemm_launches),
+                     "traffic_unit": "DRAM bytes per launch (ncu on one 8192-token layer, scaled to the "
+                                     "step's algorithmic bytes per launch)",
                      "algorithmic_bytes_per_launch": round(step.gemm_bytes / step.gemm_launches),
                      "launches_measured": n_gemm, "avg_launch_ms": round(t_gemm / max(n_gemm, 1), 4)},
         "roofline_quant": {"bound": "hbm", "kernel": "k_quant_tiles (dual X and dY, 128x128 weight + WqT launches)",
                            "achieved": round(quant_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                            "frac": round(quant_gbs / hbm_gbs, 4),
-                           "traffic": ncu_traffic("quant"),
+                           "traffic": ncu_traffic("quant", step.quant_bytes / step.quant_launches),
                            "algorithmic_bytes_per_launch": round(step.quant_bytes / step.quant_launches),
                            "peak_note": f"{peak_src} copy bandwidth; frac of nominal 8 TB/s = "
                                         f"{quant_gbs / 8000:.4f}",

@@ -394,7 +394,7 @@ def run_scales_comparison(args):
     steps = max(1, min(args.steps, 10))
     out = {}
     for mode in ("fp32", "pow2"):
-        step = Step(pf, wl, args.tokens, args.layers, dev, seed=4, scales=mode)
+        step = Step(pf, wl, args.tokens, args.layers, dev, seed=4, scales=mode, lm_head=not args.no_lm_head)
         for _ in range(args.warmup):
             step.run(stream=stream, overlap=True)
         pf.puro_fp8_sync_status()
@@ -421,7 +421,8 @@ def run_scales_comparison(args):
         torch.cuda.empty_cache()
     print(json.dumps({"comparison": "full step, FP32 scales + blockwise GEMM vs power-of-two scales + "
                                     "block-scaled GEMM",
-                      "workload": f"qwen3-1.7b-linear-stack-{args.layers}L+lm_head fwd+dgrad+wgrad, "
+                      "workload": f"qwen3-1.7b-linear-stack-{args.layers}L"
+                                  f"{'' if args.no_lm_head else '+lm_head'} fwd+dgrad+wgrad, "
                                   f"{args.tokens} tokens, seed 4",
                       "steps": steps, "warmup": args.warmup, **out,
                       "pow2_speedup": round(out["fp32"]["ms_per_step"] / out["pow2"]["ms_per_step"], 3)}),
