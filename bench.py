@@ -527,6 +527,18 @@ def run_ours(args):
     ms_total = start.elapsed_time(end)
     ms_total = _max_over_ranks(ms_total, world)
 
+    # Host enqueue cost: the wall time of issuing one step's launches (argument checks,
+    # tensor maps, launches; no synchronisation inside), each step started on an idle GPU
+    # so that no launch waits for room in the queue.
+    host_ms = []
+    for _ in range(3):
+        torch.cuda.synchronize()
+        h0 = time.perf_counter()
+        step.run(stream=stream, overlap=True)
+        host_ms.append((time.perf_counter() - h0) * 1e3)
+    torch.cuda.synchronize()
+    pf.puro_fp8_sync_status()
+
     # Kernel-level pass after the timed region: an event after every launch gives each
     # kernel's duration for the rooflines.
     kernel_steps = max(1, min(args.steps, 5))
@@ -581,6 +593,7 @@ def run_ours(args):
                                         f"{quant_gbs / 8000:.4f}",
                            "launches_measured": n_quant, "avg_launch_ms": round(t_quant / max(n_quant, 1), 4)},
         "gpu_launches": step.launches_per_step * args.steps,
+        "host_enqueue_ms_per_step": round(statistics.median(host_ms), 3),
         "clocks": clk,
     }
 
