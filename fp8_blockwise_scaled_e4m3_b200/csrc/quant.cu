@@ -158,16 +158,13 @@ __device__ __forceinline__ void column_codes_to_smem(const uint32_t (&w)[TG],
 #pragma unroll
   for (int i = 0; i < TG / 4; ++i) {
     // column 2cp is the low half of each word, column 2cp+1 the high half
-    const uint32_t a0 = __byte_perm(w[4 * i], w[4 * i + 1], 0x5410);
-    const uint32_t a1 = __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x5410);
-    const uint32_t b0 = __byte_perm(w[4 * i], w[4 * i + 1], 0x7632);
-    const uint32_t b1 = __byte_perm(w[4 * i + 2], w[4 * i + 3], 0x7632);
+    const uint32_t *wi = &w[4 * i];
     if constexpr (FAST) {
-      q0[i] = block_codes4_fast(a0, a1, pack2(-div0.r, -div0.r), pack2(div0.s, div0.s));
-      q1[i] = block_codes4_fast(b0, b1, pack2(-div1.r, -div1.r), pack2(div1.s, div1.s));
+      q0[i] = half_codes4_fast<false>(wi[0], wi[1], wi[2], wi[3], pack2(-div0.r, -div0.r), pack2(div0.s, div0.s));
+      q1[i] = half_codes4_fast<true>(wi[0], wi[1], wi[2], wi[3], pack2(-div1.r, -div1.r), pack2(div1.s, div1.s));
     } else {
-      q0[i] = block_codes4(a0, a1, div0);
-      q1[i] = block_codes4(b0, b1, div1);
+      q0[i] = block_codes4(__byte_perm(wi[0], wi[1], 0x5410), __byte_perm(wi[2], wi[3], 0x5410), div0);
+      q1[i] = block_codes4(__byte_perm(wi[0], wi[1], 0x7632), __byte_perm(wi[2], wi[3], 0x7632), div1);
     }
   }
   const int r0 = 2 * cp, r1 = 2 * cp + 1;
@@ -305,33 +302,42 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
       // every block the warp holds allows it (the slow path only serves tiny, infinite
       // or NaN maxima).
       constexpr int NP = kTile / RSTEP;
+      static_assert(NP <= 8, "one lane of the row's 8 forms each of a thread's row scales");
       uint4 v0[NP], v1[NP];
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
         v0[p] = row_chunk(stage, rg + RSTEP * p, 0, j8);
         v1[p] = row_chunk(stage, rg + RSTEP * p, 1, j8);
       }
-      float srow[NP], amax[NP];
-      uint32_t brow[NP];  // P2: scale bytes
+      // One lane per row forms the row's scale and divider (lane j8 of the row group takes
+      // row p = j8) and shares the divider by shuffle; it also writes the row's scale.
+      float srow_mine = 0.0f;   // lane j8 < NP: the scale of its row p = j8
+      uint32_t brow_mine = 0u;  // P2: its scale byte
+      uint32_t m[NP];
       BlockDivider div[NP];
       bool ok = true;
       if (kRows) {
-        uint32_t m[NP];
 #pragma unroll
         for (int p = 0; p < NP; ++p) m[p] = absmax16(v0[p], v1[p]);
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1)
 #pragma unroll
           for (int p = 0; p < NP; ++p) m[p] = bf16x2_absmax(m[p], __shfl_xor_sync(0xffffffffu, m[p], o));
+        uint32_t mm = 0u;  // lanes j8 >= NP take amax 0, which stays on the fast path
+#pragma unroll
+        for (int p = 0; p < NP; ++p)
+          if (j8 == p) mm = m[p];
+        BlockDivider dm;
+        if constexpr (P2)
+          brow_mine = pow2_scale(bf16x2_absmax_to_f32(mm), dm);
+        else
+          block_scale_fast(bf16x2_absmax_to_f32(mm), srow_mine, dm, ok);
+        const int src = lane & ~7;
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          bool okp = true;
-          amax[p] = bf16x2_absmax_to_f32(m[p]);
-          if constexpr (P2)
-            brow[p] = pow2_scale(amax[p], div[p]);
-          else
-            block_scale_fast(amax[p], srow[p], div[p], okp);
-          ok = ok && okp;
+          div[p].s = __shfl_sync(0xffffffffu, dm.s, src + p);
+          div[p].r = __shfl_sync(0xffffffffu, dm.r, src + p);
+          div[p].fast = true;
         }
       } else {
 #pragma unroll
@@ -349,7 +355,11 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
       } else {
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
-          if constexpr (kRows && !P2) block_scale(amax[p], srow[p], div[p]);
+          if constexpr (kRows && !P2) {  // the general scale and divider, on every lane
+            float sp;
+            block_scale(bf16x2_absmax_to_f32(m[p]), sp, div[p]);
+            if (j8 == p) srow_mine = sp;
+          }
           q0[p] = codes8(v0[p], div[p]);
           q1[p] = codes8(v1[p], div[p]);
         }
@@ -361,11 +371,11 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
           uint8_t *qrow = args.q + row * args.ldq + c0 + 8 * j8;
           *reinterpret_cast<uint2 *>(qrow) = q0[p];
           *reinterpret_cast<uint2 *>(qrow + 64) = q1[p];
-          if (kRows && j8 == 0) {
+          if (kRows && j8 == p) {
             if constexpr (P2)
-              args.sb[(c0 / kTile) * args.R + row] = static_cast<uint8_t>(brow[p]);
+              args.sb[(c0 / kTile) * args.R + row] = static_cast<uint8_t>(brow_mine);
             else
-              args.s[(c0 / kTile) * args.R + row] = srow[p];
+              args.s[(c0 / kTile) * args.R + row] = srow_mine;
           }
         }
       }
