@@ -8,10 +8,13 @@
 // column of B for every 32 elements of K and accumulates the whole K in FP32 in TMEM, so
 // no promotion runs on the CUDA cores: the tile's accumulator is read once, at its end.
 //
-// One CTA per SM, 128 x 256 tiles, 512 threads in four warpgroups:
-//   warp 0       TMA producer: A and B K blocks (128 wide) into a 3-stage ring
-//   warp 1       MMA issuer and TMEM owner: per K block 4 block-scaled MMAs (K = 32 each)
-//                into the tile's accumulator
+// One CTA per SM with 128 x 256 tiles when the output has at most 128 rows, otherwise a
+// cluster of two CTAs (cta_group::2 MMAs) with 256 x 256 tiles, each CTA staging its own 128
+// rows of A and half of B and holding its 128 rows of the accumulator. 512 threads in four
+// warpgroups:
+//   warp 0       TMA producer: A and B K blocks (128 wide) into a 3-stage ring (pair: 4)
+//   warp 1       MMA issuer (pair: the leader CTA's, for both CTAs) and TMEM owner: per K
+//                block 4 block-scaled MMAs (K = 32 each) into the tile's accumulator
 //   warps 4..11  epilogue: at a tile's end each reads its 32 rows x 128 columns of the
 //                accumulator, hands it back to the MMA issuer, then rounds to BF16 into
 //                swizzled shared memory and stores with the TMA unit
@@ -19,11 +22,13 @@
 //                its scale factors into a ring slot of TMEM columns, loading them from
 //                global memory as many K blocks ahead as the ring has slots. The MMA reads
 //                the factor of A row m from lane m, column m / 32, and that of B column n
-//                from lane 32q + n % 32, column n / 32, in the lane quadrant q of the row it
-//                computes; each quadrant therefore holds its 32 rows' A factors (written
+//                from lane 32q + n % 32, column n / 32, in the lane quadrant q of the row
+//                it computes; each quadrant therefore holds its 32 rows' A factors (written
 //                into all 4 A columns of its lanes) and all 256 columns' B factors (8
-//                columns). A 32-bit cell holds the factors of four K sub-blocks; one scale
-//                covers all 128 of K here, so its byte is written four times.
+//                columns). A CTA pair's MMA reads each CTA's factors from that CTA's own
+//                TMEM in the same layout (its own rows of A, all of B). A 32-bit cell holds
+//                the factors of four K sub-blocks; one scale covers all 128 of K here, so
+//                its byte is written four times.
 // TMEM: accumulator columns 0..255; ring slot i: A factors at 256 + 16i (4 columns), B
 // factors at 260 + 16i (8 columns). Every mbarrier wait is bounded; a wait that gives up
 // sets the abort flag and the device status word, and the CTA drains and exits.
@@ -43,24 +48,32 @@
 namespace puro {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128;
-constexpr int STAGES = 3;
+constexpr int BM = 128, BN = 256, BK = 128;  // BM: rows per CTA (a CTA pair: 256-row tiles)
 constexpr int SF_SLOTS = 4;
 constexpr int THREADS = 512;
 constexpr int EPI_FIRST = 4, EPI_WARPS = 8, SFW_FIRST = 12;
-constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK;
+constexpr int A_BYTES = BM * BK;
 constexpr int STG_BOX_BYTES = 32 * 128;               // 32 rows x 64 BF16, 128B-swizzled
 constexpr int STG_WARP_BYTES = 2 * STG_BOX_BYTES;     // 128 columns per epilogue warp
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
-// full/empty per stage, sf_full/sf_empty per slot, tfull, tempty, drain
-constexpr int N_BARS = 2 * STAGES + 2 * SF_SLOTS + 3;
-constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+// PAIR: a cluster of two CTAs computes a 256 x 256 tile with cta_group::2 MMAs; each CTA
+// stages its own 128 rows of A and half of B, and holds its 128 rows of the accumulator.
+template <bool PAIR>
+struct MxCfg {
+  static constexpr int STAGES = PAIR ? 4 : 3;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B this CTA stages
+  static constexpr int B_BYTES = B_ROWS * BK;
+  static constexpr int TILE_ROWS = PAIR ? 2 * BM : BM;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
+  // full/empty per stage, sf_full/sf_empty per slot, tfull, tempty, drain
+  static constexpr int N_BARS = 2 * STAGES + 2 * SF_SLOTS + 3;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
 constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_SLOT_COLS = 16;
 constexpr int LAUNCH_REGS = 128;   // 65536 / 512
 constexpr int REGS_SMALL = 56;     // warpgroups 0 and 3
@@ -80,6 +93,16 @@ __device__ __forceinline__ void mma_mx(uint32_t d, uint64_t ad, uint64_t bd, uin
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %6, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mx_pair(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
       "l"(ad), "l"(bd), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
       : "memory");
 }
@@ -122,15 +145,17 @@ __device__ __forceinline__ uint32_t bf16x2_bits_mx(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-template <int LAYOUT>
+template <int LAYOUT, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_mx(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmC, const MxArgs args) {
+  using C = MxCfg<PAIR>;
+  constexpr int STAGES = C::STAGES, B_BYTES = C::B_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + OFF_BAR;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto sf_full_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + i); };
@@ -138,9 +163,23 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tfull_bar = bar0 + 8u * (2 * STAGES + 2 * SF_SLOTS);
   const uint32_t tempty_bar = tfull_bar + 8u;
   const uint32_t drain_bar = tfull_bar + 16u;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-  volatile int *abort = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // PAIR: rank 0 of the cluster is the leader: it issues the MMAs for both CTAs and holds the
+  // barriers both CTAs report to (the operands' arrival, the scale factors, the accumulator's
+  // hand-back). Tiles are walked per cluster; rank r owns rows 128 r .. of a 256-row tile.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  auto row_base = [&](int mt) { return mt * C::TILE_ROWS + static_cast<int>(rank) * BM; };
+  auto arrive_leader = [&](uint32_t bar) {
+    if constexpr (PAIR)
+      mbar_arrive_cluster(map_to_rank(bar, 0));
+    else
+      mbar_arrive(bar);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -148,11 +187,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(empty_bar(s), 1);
     }
     for (int i = 0; i < SF_SLOTS; ++i) {
-      mbar_init(sf_full_bar(i), 4);   // the four scale-writer warps
-      mbar_init(sf_empty_bar(i), 1);  // the MMA commit
+      mbar_init(sf_full_bar(i), PAIR ? 8 : 4);  // the scale-writer warps (of both CTAs)
+      mbar_init(sf_empty_bar(i), 1);            // the MMA commit
     }
     mbar_init(tfull_bar, 1);
-    mbar_init(tempty_bar, EPI_WARPS);
+    mbar_init(tempty_bar, PAIR ? 2 * EPI_WARPS : EPI_WARPS);
     mbar_init(drain_bar, 1);
     *abort = 0;
     fence_barrier_init();
@@ -163,11 +202,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // both CTAs' barriers exist before either reports to the other
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
   const int tiles = args.num_m * args.num_n;
@@ -181,7 +228,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_parity = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
         int mt, nt;
         mx_tile_coords(tile, args, mt, nt);
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -189,9 +236,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
-          tma_load_2d(sbase + OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
-          tma_load_2d(sbase + OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
+          if constexpr (PAIR) {
+            // Both CTAs' loads count on the leader's barrier, armed by the leader with the
+            // pair's bytes; a peer load for a stage's next use starts only after the MMA that
+            // read the stage completed (its empty barrier), so never in the previous phase.
+            const uint32_t fb = map_to_rank(full_bar(s), 0);
+            if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (A_BYTES + B_BYTES));
+            tma_load_2d_pair(sbase + C::OFF_A + s * A_BYTES, &tmA, fb, kb * BK, row_base(mt));
+            tma_load_2d_pair(sbase + C::OFF_B + s * B_BYTES, &tmB, fb, kb * BK,
+                             nt * BN + static_cast<int>(rank) * C::B_ROWS);
+          } else {
+            mbar_arrive_expect_tx(full_bar(s), A_BYTES + B_BYTES);
+            tma_load_2d(sbase + C::OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
+            tma_load_2d(sbase + C::OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
+          }
           issued |= 1u << s;
           issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
           if (++s == STAGES) s = 0, ph ^= 1u;
@@ -200,15 +258,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) {
         *abort = 1;
         atomicOr(args.status, 1);
-        for (int i = 0; i < STAGES; ++i)
-          if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
+        // Every issued load lands before the CTA can exit (a peer's loads count on the
+        // leader's barriers; the peer stays alive through the final cluster barrier).
+        if (leader)
+          for (int i = 0; i < STAGES; ++i)
+            if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
       }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1 && lane == 0 && leader) {
       // ---------------------------------------------------------------- MMA issuer
       int s = 0, slot = 0;
       uint32_t ph = 0, sph = 0, it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++it) {
+      for (int tile = first_tile; ok && tile < tiles; tile += tile_step, ++it) {
         if (!mbar_wait(tempty_bar, (it & 1u) ^ 1u, tmo, abort)) {  // the accumulator is free
           ok = false;
           break;
@@ -220,23 +281,43 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = sbase + OFF_A + s * A_BYTES, b_addr = sbase + OFF_B + s * B_BYTES;
+          const uint32_t a_addr = sbase + C::OFF_A + s * A_BYTES, b_addr = sbase + C::OFF_B + s * B_BYTES;
           const uint32_t sfa = tmem + SF_COL + SF_SLOT_COLS * slot, sfb = sfa + 4;
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k)
-            mma_mx(tmem + ACC_COL, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k),
-                   idesc_mx(BM, BN, k, k), sfa, sfb, (kb > 0 || k > 0) ? 1u : 0u);
-          mma_commit(empty_bar(s));
-          mma_commit(sf_empty_bar(slot));
+          for (int k = 0; k < BK / 32; ++k) {
+            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+            if constexpr (PAIR)
+              mma_mx_pair(tmem + ACC_COL, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k),
+                          idesc_mx(2 * BM, BN, k, k), sfa, sfb, acc);
+            else
+              mma_mx(tmem + ACC_COL, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k),
+                     idesc_mx(BM, BN, k, k), sfa, sfb, acc);
+          }
+          if constexpr (PAIR) {
+            mma_commit_pair_mc(empty_bar(s), 0x3);        // both CTAs' stage s is free again
+            mma_commit_pair_mc(sf_empty_bar(slot), 0x3);  // and their scale-factor slot
+          } else {
+            mma_commit(empty_bar(s));
+            mma_commit(sf_empty_bar(slot));
+          }
           if (++s == STAGES) s = 0, ph ^= 1u;
           if (++slot == SF_SLOTS) slot = 0, sph ^= 1u;
         }
-        if (ok) mma_commit(tfull_bar);
+        if (ok) {
+          if constexpr (PAIR)
+            mma_commit_pair_mc(tfull_bar, 0x3);  // both CTAs' accumulators are complete
+          else
+            mma_commit(tfull_bar);
+        }
       }
       if (!ok) {
         *abort = 1;
         atomicOr(args.status, 1);
-        mma_commit(drain_bar);
+        // arrives once every MMA issued here has finished
+        if constexpr (PAIR)
+          mma_commit_pair(drain_bar);
+        else
+          mma_commit(drain_bar);
         mbar_wait(drain_bar, 0, tmo, nullptr);
       }
     }
@@ -244,17 +325,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_SMALL));
     // ------------------------------------------------------------------ scale writers
     // Loads run SF_SLOTS K blocks ahead of the stores, in a register ring of raw loaded
-    // values (3 registers per K block), so their latency is hidden behind the MMAs.
+    // values (3 registers per K block), so their latency is hidden behind the MMAs. A CTA
+    // pair reads each CTA's factors from that CTA's own TMEM: its 128 rows of A and all 256
+    // columns of B.
     const int quad = warp & 3;
     const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
     const int nb_total = (args.N + 127) / 128;
-    // raw values of one K block: this lane's A byte (row 32 quad + lane of the tile) and
-    // two words for B (wgrad: bytes 8 lane .. 8 lane + 7 of the tile's 256 columns;
+    // raw values of one K block: this lane's A byte (row 32 quad + lane of this CTA's rows)
+    // and two words for B (wgrad: bytes 8 lane .. 8 lane + 7 of the tile's 256 columns;
     // fprop/dgrad: the bytes of the tile's two 128-column blocks)
     auto fetch = [&](int tile, int kb, uint32_t &ra, uint32_t &rb0, uint32_t &rb1) {
       int mt, nt;
       mx_tile_coords(tile, args, mt, nt);
-      const int m = mt * BM + 32 * quad + lane;
+      const int m = row_base(mt) + 32 * quad + lane;
       ra = m < args.M ? __ldg(args.As + static_cast<int64_t>(kb) * args.M + m) : 127u;
       if (LAYOUT == PURO_WGRAD) {
         const int n0 = nt * BN + 8 * lane;  // N % 8 == 0: the 8 bytes exist or none do
@@ -301,10 +384,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_st_x8(tmem + lane_field + SF_COL + SF_SLOT_COLS * slot + 4, cb);
     };
     auto advance = [&](int &tile, int &kb) {
-      if (++kb == kblocks) kb = 0, tile += gridDim.x;
+      if (++kb == kblocks) kb = 0, tile += tile_step;
     };
     uint32_t ra[SF_SLOTS], rb0[SF_SLOTS], rb1[SF_SLOTS];
-    int ft = blockIdx.x, fk = 0;  // the next K block to fetch
+    int ft = first_tile, fk = 0;  // the next K block to fetch
 #pragma unroll
     for (int d = 0; d < SF_SLOTS; ++d) {
       if (ft < tiles) fetch(ft, fk, ra[d], rb0[d], rb1[d]);
@@ -312,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     uint32_t sph = 0;
     bool ok = true;
-    int ct = blockIdx.x, ck = 0;  // the next K block to store
+    int ct = first_tile, ck = 0;  // the next K block to store
     while (ok && ct < tiles) {
 #pragma unroll
       for (int d = 0; d < SF_SLOTS; ++d) {  // ring slot d holds the K block fetched into set d
@@ -329,7 +412,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_wait_st();
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(sf_full_bar(d));
+          if (lane == 0) arrive_leader(sf_full_bar(d));
           advance(ct, ck);
         }
       }
@@ -344,10 +427,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3, half = (warp - EPI_FIRST) >> 2;
     const uint32_t taddr = tmem + ACC_COL + (static_cast<uint32_t>(quad * 32) << 16) + half * 128;
-    const uint32_t stg = sbase + OFF_STG + (warp - EPI_FIRST) * STG_WARP_BYTES;
+    const uint32_t stg = sbase + C::OFF_STG + (warp - EPI_FIRST) * STG_WARP_BYTES;
     uint32_t it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+    for (int tile = first_tile; tile < tiles; tile += tile_step, ++it) {
       int mt, nt;
       mx_tile_coords(tile, args, mt, nt);
       if (!mbar_wait(tfull_bar, it & 1u, tmo, abort)) {
@@ -362,7 +445,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_wait_ld_dep(r1);
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar);  // the MMA may start the next tile
+      if (lane == 0) arrive_leader(tempty_bar);  // the MMA may start the next tile
       if (lane == 0) bulk_wait_group_read<0>();  // the previous tile's stores left the staging
       __syncwarp();
 #pragma unroll
@@ -380,7 +463,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        const int row0 = mt * BM + quad * 32, col0 = nt * BN + half * 128;
+        const int row0 = row_base(mt) + quad * 32, col0 = nt * BN + half * 128;
         if (row0 < args.M) {
           if (col0 < args.N) tma_store_2d(&tmC, stg, col0, row0);
           if (col0 + 64 < args.N) tma_store_2d(&tmC, stg + STG_BOX_BYTES, col0 + 64, row0);
@@ -396,10 +479,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // neither CTA leaves while the other may still use its shared memory or TMEM
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, 512);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
   }
 }
 
@@ -445,9 +534,10 @@ unsigned long long mx_timeout_ns() {
   return ns;
 }
 
-template <int LAYOUT>
+template <int LAYOUT, bool PAIR>
 int launch_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs, uint16_t *C,
               int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  using CF = MxCfg<PAIR>;
   int sms = 0;
   if (!sm_count(sms)) return PURO_ERR_CUDA;
   static PerDevice<int *> status_addr;
@@ -458,7 +548,7 @@ int launch_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uin
     return PURO_ERR_CUDA;
   CUtensorMap ta, tb, tc;
   if (!mx_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, BM, BK) ||
-      !mx_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, BN, BK) ||
+      !mx_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, CF::B_ROWS, BK) ||
       !mx_map(&tc, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64))
     return PURO_ERR_CUDA;
   args.As = As;
@@ -467,15 +557,29 @@ int launch_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uin
   args.N = static_cast<int>(N);
   args.K = static_cast<int>(K);
   args.kblocks = static_cast<int>(K / BK);
-  args.num_m = static_cast<int>((M + BM - 1) / BM);
+  args.num_m = static_cast<int>((M + CF::TILE_ROWS - 1) / CF::TILE_ROWS);
   args.num_n = static_cast<int>((N + BN - 1) / BN);
   args.m_fastest = M <= N ? 1 : 0;
   args.timeout_ns = mx_timeout_ns();
   const int64_t tiles = static_cast<int64_t>(args.num_m) * args.num_n;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  auto kern = k_gemm_mx<LAYOUT>;
+  auto kern = k_gemm_mx<LAYOUT, PAIR>;
+  auto cluster_cfg = [&](int grid, cudaLaunchAttribute *attr) {
+    cudaLaunchConfig_t cfg{};
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = CF::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+  };
   // Once per device: the register split assumes exactly LAUNCH_REGS per thread at launch
-  // (otherwise the epilogue's setmaxnreg.inc could wait forever); shared memory opt-in.
+  // (otherwise the epilogue's setmaxnreg.inc could wait forever); shared memory opt-in; for
+  // a CTA pair, the clusters that can be resident at once (the persistent grid's size).
   static PerDevice<int> prepared;
   int prep = PURO_ERR_CUDA;
   if (!prepared.get(prep, [&](int, int &v) {
@@ -487,15 +591,37 @@ int launch_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uin
           v = PURO_ERR_LAUNCH;
           return true;
         }
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES) != cudaSuccess)
           return false;
         v = PURO_OK;
+        if constexpr (PAIR) {
+          cudaLaunchAttribute attr[1];
+          cudaLaunchConfig_t cfg = cluster_cfg(2 * (sms / 2), attr);
+          int clusters = 0;
+          if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+            std::fprintf(stderr, "puro_fp8: no CTA pair of the MX GEMM kernel fits on this device\n");
+            v = PURO_ERR_LAUNCH;
+            return true;
+          }
+          v = clusters;  // > 0
+        }
         return true;
       }))
     return PURO_ERR_CUDA;
-  if (prep != PURO_OK) return prep;
-  kern<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, tc, args);
-  const cudaError_t e = cudaGetLastError();
+  if (prep < 0) return prep;
+  cudaError_t e;
+  int grid;
+  if constexpr (PAIR) {
+    grid = static_cast<int>(2 * (tiles < prep ? tiles : prep));
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = cluster_cfg(grid, attr);
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  } else {
+    grid = static_cast<int>(tiles < sms ? tiles : sms);
+    kern<<<grid, THREADS, CF::SMEM_BYTES, stream>>>(ta, tb, tc, args);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) {
     std::fprintf(stderr, "puro_fp8: MX GEMM launch (grid %d): %s\n", grid, cudaGetErrorString(e));
     return PURO_ERR_LAUNCH;
@@ -503,14 +629,33 @@ int launch_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uin
   return PURO_OK;
 }
 
+// CTA pairs unless the output has at most 128 rows; PURO_MX_PAIR=0 or 1 forces one of them
+// (read once per process).
+bool mx_use_pair(int64_t M) {
+  static const int mode = [] {
+    const char *e = std::getenv("PURO_MX_PAIR");
+    return e == nullptr ? -1 : std::atoi(e);
+  }();
+  if (mode == 0) return false;
+  if (mode == 1) return true;
+  return M > BM;
+}
+
+template <int LAYOUT>
+int launch_mx_layout(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs, uint16_t *C,
+                     int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+  return mx_use_pair(M) ? launch_mx<LAYOUT, true>(Aq, As, Bq, Bs, C, M, N, K, stream)
+                        : launch_mx<LAYOUT, false>(Aq, As, Bq, Bs, C, M, N, K, stream);
+}
+
 }  // namespace
 
 int launch_gemm_mx(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, const uint8_t *Bs, uint16_t *C,
                    int64_t M, int64_t N, int64_t K, int layout, cudaStream_t stream) {
   switch (layout) {
-    case PURO_FPROP: return launch_mx<PURO_FPROP>(Aq, As, Bq, Bs, C, M, N, K, stream);
-    case PURO_DGRAD: return launch_mx<PURO_DGRAD>(Aq, As, Bq, Bs, C, M, N, K, stream);
-    case PURO_WGRAD: return launch_mx<PURO_WGRAD>(Aq, As, Bq, Bs, C, M, N, K, stream);
+    case PURO_FPROP: return launch_mx_layout<PURO_FPROP>(Aq, As, Bq, Bs, C, M, N, K, stream);
+    case PURO_DGRAD: return launch_mx_layout<PURO_DGRAD>(Aq, As, Bq, Bs, C, M, N, K, stream);
+    case PURO_WGRAD: return launch_mx_layout<PURO_WGRAD>(Aq, As, Bq, Bs, C, M, N, K, stream);
     default: return PURO_ERR_LAYOUT;
   }
 }
