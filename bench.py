@@ -65,6 +65,8 @@ def _args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="issue the timed steps' launches one by one instead of replaying a CUDA graph")
     p.add_argument("--no-lm-head", action="store_true",
                    help="leave the LM head out of the step (small profiling cases with --layers)")
     p.add_argument("--no-group", action="store_true",
@@ -74,7 +76,8 @@ def _args():
                         "4 the LM head, 5 the full 28-layer step (default), 'all' for 1-4 then 5, or "
                         "'fused' for the fused epilogue quantisation against GEMM + separate quantiser, "
                         "'grouped' for one block's four wgrads in one launch against four, "
-                        "'scales' for the full step with FP32 scales against power-of-two scales")
+                        "'scales' for the full step with FP32 scales against power-of-two scales, "
+                        "'vendor' for the library FP8 and BF16 GEMMs on the step's shapes (roofline context)")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions of configs 1-4")
     return p.parse_args()
 
@@ -504,13 +507,29 @@ def run_ours(args):
 
     step = Step(pf, wl, args.tokens, args.layers, device, seed=4 + 1000 * rank, group_wgrad=not args.no_group,
                 lm_head=not args.no_lm_head)
-    stream = torch.cuda.current_stream()
+    # A stream of its own (a CUDA graph cannot be captured on the legacy default stream);
+    # every launch, event and collective of this rank runs on it or waits for it.
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.set_stream(stream)
 
     clocks = Clocks(torch.cuda.current_device())
     clocks.start()  # sampling starts before the warm-up; only the timed region is kept
     for _ in range(args.warmup):
         step.run(stream=stream, overlap=True)
     pf.puro_fp8_sync_status()
+
+    # By default the step's 483 launches (both streams, with their events) are captured once
+    # into a CUDA graph, and each timed step is one replay of it: the same kernels on the
+    # same buffers, without the host issuing each launch.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step.run(stream=stream, overlap=True)
+        graph.replay()  # one more warm-up step, through the graph
+        torch.cuda.synchronize()
+        pf.puro_fp8_sync_status()
+    run_step = graph.replay if graph is not None else (lambda: step.run(stream=stream, overlap=True))
     _barrier_sync(world)
 
     # The timed region: whole steps, CUDA events only at its two ends (an event between
@@ -518,7 +537,7 @@ def run_ours(args):
     t_begin = time.time()
     start = _record(torch)
     for _ in range(args.steps):
-        step.run(stream=stream, overlap=True)
+        run_step()
     end = _record(torch)
     end.synchronize()
     _barrier_sync(world)
@@ -593,6 +612,7 @@ def run_ours(args):
                                         f"{quant_gbs / 8000:.4f}",
                            "launches_measured": n_quant, "avg_launch_ms": round(t_quant / max(n_quant, 1), 4)},
         "gpu_launches": step.launches_per_step * args.steps,
+        "launch": "one CUDA graph replay per step" if graph is not None else "eager launches",
         "host_enqueue_ms_per_step": round(statistics.median(host_ms), 3),
         "clocks": clk,
     }
@@ -605,6 +625,8 @@ def run_ours(args):
         line["cpu_baseline"] = cpu_baseline(args.tokens)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del run_step, graph  # released before the process group (it holds no collective)
+    torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -682,10 +704,10 @@ def main():
     if args.impl == "reference":
         run_reference(args)
         return
-    if args.config in ("fused", "grouped", "scales"):
+    if args.config in ("fused", "grouped", "scales", "vendor"):
         import bench_configs
         {"fused": bench_configs.run_fused_comparison, "grouped": bench_configs.run_grouped_comparison,
-         "scales": bench_configs.run_scales_comparison}[args.config](args)
+         "scales": bench_configs.run_scales_comparison, "vendor": bench_configs.run_vendor_reference}[args.config](args)
         return
     if args.config in ("1", "2", "3", "4", "all"):
         from bench_configs import run_config

@@ -427,3 +427,43 @@ def run_scales_comparison(args):
                       "steps": steps, "warmup": args.warmup, **out,
                       "pow2_speedup": round(out["fp32"]["ms_per_step"] / out["pow2"]["ms_per_step"], 3)}),
           flush=True)
+
+
+def run_vendor_reference(args):
+    """Context for the GEMM roofline, not part of the path: the library FP8 GEMM
+    (torch._scaled_mm, per-tensor scales, BF16 output, no blockwise scaling) and the BF16 GEMM
+    on the step's GEMM shapes, back to back with CUDA events. What a plain FP8 GEMM reaches on
+    this GPU bounds what a blockwise one can."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    T = args.tokens
+    shapes = [("fprop QKV", T, 4096, 2048), ("fprop gate/up", T, 12288, 2048), ("fprop down", T, 2048, 6144),
+              ("dgrad gate/up", T, 2048, 12288), ("wgrad gate/up", 12288, 2048, T), ("square", 8192, 8192, 8192)]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    rows = []
+    for label, M, N, K in shapes:
+        a = torch.randn(M, K, device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn(N, K, device=dev, generator=g).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev)
+        fns = {"fp8": lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)}
+        a16, b16 = a.to(torch.bfloat16), b.to(torch.bfloat16)
+        fns["bf16"] = lambda: a16 @ b16.t()
+        row = {"op": label, "M": M, "N": N, "K": K}
+        for kind, fn in fns.items():
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            t = []
+            for _ in range(max(3, args.reps // 2)):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(10):
+                    fn()
+                e1.record()
+                e1.synchronize()
+                t.append(e0.elapsed_time(e1) / 10)
+            row[f"{kind}_tflops"] = round(2.0 * M * N * K / statistics.median(t) / 1e9, 1)
+        rows.append(row)
+        del a, b, a16, b16
+    print(json.dumps({"reference": "library GEMMs (torch._scaled_mm FP8 with per-tensor scales; BF16 matmul)",
+                      "note": "context for the roofline only; not on the path", "ops": rows}), flush=True)
