@@ -77,7 +77,8 @@ def _args():
                         "'fused' for the fused epilogue quantisation against GEMM + separate quantiser, "
                         "'grouped' for one block's four wgrads in one launch against four, "
                         "'scales' for the full step with FP32 scales against power-of-two scales, "
-                        "'vendor' for the library FP8 and BF16 GEMMs on the step's shapes (roofline context)")
+                        "'vendor' for the library FP8 and BF16 GEMMs on the step's shapes (roofline context), "
+                        "'kernels' for single GEMMs with FP32 against power-of-two scales")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions of configs 1-4")
     return p.parse_args()
 
@@ -704,10 +705,11 @@ def main():
     if args.impl == "reference":
         run_reference(args)
         return
-    if args.config in ("fused", "grouped", "scales", "vendor"):
+    if args.config in ("fused", "grouped", "scales", "vendor", "kernels"):
         import bench_configs
         {"fused": bench_configs.run_fused_comparison, "grouped": bench_configs.run_grouped_comparison,
-         "scales": bench_configs.run_scales_comparison, "vendor": bench_configs.run_vendor_reference}[args.config](args)
+         "scales": bench_configs.run_scales_comparison, "vendor": bench_configs.run_vendor_reference,
+         "kernels": bench_configs.run_kernel_comparison}[args.config](args)
         return
     if args.config in ("1", "2", "3", "4", "all"):
         from bench_configs import run_config

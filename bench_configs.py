@@ -467,3 +467,54 @@ def run_vendor_reference(args):
         del a, b, a16, b16
     print(json.dumps({"reference": "library GEMMs (torch._scaled_mm FP8 with per-tensor scales; BF16 matmul)",
                       "note": "context for the roofline only; not on the path", "ops": rows}), flush=True)
+
+
+def run_kernel_comparison(args):
+    """Single GEMMs at the step's shapes (8192 tokens), each with FP32 scales
+    (puro_fp8_gemm_blockwise) and with power-of-two scales (puro_fp8_mx_gemm) on the same
+    random codes (the scale bytes 2^(byte - 127) as the FP32 scales), back to back with CUDA
+    events, interleaved, median over repetitions."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    T = args.tokens
+    shapes = [("fprop", T, 4096, 2048), ("fprop", T, 12288, 2048), ("fprop", T, 2048, 6144),
+              ("dgrad", T, 2048, 12288), ("dgrad", T, 2048, 4096), ("wgrad", 12288, 2048, T),
+              ("wgrad", 4096, 2048, T), ("wgrad", 2048, 6144, T), ("fprop", T, 151936, 2048)]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    rows = []
+    for lay, M, N, K in shapes:
+        aq = torch.randint(0, 256, (M, K), dtype=torch.uint8, device=dev, generator=g)
+        bq = torch.randint(0, 256, (N, K), dtype=torch.uint8, device=dev, generator=g)
+        for t in (aq, bq):
+            t[(t & 0x7F) == 0x7F] = 0x38  # no NaN codes
+        nb = (N + 127) // 128
+        bs_shape = {"fprop": (nb, K // 128), "dgrad": (K // 128, nb), "wgrad": (K // 128, N)}[lay]
+        ab = torch.randint(112, 124, (K // 128, M), dtype=torch.uint8, device=dev, generator=g)
+        bb = torch.randint(112, 124, bs_shape, dtype=torch.uint8, device=dev, generator=g)
+        a_s, b_s = torch.exp2(ab.float() - 127), torch.exp2(bb.float() - 127)
+        c32 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        cmx = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fns = {"fp32_scales": lambda: pf.puro_fp8_gemm_blockwise(aq, a_s, bq, b_s, c32, lay),
+               "pow2_scales": lambda: pf.puro_fp8_mx_gemm(aq, ab, bq, bb, cmx, lay)}
+        for fn in fns.values():
+            fn()
+            fn()
+        torch.cuda.synchronize()
+        t = {k: [] for k in fns}
+        for _ in range(max(3, args.reps // 2)):
+            for k, fn in fns.items():
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(5):
+                    fn()
+                e1.record()
+                e1.synchronize()
+                t[k].append(e0.elapsed_time(e1) / 5)
+        pf.puro_fp8_sync_status()
+        flops = 2.0 * M * N * K
+        rows.append({"op": lay, "M": M, "N": N, "K": K,
+                     **{f"{k}_tflops": round(flops / statistics.median(v) / 1e9, 1) for k, v in t.items()}})
+        del aq, bq, ab, bb, a_s, b_s, c32, cmx
+    print(json.dumps({"comparison": "single GEMMs at the step's shapes: FP32 scales vs power-of-two scales",
+                      "inputs": "random E4M3 codes, scale bytes 112..123 (the same scales as FP32 for the other kernel)",
+                      "ops": rows}), flush=True)
