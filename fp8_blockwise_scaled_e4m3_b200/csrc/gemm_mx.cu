@@ -130,6 +130,17 @@ struct MxArgs {
 
 __device__ int g_mx_status;  // non-zero: a bounded wait gave up since the last read
 
+#ifdef PURO_TEST_HOOKS
+// Test builds only, never libpuro_fp8.so: while set, the scale writers withhold their
+// arrival for the first K block, so the MMA issuer's bounded wait for the scale factors runs
+// out. The failure-detection test uses this to check that a give-up inside this kernel
+// reaches the status word and that the kernel drains and exits with the context intact.
+__device__ int g_test_mx_skip_sf;
+#define PURO_MX_SKIP_SF(seq) (g_test_mx_skip_sf != 0 && (seq) == 0)
+#else
+#define PURO_MX_SKIP_SF(seq) false
+#endif
+
 __device__ __forceinline__ void mx_tile_coords(int tile, const MxArgs &a, int &mt, int &nt) {
   if (a.m_fastest) {
     mt = tile % a.num_m;
@@ -393,7 +404,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ft < tiles) fetch(ft, fk, ra[d], rb0[d], rb1[d]);
       advance(ft, fk);
     }
-    uint32_t sph = 0;
+    uint32_t sph = 0, seq = 0;  // seq: K blocks stored so far
     bool ok = true;
     int ct = first_tile, ck = 0;  // the next K block to store
     while (ok && ct < tiles) {
@@ -412,8 +423,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_wait_st();
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) arrive_leader(sf_full_bar(d));
+          if (lane == 0 && !PURO_MX_SKIP_SF(seq)) arrive_leader(sf_full_bar(d));
           advance(ct, ck);
+          ++seq;
         }
       }
       sph ^= 1u;
@@ -674,3 +686,9 @@ int read_and_clear_mx_status(cudaStream_t stream, int *status_out) {
 }
 
 }  // namespace puro
+
+#ifdef PURO_TEST_HOOKS
+extern "C" __attribute__((visibility("default"))) int puro_test_set_mx_skip_sf(int on) {
+  return cudaMemcpyToSymbol(puro::g_test_mx_skip_sf, &on, sizeof(int)) == cudaSuccess ? 0 : -1;
+}
+#endif

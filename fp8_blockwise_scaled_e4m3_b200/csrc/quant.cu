@@ -103,6 +103,17 @@ __device__ __forceinline__ int problem_of(const QParams<G> &prm, int p, int tile
 
 __device__ int g_quant_status;  // non-zero: a bounded wait gave up since the last read
 
+#ifdef PURO_TEST_HOOKS
+// Test builds only, never libpuro_fp8.so: while set, each CTA skips the load of its first
+// tile, so the bounded wait for that tile runs out. The failure-detection test uses this to
+// check that a give-up inside the quantiser reaches the status word and that the kernel
+// drains and exits with the context intact.
+__device__ int g_test_quant_skip_load;
+#define PURO_QUANT_SKIP_LOAD(i) (g_test_quant_skip_load != 0 && (i) == 0)
+#else
+#define PURO_QUANT_SKIP_LOAD(i) false
+#endif
+
 
 // Packed magnitude maximum of the 16 BF16 values in v0 and v1 (per half, see
 // bf16x2_absmax).
@@ -224,7 +235,7 @@ __global__ void __launch_bounds__(Threads<MODE>::value, kCtasPerSm)
   int p_issue = 0;  // thread 0: the problem of the last tile it issued
   auto issue = [&](int i) {
     const int tile = blockIdx.x + i * gridDim.x;
-    if (tile >= tiles) return;
+    if (tile >= tiles || PURO_QUANT_SKIP_LOAD(i)) return;
     const int p = problem_of(prm, p_issue, tile);
     if (p != p_issue) {
       prefetch_tensormap(&prm.tmX[p]);
@@ -659,3 +670,9 @@ int read_and_clear_quant_status(cudaStream_t stream, int *status_out) {
 }
 
 }  // namespace puro
+
+#ifdef PURO_TEST_HOOKS
+extern "C" __attribute__((visibility("default"))) int puro_test_set_quant_skip_load(int on) {
+  return cudaMemcpyToSymbol(puro::g_test_quant_skip_load, &on, sizeof(int)) == cudaSuccess ? 0 : -1;
+}
+#endif
