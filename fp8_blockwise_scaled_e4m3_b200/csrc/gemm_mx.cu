@@ -19,7 +19,9 @@
 //                accumulator, hands it back to the MMA issuer, then rounds to BF16 into
 //                swizzled shared memory and stores with the TMA unit
 //   warps 12..15 scale writers, one per TMEM lane quadrant: for every K block they write
-//                its scale factors into a ring slot of TMEM columns, loading them from
+//                its scale factors into a ring slot of TMEM columns (one slot per pipeline
+//                stage, reported on the stage's full barrier beside the TMA bytes, so the
+//                MMA issuer waits once and commits once per K block), loading them from
 //                global memory as many K blocks ahead as the ring has slots. The MMA reads
 //                the factor of A row m from lane m, column m / 32, and that of B column n
 //                from lane 32q + n % 32, column n / 32, in the lane quadrant q of the row
@@ -49,7 +51,6 @@ namespace puro {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 128;  // BM: rows per CTA (a CTA pair: 256-row tiles)
-constexpr int SF_SLOTS = 4;
 constexpr int THREADS = 512;
 constexpr int EPI_FIRST = 4, EPI_WARPS = 8, SFW_FIRST = 12;
 constexpr int A_BYTES = BM * BK;
@@ -60,6 +61,10 @@ constexpr int STG_WARP_BYTES = 2 * STG_BOX_BYTES;     // 128 columns per epilogu
 template <bool PAIR>
 struct MxCfg {
   static constexpr int STAGES = PAIR ? 4 : 3;
+  // One scale-factor ring slot per stage: a K block's factors are written into the slot of
+  // its operands' stage and counted on the same full barrier, and the MMA's one commit frees
+  // both, so the MMA issuer waits on one barrier and commits one per K block.
+  static constexpr int SF_SLOTS = STAGES;
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B this CTA stages
   static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int TILE_ROWS = PAIR ? 2 * BM : BM;
@@ -67,14 +72,15 @@ struct MxCfg {
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
-  // full/empty per stage, sf_full/sf_empty per slot, tfull, tempty, drain
-  static constexpr int N_BARS = 2 * STAGES + 2 * SF_SLOTS + 3;
+  // full/empty per stage, tfull, tempty, drain
+  static constexpr int N_BARS = 2 * STAGES + 3;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_SLOT_COLS = 16;
+static_assert(SF_COL + MxCfg<true>::SF_SLOTS * SF_SLOT_COLS <= 512, "TMEM columns");
 constexpr int LAUNCH_REGS = 128;   // 65536 / 512
 constexpr int REGS_SMALL = 56;     // warpgroups 0 and 3
 constexpr int REGS_EPI = 200;      // warpgroups 1 and 2
@@ -169,9 +175,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t bar0 = sbase + C::OFF_BAR;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
-  auto sf_full_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + i); };
-  auto sf_empty_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + SF_SLOTS + i); };
-  const uint32_t tfull_bar = bar0 + 8u * (2 * STAGES + 2 * SF_SLOTS);
+  constexpr int SF_SLOTS = C::SF_SLOTS;
+  const uint32_t tfull_bar = bar0 + 8u * (2 * STAGES);
   const uint32_t tempty_bar = tfull_bar + 8u;
   const uint32_t drain_bar = tfull_bar + 16u;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
@@ -194,12 +199,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
-    }
-    for (int i = 0; i < SF_SLOTS; ++i) {
-      mbar_init(sf_full_bar(i), PAIR ? 8 : 4);  // the scale-writer warps (of both CTAs)
-      mbar_init(sf_empty_bar(i), 1);            // the MMA commit
+      // the producer's arrival (with the stage's TMA bytes) and the scale-writer warps' (of
+      // both CTAs of a pair)
+      mbar_init(full_bar(s), 1 + (PAIR ? 8 : 4));
+      mbar_init(empty_bar(s), 1);  // the MMA commit
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, PAIR ? 2 * EPI_WARPS : EPI_WARPS);
@@ -277,8 +280,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     } else if (warp == 1 && lane == 0 && leader) {
       // ---------------------------------------------------------------- MMA issuer
-      int s = 0, slot = 0;
-      uint32_t ph = 0, sph = 0, it = 0;
+      int s = 0;
+      uint32_t ph = 0, it = 0;
       bool ok = true;
       for (int tile = first_tile; ok && tile < tiles; tile += tile_step, ++it) {
         if (!mbar_wait(tempty_bar, (it & 1u) ^ 1u, tmo, abort)) {  // the accumulator is free
@@ -287,13 +290,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_after_sync();
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(full_bar(s), ph, tmo, abort) || !mbar_wait(sf_full_bar(slot), sph, tmo, abort)) {
+          if (!mbar_wait(full_bar(s), ph, tmo, abort)) {  // operands and scale factors
             ok = false;
             break;
           }
           tc_fence_after_sync();
           const uint32_t a_addr = sbase + C::OFF_A + s * A_BYTES, b_addr = sbase + C::OFF_B + s * B_BYTES;
-          const uint32_t sfa = tmem + SF_COL + SF_SLOT_COLS * slot, sfb = sfa + 4;
+          const uint32_t sfa = tmem + SF_COL + SF_SLOT_COLS * s, sfb = sfa + 4;
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k) {
             const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
@@ -304,15 +307,11 @@ __global__ void __launch_bounds__(THREADS, 1)
               mma_mx(tmem + ACC_COL, sdesc_k_sw128(a_addr + 32 * k), sdesc_k_sw128(b_addr + 32 * k),
                      idesc_mx(BM, BN, k, k), sfa, sfb, acc);
           }
-          if constexpr (PAIR) {
-            mma_commit_pair_mc(empty_bar(s), 0x3);        // both CTAs' stage s is free again
-            mma_commit_pair_mc(sf_empty_bar(slot), 0x3);  // and their scale-factor slot
-          } else {
+          if constexpr (PAIR)
+            mma_commit_pair_mc(empty_bar(s), 0x3);  // both CTAs' stage s and its factors are free
+          else
             mma_commit(empty_bar(s));
-            mma_commit(sf_empty_bar(slot));
-          }
           if (++s == STAGES) s = 0, ph ^= 1u;
-          if (++slot == SF_SLOTS) slot = 0, sph ^= 1u;
         }
         if (ok) {
           if constexpr (PAIR)
@@ -412,7 +411,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int d = 0; d < SF_SLOTS; ++d) {  // ring slot d holds the K block fetched into set d
         if (ct < tiles) {
           // warp-uniform outcome: the stores and shuffles below need the whole warp
-          if (!__all_sync(0xffffffffu, mbar_wait(sf_empty_bar(d), sph ^ 1u, tmo, abort))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(d), sph ^ 1u, tmo, abort))) {
             ok = false;
             break;
           }
@@ -423,7 +422,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_wait_st();
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0 && !PURO_MX_SKIP_SF(seq)) arrive_leader(sf_full_bar(d));
+          if (lane == 0 && !PURO_MX_SKIP_SF(seq)) arrive_leader(full_bar(d));
           advance(ct, ck);
           ++seq;
         }
