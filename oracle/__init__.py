@@ -37,6 +37,10 @@ Modules
 ``mx``          the power-of-two (UE8M0) scale mode of the same groups (scale rounded up
                 to a power of two, stored as an exponent byte), pinned by its exponent
                 rule in exact rationals, a hand-worked group and nearest-value checks.
+``nvfp4``       the NVFP4 mode (E2M1 codes, a UE4M3 factor per 16 elements along the
+                reduction dimension, an FP32 tensor scale amax / 2688), pinned by the E2M1
+                table, a brute-force encoder, a hand-worked row of groups, invariants of the
+                two-level scale and an exact rational contraction.
 ``gemm``        the FP64 reference contraction for the fprop / dgrad / wgrad operand
                 layouts, pinned by exact rational brute force and an exact-integer case.
 ``accounting``  parameter and FLOP accounting (C = 6ND), pinned by the numbers the
@@ -45,4 +49,4 @@ Modules
 No function here is "parity unpinned".
 """
 
-from . import e4m3, quant, gemm, accounting  # noqa: F401
+from . import e4m3, quant, gemm, accounting, nvfp4  # noqa: F401
