@@ -168,6 +168,46 @@ int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_t *Bq, co
   return puro::launch_gemm_mx(Aq, As, Bq, Bs, C, M, N, K, layout, stream);
 }
 
+int puro_nvfp4_quantize_1x16(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq, int64_t ldq,
+                             uint8_t *F, float *amax, puro_stream_t stream) {
+  if (X == nullptr || Xq == nullptr || F == nullptr || amax == nullptr) return PURO_ERR_NULL;
+  if (R < 1 || C < 16 || C % 16 != 0 || ldx < C || ldq < C / 2) return PURO_ERR_SHAPE;
+  if (R > (1ll << 31) - 1 || C > (1ll << 31) - 1) return PURO_ERR_SHAPE;
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(F, 16) || !aligned(amax, 4) || ldx % 8 != 0 ||
+      ldq % 8 != 0)
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_nvfp4_quant_rows(X, R, C, ldx, Xq, ldq, F, amax, stream);
+}
+
+int puro_nvfp4_quantize_1x16_transposed(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *XqT,
+                                        int64_t ldq, uint8_t *FT, float *amax, puro_stream_t stream) {
+  if (X == nullptr || XqT == nullptr || FT == nullptr || amax == nullptr) return PURO_ERR_NULL;
+  if (R < 64 || R % 64 != 0 || C < 8 || C % 8 != 0 || ldx < C || ldq < R / 2) return PURO_ERR_SHAPE;
+  if (R > (1ll << 31) - 1 || C > (1ll << 31) - 1) return PURO_ERR_SHAPE;
+  if (!aligned(X, 16) || !aligned(XqT, 16) || !aligned(FT, 16) || !aligned(amax, 4) || ldx % 8 != 0 ||
+      ldq % 16 != 0)
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_nvfp4_quant_cols(X, R, C, ldx, XqT, ldq, FT, amax, stream);
+}
+
+int puro_nvfp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *a_amax, const uint8_t *Bq,
+                    const uint8_t *Bs, const float *b_amax, uint16_t *C, int64_t M, int64_t N, int64_t K,
+                    puro_stream_t stream) {
+  if (Aq == nullptr || As == nullptr || a_amax == nullptr || Bq == nullptr || Bs == nullptr ||
+      b_amax == nullptr || C == nullptr)
+    return PURO_ERR_NULL;
+  if (M < 1 || N < 8 || N % 8 != 0 || K < 128 || K % 128 != 0) return PURO_ERR_SHAPE;
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31) - 256) return PURO_ERR_SHAPE;
+  if (!tiles_fit(M, 128, N, 256)) return PURO_ERR_SHAPE;
+  if (!aligned(Aq, 16) || !aligned(Bq, 16) || !aligned(As, 16) || !aligned(Bs, 16) || !aligned(C, 16) ||
+      !aligned(a_amax, 4) || !aligned(b_amax, 4))
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_gemm_nvfp4(Aq, As, a_amax, Bq, Bs, b_amax, C, M, N, K, stream);
+}
+
 int puro_fp8_gemm_blockwise_grouped(const puro_gemm_problem *problems, int count, int layout,
                                     puro_stream_t stream) {
   if (problems == nullptr) return PURO_ERR_NULL;
@@ -218,11 +258,12 @@ int puro_fp8_sync_status(puro_stream_t stream) {
   // The status words are per device and collect timeouts from kernels on every stream:
   // join the whole device first so that none is missed.
   if (cudaDeviceSynchronize() != cudaSuccess) return PURO_ERR_CUDA;
-  int gemm = 0, quant = 0, mx = 0;
+  int gemm = 0, quant = 0, mx = 0, nv = 0;
   if (int e = puro::read_and_clear_device_status(stream, &gemm)) return e;
   if (int e = puro::read_and_clear_quant_status(stream, &quant)) return e;
   if (int e = puro::read_and_clear_mx_status(stream, &mx)) return e;
-  return (gemm | quant | mx) != 0 ? PURO_ERR_TIMEOUT : PURO_OK;
+  if (int e = puro::read_and_clear_nv_status(stream, &nv)) return e;
+  return (gemm | quant | mx | nv) != 0 ? PURO_ERR_TIMEOUT : PURO_OK;
 }
 
 const char *puro_strerror(int status) {

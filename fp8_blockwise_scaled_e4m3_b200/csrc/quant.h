@@ -24,6 +24,18 @@ int launch_quant_weight(const uint16_t *W, int64_t R, int64_t C, int64_t ldw, ui
 using WeightProblem = puro_weight_problem;
 int launch_quant_weight_grouped(const WeightProblem *problems, int count, cudaStream_t stream);
 
+// NVFP4 (E2M1 codes, a UE4M3 factor per 16 elements along the reduction dimension, an FP32
+// tensor amax): the row-wise and transposed 1x16 quantisers (each also writes the tensor's
+// amax) and the GEMM C = A . B^T of two operands quantised along K.
+int launch_nvfp4_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq, int64_t ldq,
+                            uint8_t *F, float *amax, cudaStream_t stream);
+int launch_nvfp4_quant_cols(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *XqT, int64_t ldq,
+                            uint8_t *FT, float *amax, cudaStream_t stream);
+int launch_gemm_nvfp4(const uint8_t *Aq, const uint8_t *As, const float *a_amax, const uint8_t *Bq,
+                      const uint8_t *Bs, const float *b_amax, uint16_t *C, int64_t M, int64_t N, int64_t K,
+                      cudaStream_t stream);
+int read_and_clear_nv_status(cudaStream_t stream, int *status_out);
+
 // Reads and clears the quantisers' device status word (after a stream sync).
 int read_and_clear_quant_status(cudaStream_t stream, int *status_out);
 

@@ -63,6 +63,9 @@ def _load():
         "puro_fp8_mx_gemm": [_p, _p, _p, _p, _p, _i64, _i64, _i64, ctypes.c_int, _p],
         "puro_fp8_quantize_1x128_transposed_pow2": [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p],
         "puro_fp8_quantize_128x128_pow2": [_p, _i64, _i64, _i64, _p, _p, _p, _p],
+        "puro_nvfp4_quantize_1x16": [_p, _i64, _i64, _i64, _p, _i64, _p, _p, _p],
+        "puro_nvfp4_quantize_1x16_transposed": [_p, _i64, _i64, _i64, _p, _i64, _p, _p, _p],
+        "puro_nvfp4_gemm": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p],
         "puro_fp8_sync_status": [_p],
     }
     for name, args in sig.items():
@@ -298,6 +301,81 @@ def mx_gemm(Aq, As, Bq, Bs, layout, stream=None):
     """C [M, N] bf16 from the block-scaled GEMM (allocating helper)."""
     C = torch.empty((Aq.shape[0], Bq.shape[0]), dtype=torch.bfloat16, device=Aq.device)
     puro_fp8_mx_gemm(Aq, As, Bq, Bs, C, layout, stream)
+    return C
+
+
+def puro_nvfp4_quantize_1x16(X, Xq, F, amax, stream=None):
+    """NVFP4 1x16 quantisation along the columns of X [R, C] bf16 (see the C declaration):
+    Xq uint8 [R, C/2] packed codes (row stride may exceed C/2), F uint8 [R, C/16] dense,
+    amax float32 [1] (the tensor's max |x|, written by the call)."""
+    _need(X, torch.bfloat16, "X"); _need(Xq, torch.uint8, "Xq"); _need(F, torch.uint8, "F")
+    _need(amax, torch.float32, "amax")
+    R, C = X.shape
+    if tuple(Xq.shape) != (R, C // 2) or tuple(F.shape) != (R, C // 16) or amax.numel() != 1:
+        raise ValueError("Xq must be [R, C/2], F [R, C/16] and amax one float")
+    _dense(F, "F")
+    with torch.cuda.device(X.device):
+        st = _stream(stream)
+        _check(_lib.puro_nvfp4_quantize_1x16(_ptr(X), R, C, X.stride(0), _ptr(Xq), Xq.stride(0), _ptr(F),
+                                             _ptr(amax), st), "puro_nvfp4_quantize_1x16", st)
+
+
+def puro_nvfp4_quantize_1x16_transposed(X, XqT, FT, amax, stream=None):
+    """NVFP4 1x16 quantisation along the rows (tokens) of X [R, C] bf16, written transposed:
+    XqT uint8 [C, R/2] packed codes, FT uint8 [C, R/16] dense, amax float32 [1]."""
+    _need(X, torch.bfloat16, "X"); _need(XqT, torch.uint8, "XqT"); _need(FT, torch.uint8, "FT")
+    _need(amax, torch.float32, "amax")
+    R, C = X.shape
+    if tuple(XqT.shape) != (C, R // 2) or tuple(FT.shape) != (C, R // 16) or amax.numel() != 1:
+        raise ValueError("XqT must be [C, R/2], FT [C, R/16] and amax one float")
+    _dense(FT, "FT")
+    with torch.cuda.device(X.device):
+        st = _stream(stream)
+        _check(_lib.puro_nvfp4_quantize_1x16_transposed(_ptr(X), R, C, X.stride(0), _ptr(XqT), XqT.stride(0),
+                                                        _ptr(FT), _ptr(amax), st),
+               "puro_nvfp4_quantize_1x16_transposed", st)
+
+
+def puro_nvfp4_gemm(Aq, As, a_amax, Bq, Bs, b_amax, C, stream=None):
+    """NVFP4 GEMM C [M, N] bf16 = A . B^T of two operands quantised along K (see the C
+    declaration): Aq [M, K/2], As [M, K/16], Bq [N, K/2], Bs [N, K/16] uint8, dense; the amax
+    arguments float32 [1] on the device."""
+    for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs")):
+        _need(t, torch.uint8, n)
+        _dense(t, n)
+    _need(C, torch.bfloat16, "C"); _dense(C, "C")
+    _need(a_amax, torch.float32, "a_amax"); _need(b_amax, torch.float32, "b_amax")
+    M, K = Aq.shape[0], 2 * Aq.shape[1]
+    N = Bq.shape[0]
+    if (tuple(As.shape) != (M, K // 16) or tuple(Bq.shape) != (N, K // 2) or tuple(Bs.shape) != (N, K // 16)
+            or tuple(C.shape) != (M, N)):
+        raise ValueError("operand shapes do not match: Aq [M, K/2], As [M, K/16], Bq [N, K/2], Bs [N, K/16], C [M, N]")
+    with torch.cuda.device(Aq.device):
+        st = _stream(stream)
+        _check(_lib.puro_nvfp4_gemm(_ptr(Aq), _ptr(As), _ptr(a_amax), _ptr(Bq), _ptr(Bs), _ptr(b_amax), _ptr(C),
+                                    M, N, K, st), "puro_nvfp4_gemm", st)
+
+
+def nvfp4_quantize(X, transposed=False, stream=None):
+    """(packed codes, factors, amax) of X along its columns, or along its rows written
+    transposed (allocating helper)."""
+    R, C = X.shape
+    amax = torch.empty(1, dtype=torch.float32, device=X.device)
+    if transposed:
+        q = torch.empty((C, R // 2), dtype=torch.uint8, device=X.device)
+        f = torch.empty((C, R // 16), dtype=torch.uint8, device=X.device)
+        puro_nvfp4_quantize_1x16_transposed(X, q, f, amax, stream)
+    else:
+        q = torch.empty((R, C // 2), dtype=torch.uint8, device=X.device)
+        f = torch.empty((R, C // 16), dtype=torch.uint8, device=X.device)
+        puro_nvfp4_quantize_1x16(X, q, f, amax, stream)
+    return q, f, amax
+
+
+def nvfp4_gemm(Aq, As, a_amax, Bq, Bs, b_amax, stream=None):
+    """C [M, N] bf16 from the NVFP4 GEMM (allocating helper)."""
+    C = torch.empty((Aq.shape[0], Bq.shape[0]), dtype=torch.bfloat16, device=Aq.device)
+    puro_nvfp4_gemm(Aq, As, a_amax, Bq, Bs, b_amax, C, stream)
     return C
 
 

@@ -193,6 +193,62 @@ PURO_API int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_
                               uint16_t *C, int64_t M, int64_t N, int64_t K, int layout, puro_stream_t stream);
 
 /*
+ * NVFP4 mode: E2M1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one UE4M3 factor per 16
+ * consecutive elements along the reduction dimension, and one FP32 tensor scale. Source: the
+ * pages name FP4 only as a capability of the hardware they chose (the jj-blog page, the
+ * paragraph after its Table 2); the format is NVIDIA's published NVFP4, with the method's
+ * choices carried over (scales from the tensor being quantised, groups along the reduction
+ * dimension, correctly rounded FP32 arithmetic):
+ *     s_t = amax_t / 2688                       (2688 = 6 * 448)
+ *     e   = E4M3_RNE_sat((amax_g / 6) / s_t)     the group's factor, a UE4M3 byte
+ *     S   = dec(e) * s_t
+ *     q   = E2M1_RNE_sat(x / S)                  (S == 0: a signed zero)
+ * every step correctly rounded in FP32. Two codes per byte, element 2i in the low nibble.
+ * Inputs must be finite. Each quantiser runs two kernels on `stream`: the tensor's absolute
+ * maximum (written to *amax, which the call first sets to zero), then the codes, which read
+ * *amax on the device. Nothing else is written and nothing is allocated.
+ *
+ * puro_nvfp4_quantize_1x16: groups along the columns of X.
+ *   X    [R, C] BF16, row stride ldx (>= C, % 8 == 0)   input
+ *   Xq   [R, C/2] bytes, row stride ldq (>= C/2, % 8)   output: packed codes
+ *   F    [R, C/16] bytes, dense                          output: F[r, j] factor of X[r, 16j..16j+15]
+ *   amax one float                                       output: max |X|
+ *   Requires R >= 1, C >= 16, C % 16 == 0; X, Xq, F 16-byte aligned, amax 4-byte aligned.
+ * puro_nvfp4_quantize_1x16_transposed: groups of 16 consecutive rows (tokens), written
+ * transposed (the wgrad operands, and W along N_out for dgrad).
+ *   X    [R, C] BF16, row stride ldx (>= C, % 8 == 0)   input
+ *   XqT  [C, R/2] bytes, row stride ldq (>= R/2, % 16)  output: packed codes of X^T
+ *   FT   [C, R/16] bytes, dense                          output: FT[c, j] factor of X[16j..16j+15, c]
+ *   amax one float                                       output: max |X|
+ *   Requires R % 64 == 0 (R >= 64), C % 8 == 0; alignment as above.
+ * Status: PURO_ERR_NULL, PURO_ERR_SHAPE, PURO_ERR_ALIGN, PURO_ERR_DEVICE, PURO_ERR_CUDA or
+ * PURO_ERR_LAUNCH, checked on the host before any launch.
+ */
+PURO_API int puro_nvfp4_quantize_1x16(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                                      int64_t ldq, uint8_t *F, float *amax, puro_stream_t stream);
+PURO_API int puro_nvfp4_quantize_1x16_transposed(const uint16_t *X, int64_t R, int64_t C, int64_t ldx,
+                                                 uint8_t *XqT, int64_t ldq, uint8_t *FT, float *amax,
+                                                 puro_stream_t stream);
+
+/*
+ * NVFP4 GEMM on the tensor cores' block-scaled FP4 MMA, which applies the UE4M3 factors
+ * itself and accumulates all of K in FP32:
+ *     C[m, n] = s_tA * s_tB * sum_k dec(qA[m, k]) fA[m, k/16] dec(qB[n, k]) fB[n, k/16]
+ * with s_t = amax / 2688 of each operand's tensor, rounded to BF16 (nearest even) once.
+ * Both operands are quantised along K (the 1x16 quantisers above): fprop takes X and W
+ * row-wise, dgrad dY row-wise and W transposed, wgrad dY and X transposed.
+ *   Aq [M, K/2] packed codes, dense     As [M, K/16] factors, dense     a_amax: A's tensor amax
+ *   Bq [N, K/2] packed codes, dense     Bs [N, K/16] factors, dense     b_amax: B's tensor amax
+ *   C  [M, N] BF16, dense               output
+ * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, As, Bq, Bs, C 16-byte
+ * aligned, the amax pointers 4-byte aligned (device memory). Status codes as for
+ * puro_fp8_gemm_blockwise.
+ */
+PURO_API int puro_nvfp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *a_amax, const uint8_t *Bq,
+                             const uint8_t *Bs, const float *b_amax, uint16_t *C, int64_t M, int64_t N,
+                             int64_t K, puro_stream_t stream);
+
+/*
  * Blockwise-FP8 GEMM  C[m, n] = sum_kb sA(kb, m) * sB(kb, n) * sum_{k in kb} A[m, k] B[n, k]
  * with an FP32 tensor-core partial per 128-wide K block, FP32 promotion and BF16 output.
  * Source: "Lever 2: use blockwise FP8 from step zero" (the linear-layer GEMMs in FP8

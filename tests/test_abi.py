@@ -47,6 +47,7 @@ def test_header_declares_the_entry_points():
         "puro_fp8_gemm_blockwise_grouped", "puro_fp8_quantize_1x128_pow2",
         "puro_fp8_quantize_1x128_transposed_pow2", "puro_fp8_quantize_128x128_pow2", "puro_fp8_mx_gemm",
         "puro_fp8_quantize_128x128_grouped",
+        "puro_nvfp4_quantize_1x16", "puro_nvfp4_quantize_1x16_transposed", "puro_nvfp4_gemm",
         "puro_fp8_sync_status", "puro_strerror"])
 
 
@@ -281,3 +282,30 @@ def test_mx_gemm_rejects_bad_arguments(lib):
     assert f(*ops, 128, 256, 200, 2, None) == ESHAPE
     assert f(*ops[:4], A16 + 2, 128, 256, 256, 1, None) == EALIGN
     assert f(*ops[:3], A16 + 4, A16, 128, 256, 256, 2, None) == EALIGN   # wgrad Bs 8-byte aligned
+
+
+def test_nvfp4_entry_points_reject_bad_arguments(lib):
+    """NVFP4 quantisers and GEMM: NULL pointers, shapes and alignment are refused on the host,
+    before any device work."""
+    q = lib.puro_nvfp4_quantize_1x16
+    assert q(None, 4, 32, 32, A16, 16, A16, A16, None) == ENULL
+    assert q(A16, 4, 32, 32, A16, 16, A16, None, None) == ENULL              # amax
+    assert q(A16, 4, 24, 32, A16, 16, A16, A16, None) == ESHAPE              # C % 16
+    assert q(A16, 4, 32, 32, A16, 8, A16, A16, None) == ESHAPE               # ldq < C / 2
+    assert q(A16, 4, 32, 32, A16 + 8, 16, A16, A16, None) == EALIGN          # Xq 16-byte aligned
+    assert q(A16, 4, 32, 36, A16, 16, A16, A16, None) == EALIGN              # ldx % 8
+    assert q(A16, 4, 32, 32, A16, 16, A16, A16 + 2, None) == EALIGN          # amax 4-byte aligned
+    qt = lib.puro_nvfp4_quantize_1x16_transposed
+    assert qt(A16, 100, 64, 64, A16, 64, A16, A16, None) == ESHAPE           # R % 64
+    assert qt(A16, 128, 60, 64, A16, 64, A16, A16, None) == ESHAPE           # C % 8
+    assert qt(A16, 128, 64, 64, A16, 32, A16, A16, None) == ESHAPE           # ldq < R / 2
+    assert qt(A16, 128, 64, 64, A16, 72, A16, A16, None) == EALIGN           # ldq % 16
+    g = lib.puro_nvfp4_gemm
+    ops = [A16, A16, A16, A16, A16, A16, A16]
+    assert g(None, *ops[1:], 128, 256, 256, None) == ENULL
+    assert g(*ops[:2], None, *ops[3:], 128, 256, 256, None) == ENULL        # a_amax
+    assert g(*ops, 128, 250, 256, None) == ESHAPE                            # N % 8
+    assert g(*ops, 128, 256, 200, None) == ESHAPE                            # K % 128
+    assert g(*ops, 0, 256, 256, None) == ESHAPE
+    assert g(A16, A16 + 8, *ops[2:], 128, 256, 256, None) == EALIGN          # As 16-byte aligned
+    assert g(*ops[:6], A16 + 2, 128, 256, 256, None) == EALIGN               # C
