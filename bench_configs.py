@@ -518,3 +518,89 @@ def run_kernel_comparison(args):
     print(json.dumps({"comparison": "single GEMMs at the step's shapes: FP32 scales vs power-of-two scales",
                       "inputs": "random E4M3 codes, scale bytes 112..123 (the same scales as FP32 for the other kernel)",
                       "ops": rows}), flush=True)
+
+
+NVFP4_BYTES_PER_ELEMENT = 2 + 2 + 0.5 + 1 / 16  # amax read, quantise read, codes, factors
+
+
+def run_nvfp4(args):
+    """The NVFP4 mode on the step's shapes (8192 tokens), CUDA events, L2 flushed before every
+    timed call (512 MB written and read back), median over repetitions:
+    - the 1x16 quantisers (row-wise, and along the tokens written transposed) on the step's
+      activation, gradient and weight shapes, in GB/s of algorithmic bytes: the tensor-amax
+      pass reads X once, the quantising pass reads it again and writes the packed codes and
+      one factor byte per 16 elements (4.5625 bytes per element);
+    - the GEMMs of the kernel comparison (fprop, dgrad, wgrad and LM-head shapes), each on
+      operands the NVFP4 quantisers made from seeded random BF16 tensors, in TFLOP/s and as
+      a fraction of the dense FP4 tensor peak, taken as 4 x the BF16 peak (the nominal ratio
+      of the dense FP4 and BF16 rates)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    T = args.tokens
+    _, bf16_tf, _, peak_src = _peaks()
+    fp4_peak = 4.0 * bf16_tf
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    reps = max(3, args.reps // 2)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush_l2(flush)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        pf.puro_fp8_sync_status()
+        return statistics.median(ts)
+
+    def rand(shape, seed):
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        return torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+
+    quant = []
+    for name, r, c, transposed in (("X 1x16", T, 2048, False), ("X along tokens", T, 2048, True),
+                                   ("X 1x16", T, 6144, False), ("dY 1x16", T, 12288, False),
+                                   ("dY along tokens", T, 12288, True), ("W gate/up 1x16", 12288, 2048, False),
+                                   ("W gate/up along N_out", 12288, 2048, True)):
+        x = rand((r, c), 7 + len(quant))
+        amax = torch.empty(1, dtype=torch.float32, device=dev)
+        if transposed:
+            q = torch.empty((c, r // 2), dtype=torch.uint8, device=dev)
+            f = torch.empty(((r + 255) // 256, c, 16), dtype=torch.uint8, device=dev)
+            fn = lambda: pf.puro_nvfp4_quantize_1x16_transposed(x, q, f, amax)
+        else:
+            q = torch.empty((r, c // 2), dtype=torch.uint8, device=dev)
+            f = torch.empty(((c + 255) // 256, r, 16), dtype=torch.uint8, device=dev)
+            fn = lambda: pf.puro_nvfp4_quantize_1x16(x, q, f, amax)
+        ms = timed(fn)
+        gb = r * c * NVFP4_BYTES_PER_ELEMENT / 1e9
+        quant.append({"tensor": name, "R": r, "C": c, "us": round(ms * 1e3, 1), "GB_per_s": round(gb / (ms * 1e-3), 1)})
+        del x, q, f
+
+    shapes = [("fprop", T, 4096, 2048), ("fprop", T, 12288, 2048), ("fprop", T, 2048, 6144),
+              ("dgrad", T, 2048, 12288), ("dgrad", T, 2048, 4096), ("wgrad", 12288, 2048, T),
+              ("wgrad", 4096, 2048, T), ("wgrad", 2048, 6144, T), ("fprop", T, 151936, 2048)]
+    gemms = []
+    for i, (lay, M, N, K) in enumerate(shapes):
+        aq, af, aa = pf.nvfp4_quantize(rand((M, K), 100 + i))
+        b = rand((N, K), 200 + i)
+        bq, bf, ba = pf.nvfp4_quantize(b)
+        del b
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ms = timed(lambda: pf.puro_nvfp4_gemm(aq, af, aa, bq, bf, ba, c))
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        gemms.append({"op": lay, "M": M, "N": N, "K": K, "us": round(ms * 1e3, 1), "tflops": round(tf, 1),
+                      "frac_of_fp4_peak": round(tf / fp4_peak, 4)})
+        del aq, af, bq, bf, c
+        torch.cuda.empty_cache()
+    print(json.dumps({"comparison": "NVFP4 (E2M1, UE4M3 per 16, FP32 tensor scale): quantisers and GEMMs",
+                      "workload": f"the Qwen3-1.7B-shaped step's tensors at {T} tokens, seeded random BF16",
+                      "l2": "flushed before every timed call (512 MB written, then read back)",
+                      "fp4_peak_tflops": round(fp4_peak, 1),
+                      "fp4_peak_note": f"4 x {peak_src} BF16 burst ({bf16_tf}) (dense FP4 / BF16 nominal ratio)",
+                      "quant_bytes_per_element": NVFP4_BYTES_PER_ELEMENT, "quantisers": quant, "gemms": gemms}),
+          flush=True)

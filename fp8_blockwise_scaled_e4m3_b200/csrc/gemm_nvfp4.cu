@@ -12,13 +12,18 @@
 //
 // Structure as the block-scaled FP8 kernel (gemm_mx.cu): persistent, one CTA (M <= 128) or
 // one CTA pair (cta_group::2, 256-row tiles) per SM (pair), 512 threads:
-//   warp 0       TMA producer: A and B K blocks of 128 bytes (256 codes) per ring stage
+//   warp 0       TMA producer: A and B K blocks of 128 bytes (256 codes) per ring stage, and
+//                the stage's factors (this CTA's 128 A rows and the tile's 256 B rows, 16
+//                bytes each) into shared memory, counted on the stage's factor barrier
 //   warp 1       MMA issuer: per K block four MMAs of K = 64 (32 bytes), each with its own
 //                factor cells, one commit to the stage's empty barrier
 //   warps 4..11  epilogue: the tile's FP32 accumulator times s_tA * s_tB, BF16, TMA stores
-//   warps 12..15 scale writers, one per TMEM lane quadrant: for every K block they load the
-//                16 factor bytes of each row they serve and store them as TMEM cells in the
-//                layout the MMA reads (below), counted on the stage's full barrier
+//   warps 12..15 scale writers, one per TMEM lane quadrant: for every K block they read the
+//                16 factor bytes of each row they serve from the stage's shared memory (a
+//                warp's 32 rows are 512 contiguous bytes) and store them as TMEM cells in the
+//                layout the MMA reads (below), counted on the stage's full barrier. (Loading
+//                the factors from global memory in these warps, even coalesced, held the
+//                kernel near 1.5 PFLOP/s; without those loads it ran near 4.5.)
 // Factor layout in TMEM (probed on B200 with single MMAs): for each MMA, the factors of A row
 // m are read from lane m, column m / 32, and those of B row n from lane 32 q + n % 32, column
 // n / 32 of the lane quadrant q of the row being computed; byte j of a 32-bit cell is the
@@ -54,17 +59,23 @@ constexpr int A_BYTES = BM * BK;
 constexpr int STG_BOX_BYTES = 32 * 128;            // 32 rows x 64 BF16, 128B-swizzled
 constexpr int STG_WARP_BYTES = 2 * STG_BOX_BYTES;  // 128 columns per epilogue warp
 
+constexpr int SFA_BYTES = BM * 16;  // one K block's factors of 128 A rows
+constexpr int SFB_BYTES = BN * 16;  // ... and of 256 B rows
+
 template <bool PAIR>
 struct NvCfg {
-  static constexpr int STAGES = PAIR ? 4 : 3;
+  static constexpr int STAGES = PAIR ? 4 : 2;  // single CTAs (M <= 128) stage all 256 B rows
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B this CTA stages
   static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int TILE_ROWS = PAIR ? 2 * BM : BM;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_STG = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+  static constexpr int OFF_STG = OFF_SFB + STAGES * SFB_BYTES;
   static constexpr int OFF_BAR = OFF_STG + EPI_WARPS * STG_WARP_BYTES;
-  static constexpr int N_BARS = 2 * STAGES + 3;  // full/empty per stage, tfull, tempty, drain
+  // full/empty per stage, tfull, tempty, drain, a factor barrier per stage
+  static constexpr int N_BARS = 3 * STAGES + 3;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(OFF_STG % 1024 == 0, "swizzled staging must be 1024-byte aligned");
@@ -73,7 +84,7 @@ struct NvCfg {
 constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_SLOT_COLS = 48, SF_MMA_COLS = 12;
 static_assert(SF_COL + NvCfg<true>::STAGES * SF_SLOT_COLS <= 512, "TMEM columns");
 // Register split: warpgroup 0 (producer, issuer), warpgroups 1-2 (epilogue: 128 accumulator
-// registers), warpgroup 3 (scale writers: two K blocks of factor words in flight)
+// registers), warpgroup 3 (scale writers)
 constexpr int LAUNCH_REGS = 128;  // 65536 / 512
 constexpr int REGS_WG0 = 56, REGS_EPI = 168, REGS_SFW = 120;
 static_assert(128 * REGS_WG0 + 256 * REGS_EPI + 128 * REGS_SFW == THREADS * LAUNCH_REGS, "register split");
@@ -118,8 +129,8 @@ __device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 struct NvArgs {
-  const uint8_t *As;  // UE4M3 [M, K/16]
-  const uint8_t *Bs;  // UE4M3 [N, K/16]
+  const uint8_t *As;  // UE4M3 [K blocks][M][16]
+  const uint8_t *Bs;  // UE4M3 [K blocks][N][16]
   const float *a_amax, *b_amax;
   int M, N, K;
   int num_m, num_n, kblocks, m_fastest;
@@ -144,28 +155,11 @@ __device__ __forceinline__ uint32_t bf16x2_bits_nv(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-// The 16 factor bytes of one row for K block kb as four words (word k: MMA k's groups
-// 0..3), zero beyond the row's K / 16 factors or for rows outside the matrix. Rows of
-// factors are 8-byte aligned (K % 128 == 0), so two 8-byte loads.
-__device__ __forceinline__ void load_factors(const uint8_t *base, int rows, int row, int kfac, int kb,
-                                             uint32_t (&w)[4]) {
-  w[0] = w[1] = w[2] = w[3] = 0;
-  if (row >= rows) return;
-  const uint8_t *p = base + static_cast<int64_t>(row) * kfac + 16 * kb;
-  const uint2 lo = __ldg(reinterpret_cast<const uint2 *>(p));
-  w[0] = lo.x;
-  w[1] = lo.y;
-  if (16 * kb + 8 < kfac) {
-    const uint2 hi = __ldg(reinterpret_cast<const uint2 *>(p + 8));
-    w[2] = hi.x;
-    w[3] = hi.y;
-  }
-}
-
 template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_nvfp4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmC, const NvArgs args) {
+                 const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmSA,
+                 const __grid_constant__ CUtensorMap tmSB, const NvArgs args) {
   using C = NvCfg<PAIR>;
   constexpr int STAGES = C::STAGES, B_BYTES = C::B_BYTES;
   extern __shared__ uint8_t smem_raw[];
@@ -178,6 +172,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tfull_bar = bar0 + 8u * (2 * STAGES);
   const uint32_t tempty_bar = tfull_bar + 8u;
   const uint32_t drain_bar = tfull_bar + 16u;
+  auto sf_full_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + 3 + s); };  // this CTA's factor bytes
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
   volatile int *abort = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,6 +197,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // CTAs of a pair)
       mbar_init(full_bar(s), 1 + (PAIR ? 8 : 4));
       mbar_init(empty_bar(s), 1);  // the MMA commit
+      mbar_init(sf_full_bar(s), 1);  // this CTA's producer, with the factor bytes
     }
     mbar_init(tfull_bar, 1);
     mbar_init(tempty_bar, PAIR ? 2 * EPI_WARPS : EPI_WARPS);
@@ -213,6 +209,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmC);
+    prefetch_tensormap(&tmSA);
+    prefetch_tensormap(&tmSB);
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -263,6 +261,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_load_2d(sbase + C::OFF_A + s * A_BYTES, &tmA, full_bar(s), kb * BK, mt * BM);
             tma_load_2d(sbase + C::OFF_B + s * B_BYTES, &tmB, full_bar(s), kb * BK, nt * BN);
           }
+          // this CTA's factors of the K block: its A rows and the tile's B rows (rows past the
+          // matrix read as zeros), for its own scale writers
+          mbar_arrive_expect_tx(sf_full_bar(s), SFA_BYTES + SFB_BYTES);
+          tma_load_3d(sbase + C::OFF_SFA + s * SFA_BYTES, &tmSA, sf_full_bar(s), 0, row_base(mt), kb);
+          tma_load_3d(sbase + C::OFF_SFB + s * SFB_BYTES, &tmSB, sf_full_bar(s), 0, nt * BN, kb);
           issued |= 1u << s;
           issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
           if (++s == STAGES) s = 0, ph ^= 1u;
@@ -273,9 +276,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         atomicOr(args.status, 1);
         // Every issued load lands before the CTA can exit (a peer's loads count on the
         // leader's barriers; the peer stays alive through the final cluster barrier).
-        if (leader)
-          for (int i = 0; i < STAGES; ++i)
-            if ((issued >> i) & 1u) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
+        for (int i = 0; i < STAGES; ++i)
+          if ((issued >> i) & 1u) {
+            if (leader) mbar_wait(full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
+            mbar_wait(sf_full_bar(i), (issued_parity >> i) & 1u, tmo, nullptr);
+          }
       }
     } else if (warp == 1 && lane == 0 && leader) {
       // ---------------------------------------------------------------- MMA issuer
@@ -333,71 +338,56 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp >= SFW_FIRST) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_SFW));
     // ------------------------------------------------------------------ scale writers
-    // Two K blocks of factor words are in flight: the loads for K block i + 2 are issued when
-    // K block i is stored, so their latency hides behind the MMAs. A CTA pair reads each
-    // CTA's factors from that CTA's own TMEM: its 128 rows of A and all 256 rows of B.
+    // Each K block's factors wait in the stage's shared memory (the producer's TMA); a writer
+    // reads its rows' 16 bytes per K block and stores them as TMEM cells. The factor barrier
+    // of a stage's next use completes only after the producer saw the stage's empty barrier,
+    // i.e. after the MMA that read the previous cells, so the cells are free to overwrite.
+    // A CTA pair reads each CTA's factors from that CTA's own TMEM: its 128 rows of A and all
+    // 256 rows of B.
     const int quad = warp & 3;
     const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
     const int kfac = args.K / 16;
-    struct Words {
-      uint32_t a[4];     // this lane's A row (32 quad + lane of the CTA's rows)
-      uint32_t b[8][4];  // B rows 32 g + lane of the tile
-    };
-    auto fetch = [&](int tile, int kb, Words &w) {
-      int mt, nt;
-      nv_tile_coords(tile, args, mt, nt);
-      load_factors(args.As, args.M, row_base(mt) + 32 * quad + lane, kfac, kb, w.a);
-#pragma unroll
-      for (int g = 0; g < 8; ++g) load_factors(args.Bs, args.N, nt * BN + 32 * g + lane, kfac, kb, w.b[g]);
-    };
-    auto store = [&](int slot, const Words &w) {
-#pragma unroll
-      for (int k = 0; k < BK / 32; ++k) {
-        const uint32_t ca[4] = {w.a[k], w.a[k], w.a[k], w.a[k]};
-        uint32_t cb[8];
-#pragma unroll
-        for (int g = 0; g < 8; ++g) cb[g] = w.b[g][k];
-        const uint32_t col = SF_COL + SF_SLOT_COLS * slot + SF_MMA_COLS * k;
-        tmem_st_x4(tmem + lane_field + col, ca);
-        tmem_st_x8(tmem + lane_field + col + 4, cb);
-      }
-    };
-    auto advance = [&](int &tile, int &kb) {
-      if (++kb == kblocks) kb = 0, tile += tile_step;
-    };
-    Words w0, w1;
-    int ft = first_tile, fk = 0;  // the next K block to fetch
-    if (ft < tiles) fetch(ft, fk, w0);
-    advance(ft, fk);
-    if (ft < tiles) fetch(ft, fk, w1);
-    advance(ft, fk);
     int s = 0;
-    uint32_t sph = 0, seq = 0;  // seq: K blocks stored so far
+    uint32_t ph = 0, seq = 0;
     bool ok = true;
-    int ct = first_tile, ck = 0;  // the next K block to store
-    auto step = [&](Words &w) {
-      // warp-uniform outcome: the stores below need the whole warp
-      if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), sph ^ 1u, tmo, abort))) {
-        ok = false;
-        return;
+    for (int tile = first_tile; ok && tile < tiles; tile += tile_step) {
+      for (int kb = 0; kb < kblocks; ++kb, ++seq) {
+        // warp-uniform outcome: the stores below need the whole warp
+        if (!__all_sync(0xffffffffu, mbar_wait(sf_full_bar(s), ph, tmo, abort))) {
+          ok = false;
+          break;
+        }
+        const uint8_t *fa = smem + C::OFF_SFA + s * SFA_BYTES;
+        const uint8_t *fb = smem + C::OFF_SFB + s * SFB_BYTES;
+        const uint4 va = *reinterpret_cast<const uint4 *>(fa + 16 * (32 * quad + lane));
+        uint4 vb[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) vb[g] = *reinterpret_cast<const uint4 *>(fb + 16 * (32 * g + lane));
+        // a half K block (K % 256 == 128) has factors for its first 128 codes only
+        const bool full = 16 * kb + 8 < kfac;
+        auto word = [&](const uint4 &v, int k) -> uint32_t {
+          return k == 0 ? v.x : k == 1 ? v.y : !full ? 0u : k == 2 ? v.z : v.w;
+        };
+        tc_fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < BK / 32; ++k) {
+          const uint32_t a = word(va, k);
+          const uint32_t ca[4] = {a, a, a, a};
+          uint32_t cb[8];
+#pragma unroll
+          for (int g = 0; g < 8; ++g) cb[g] = word(vb[g], k);
+          const uint32_t col = SF_COL + SF_SLOT_COLS * s + SF_MMA_COLS * k;
+          tmem_st_x4(tmem + lane_field + col, ca);
+          tmem_st_x8(tmem + lane_field + col + 4, cb);
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) arrive_leader(full_bar(s));
+        if (++s == STAGES) s = 0, ph ^= 1u;
       }
-      tc_fence_after_sync();
-      store(s, w);
-      if (ft < tiles) fetch(ft, fk, w);
-      advance(ft, fk);
-      tmem_wait_st();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) arrive_leader(full_bar(s));
-      advance(ct, ck);
-      ++seq;
-      if (++s == STAGES) s = 0, sph ^= 1u;
-    };
-    while (ok && ct < tiles) {
-      step(w0);
-      if (!ok || ct >= tiles) break;
-      step(w1);
     }
+    (void)seq;
     if (!ok && lane == 0) {
       *abort = 1;
       atomicOr(args.status, 1);
@@ -509,6 +499,21 @@ bool nv_map(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int e
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Factors stored by K block, [kblocks][rows][16] bytes, as a 3-D tensor (16 bytes, rows,
+// K blocks); a box is 16 bytes x box_rows rows of one K block, rows past the matrix read as
+// zeros.
+bool nv_factor_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t kblocks, uint32_t box_rows) {
+  EncodeTiledFn fn = nv_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {16, rows, kblocks};
+  const cuuint64_t strides[2] = {16, rows * 16};
+  const cuuint32_t box[3] = {16, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 unsigned long long nv_timeout_ns() {
   static unsigned long long ns = [] {
     const char *e = std::getenv("PURO_WAIT_TIMEOUT_MS");
@@ -531,11 +536,12 @@ int launch_nv(const uint8_t *Aq, const uint8_t *As, const float *a_amax, const u
         return cudaGetSymbolAddress(reinterpret_cast<void **>(&v), g_nv_status) == cudaSuccess;
       }))
     return PURO_ERR_CUDA;
-  CUtensorMap ta, tb, tc;
+  CUtensorMap ta, tb, tc, tsa, tsb;
   // operands as bytes: [rows, K/2], two codes per byte
   if (!nv_map(&ta, Aq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, BM, BK) ||
       !nv_map(&tb, Bq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, CF::B_ROWS, BK) ||
-      !nv_map(&tc, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64))
+      !nv_map(&tc, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 32, 64) ||
+      !nv_factor_map(&tsa, As, M, (K + 255) / 256, BM) || !nv_factor_map(&tsb, Bs, N, (K + 255) / 256, BN))
     return PURO_ERR_CUDA;
   args.As = As;
   args.Bs = Bs;
@@ -603,11 +609,11 @@ int launch_nv(const uint8_t *Aq, const uint8_t *As, const float *a_amax, const u
     grid = static_cast<int>(2 * (tiles < prep ? tiles : prep));
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = cluster_cfg(grid, attr);
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args);
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tsa, tsb, args);
     if (e == cudaSuccess) e = cudaGetLastError();
   } else {
     grid = static_cast<int>(tiles < sms ? tiles : sms);
-    kern<<<grid, THREADS, CF::SMEM_BYTES, stream>>>(ta, tb, tc, args);
+    kern<<<grid, THREADS, CF::SMEM_BYTES, stream>>>(ta, tb, tc, tsa, tsb, args);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) {

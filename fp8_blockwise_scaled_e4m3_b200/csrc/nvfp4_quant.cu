@@ -9,7 +9,11 @@
 //   e   = E4M3_RNE_sat(RN(RN(amax_g / 6) / s_t))      the group's UE4M3 factor
 //   S   = RN(dec(e) * s_t)
 //   q   = E2M1_RNE_sat(RN(x / S)), or a signed zero when S == 0
-// Two codes per byte (element 2i in the low nibble). The tensor amax is an output of its own
+// Two codes per byte (element 2i in the low nibble). Factors are stored by 256-element K
+// block: F[b][r][j] (16 bytes per row and block) is the factor of X[r, 256 b + 16 j ..], so the
+// GEMM reads a K block's factors of consecutive rows as one contiguous run. Quotients are
+// correctly rounded through the group's reciprocal with Markstein's correction (as in the FP8
+// quantisers; IEEE division below divisors of 2^-90). The tensor amax is an output of its own
 // kernel, read by the quantising kernel from device memory, so the two launches need no host
 // round trip. Inputs must be finite.
 //
@@ -17,11 +21,11 @@
 //                    floats order like their bit patterns); the word starts at zero
 //   k_nv_quant_rows  one thread per 16-element group along the columns: 32-byte loads, one
 //                    8-byte store of codes and one factor byte, consecutive threads on
-//                    consecutive groups of a row
+//                    consecutive groups of a row (16 consecutive factor bytes per K block)
 //   k_nv_quant_cols  groups of 16 consecutive rows, written transposed: a thread takes two
 //                    adjacent columns over 64 rows (4-byte loads, a warp reads 128 contiguous
-//                    bytes of each row) and writes 32 bytes of codes and 4 factor bytes per
-//                    column
+//                    bytes of each row) and writes 32 bytes of codes and 4 factor bytes (one
+//                    4-byte store into its K block's 16) per column
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -69,10 +73,14 @@ __device__ __forceinline__ void group_scale(float amax_g, float s_t, uint32_t &e
   }
 }
 
-// codes of two elements with divisor S (S == 0: signed zeros)
-__device__ __forceinline__ uint32_t codes2(float x0, float x1, float S) {
-  if (S == 0.0f) return e2m1x2(x0 * 0.0f, x1 * 0.0f);
-  return e2m1x2(__fdiv_rn(x0, S), __fdiv_rn(x1, S));
+// the divider of a group with decoded scale S (S == 0: every quotient a signed zero)
+__device__ __forceinline__ BlockDivider group_divider(float S) {
+  return S > 0.0f ? make_divider(S) : zero_block_divider();
+}
+
+// codes of two elements
+__device__ __forceinline__ uint32_t codes2(float x0, float x1, const BlockDivider &dv) {
+  return e2m1x2(block_divide(dv, x0), block_divide(dv, x1));
 }
 
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
@@ -114,18 +122,20 @@ __global__ void __launch_bounds__(kThreads) k_nv_quant_rows(const uint16_t *__re
     uint32_t e;
     float S;
     group_scale(__uint_as_float(m << 16), s_t, e, S);
+    const BlockDivider dv = group_divider(S);
     uint32_t q[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = codes2(bf16_lo(w[i]), bf16_hi(w[i]), S);
+    for (int i = 0; i < 8; ++i) q[i] = codes2(bf16_lo(w[i]), bf16_hi(w[i]), dv);
     uint2 out;
     out.x = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
     out.y = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
     *reinterpret_cast<uint2 *>(Xq + r * ldq + 8 * j) = out;
-    F[r * groups_per_row + j] = static_cast<uint8_t>(e);
+    F[((j >> 4) * R + r) * 16 + (j & 15)] = static_cast<uint8_t>(e);
   }
 }
 
-// X [R, C] -> XqT [C, R/2] (row stride ldq bytes), FT [C, R/16]; R % 64 == 0, C % 2 == 0.
+// X [R, C] -> XqT [C, R/2] (row stride ldq bytes), FT [R/256 (rounded up)][C][16]; R % 64 == 0,
+// C % 2 == 0.
 __global__ void __launch_bounds__(kThreads) k_nv_quant_cols(const uint16_t *__restrict__ X, int64_t R, int64_t C,
                                                             int64_t ldx, uint8_t *__restrict__ XqT, int64_t ldq,
                                                             uint8_t *__restrict__ FT, const float *amax_t) {
@@ -156,11 +166,12 @@ __global__ void __launch_bounds__(kThreads) k_nv_quant_cols(const uint16_t *__re
         float S;
         group_scale(__uint_as_float(m << 16), s_t, e, S);
         fac |= e << (8 * g);
+        const BlockDivider dv = group_divider(S);
         uint32_t q[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t a = w[16 * g + 2 * i], b = w[16 * g + 2 * i + 1];
-          q[i] = col ? codes2(bf16_hi(a), bf16_hi(b), S) : codes2(bf16_lo(a), bf16_lo(b), S);
+          q[i] = col ? codes2(bf16_hi(a), bf16_hi(b), dv) : codes2(bf16_lo(a), bf16_lo(b), dv);
         }
         out[2 * g] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
         out[2 * g + 1] = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
@@ -168,7 +179,8 @@ __global__ void __launch_bounds__(kThreads) k_nv_quant_cols(const uint16_t *__re
       uint8_t *dst = XqT + (c0 + col) * ldq + r0 / 2;
       *reinterpret_cast<uint4 *>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
       *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(out[4], out[5], out[6], out[7]);
-      *reinterpret_cast<uint32_t *>(FT + (c0 + col) * (R / 16) + r0 / 16) = fac;
+      // groups 4 slab .. 4 slab + 3 of column c0 + col: K block slab / 4, bytes 4 (slab % 4) ..
+      *reinterpret_cast<uint32_t *>(FT + ((slab >> 2) * C + (c0 + col)) * 16 + 4 * (slab & 3)) = fac;
     }
   }
 }

@@ -153,6 +153,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// 3-D tiled bulk tensor load global -> shared, completion counted in bytes on `bar` (a
+// barrier of this CTA). c0 is the innermost coordinate.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int32_t c0,
+                                            int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
 // The same load issued by either CTA of a 2-CTA pair: the data lands in this CTA's shared
 // memory, the completed bytes are counted on `bar_cluster`, which may be the peer CTA's
 // barrier (a shared::cluster address). No multicast: one destination CTA.

@@ -306,13 +306,13 @@ def mx_gemm(Aq, As, Bq, Bs, layout, stream=None):
 
 def puro_nvfp4_quantize_1x16(X, Xq, F, amax, stream=None):
     """NVFP4 1x16 quantisation along the columns of X [R, C] bf16 (see the C declaration):
-    Xq uint8 [R, C/2] packed codes (row stride may exceed C/2), F uint8 [R, C/16] dense,
-    amax float32 [1] (the tensor's max |x|, written by the call)."""
+    Xq uint8 [R, C/2] packed codes (row stride may exceed C/2), F uint8 [ceil(C/256), R, 16]
+    (factors by 256-element K block), amax float32 [1] (the tensor's max |x|, written by the call)."""
     _need(X, torch.bfloat16, "X"); _need(Xq, torch.uint8, "Xq"); _need(F, torch.uint8, "F")
     _need(amax, torch.float32, "amax")
     R, C = X.shape
-    if tuple(Xq.shape) != (R, C // 2) or tuple(F.shape) != (R, C // 16) or amax.numel() != 1:
-        raise ValueError("Xq must be [R, C/2], F [R, C/16] and amax one float")
+    if tuple(Xq.shape) != (R, C // 2) or tuple(F.shape) != ((C + 255) // 256, R, 16) or amax.numel() != 1:
+        raise ValueError("Xq must be [R, C/2], F [ceil(C/256), R, 16] and amax one float")
     _dense(F, "F")
     with torch.cuda.device(X.device):
         st = _stream(stream)
@@ -322,12 +322,12 @@ def puro_nvfp4_quantize_1x16(X, Xq, F, amax, stream=None):
 
 def puro_nvfp4_quantize_1x16_transposed(X, XqT, FT, amax, stream=None):
     """NVFP4 1x16 quantisation along the rows (tokens) of X [R, C] bf16, written transposed:
-    XqT uint8 [C, R/2] packed codes, FT uint8 [C, R/16] dense, amax float32 [1]."""
+    XqT uint8 [C, R/2] packed codes, FT uint8 [ceil(R/256), C, 16], amax float32 [1]."""
     _need(X, torch.bfloat16, "X"); _need(XqT, torch.uint8, "XqT"); _need(FT, torch.uint8, "FT")
     _need(amax, torch.float32, "amax")
     R, C = X.shape
-    if tuple(XqT.shape) != (C, R // 2) or tuple(FT.shape) != (C, R // 16) or amax.numel() != 1:
-        raise ValueError("XqT must be [C, R/2], FT [C, R/16] and amax one float")
+    if tuple(XqT.shape) != (C, R // 2) or tuple(FT.shape) != ((R + 255) // 256, C, 16) or amax.numel() != 1:
+        raise ValueError("XqT must be [C, R/2], FT [ceil(R/256), C, 16] and amax one float")
     _dense(FT, "FT")
     with torch.cuda.device(X.device):
         st = _stream(stream)
@@ -338,8 +338,8 @@ def puro_nvfp4_quantize_1x16_transposed(X, XqT, FT, amax, stream=None):
 
 def puro_nvfp4_gemm(Aq, As, a_amax, Bq, Bs, b_amax, C, stream=None):
     """NVFP4 GEMM C [M, N] bf16 = A . B^T of two operands quantised along K (see the C
-    declaration): Aq [M, K/2], As [M, K/16], Bq [N, K/2], Bs [N, K/16] uint8, dense; the amax
-    arguments float32 [1] on the device."""
+    declaration): Aq [M, K/2], Bq [N, K/2] packed codes, As [ceil(K/256), M, 16], Bs
+    [ceil(K/256), N, 16] factors, uint8, dense; the amax arguments float32 [1] on the device."""
     for t, n in ((Aq, "Aq"), (As, "As"), (Bq, "Bq"), (Bs, "Bs")):
         _need(t, torch.uint8, n)
         _dense(t, n)
@@ -347,9 +347,11 @@ def puro_nvfp4_gemm(Aq, As, a_amax, Bq, Bs, b_amax, C, stream=None):
     _need(a_amax, torch.float32, "a_amax"); _need(b_amax, torch.float32, "b_amax")
     M, K = Aq.shape[0], 2 * Aq.shape[1]
     N = Bq.shape[0]
-    if (tuple(As.shape) != (M, K // 16) or tuple(Bq.shape) != (N, K // 2) or tuple(Bs.shape) != (N, K // 16)
+    kb = (K + 255) // 256
+    if (tuple(As.shape) != (kb, M, 16) or tuple(Bq.shape) != (N, K // 2) or tuple(Bs.shape) != (kb, N, 16)
             or tuple(C.shape) != (M, N)):
-        raise ValueError("operand shapes do not match: Aq [M, K/2], As [M, K/16], Bq [N, K/2], Bs [N, K/16], C [M, N]")
+        raise ValueError("operand shapes do not match: Aq [M, K/2], As [ceil(K/256), M, 16], Bq [N, K/2], "
+                         "Bs [ceil(K/256), N, 16], C [M, N]")
     with torch.cuda.device(Aq.device):
         st = _stream(stream)
         _check(_lib.puro_nvfp4_gemm(_ptr(Aq), _ptr(As), _ptr(a_amax), _ptr(Bq), _ptr(Bs), _ptr(b_amax), _ptr(C),
@@ -363,11 +365,11 @@ def nvfp4_quantize(X, transposed=False, stream=None):
     amax = torch.empty(1, dtype=torch.float32, device=X.device)
     if transposed:
         q = torch.empty((C, R // 2), dtype=torch.uint8, device=X.device)
-        f = torch.empty((C, R // 16), dtype=torch.uint8, device=X.device)
+        f = torch.zeros(((R + 255) // 256, C, 16), dtype=torch.uint8, device=X.device)
         puro_nvfp4_quantize_1x16_transposed(X, q, f, amax, stream)
     else:
         q = torch.empty((R, C // 2), dtype=torch.uint8, device=X.device)
-        f = torch.empty((R, C // 16), dtype=torch.uint8, device=X.device)
+        f = torch.zeros(((C + 255) // 256, R, 16), dtype=torch.uint8, device=X.device)
         puro_nvfp4_quantize_1x16(X, q, f, amax, stream)
     return q, f, amax
 

@@ -204,6 +204,10 @@ PURO_API int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_
  *     S   = dec(e) * s_t
  *     q   = E2M1_RNE_sat(x / S)                  (S == 0: a signed zero)
  * every step correctly rounded in FP32. Two codes per byte, element 2i in the low nibble.
+ * Factors are stored by 256-element K block: F[b][r][j], 16 bytes per row and block, is the
+ * factor of row r's elements 256 b + 16 j .. 256 b + 16 j + 15 (the last block's bytes past
+ * the row's end are not written), so the GEMM reads one K block's factors of consecutive rows
+ * as one contiguous run.
  * Inputs must be finite. Each quantiser runs two kernels on `stream`: the tensor's absolute
  * maximum (written to *amax, which the call first sets to zero), then the codes, which read
  * *amax on the device. Nothing else is written and nothing is allocated.
@@ -211,14 +215,14 @@ PURO_API int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_
  * puro_nvfp4_quantize_1x16: groups along the columns of X.
  *   X    [R, C] BF16, row stride ldx (>= C, % 8 == 0)   input
  *   Xq   [R, C/2] bytes, row stride ldq (>= C/2, % 8)   output: packed codes
- *   F    [R, C/16] bytes, dense                          output: F[r, j] factor of X[r, 16j..16j+15]
+ *   F    [ceil(C/256), R, 16] bytes                       output: factors, by K block
  *   amax one float                                       output: max |X|
  *   Requires R >= 1, C >= 16, C % 16 == 0; X, Xq, F 16-byte aligned, amax 4-byte aligned.
  * puro_nvfp4_quantize_1x16_transposed: groups of 16 consecutive rows (tokens), written
  * transposed (the wgrad operands, and W along N_out for dgrad).
  *   X    [R, C] BF16, row stride ldx (>= C, % 8 == 0)   input
  *   XqT  [C, R/2] bytes, row stride ldq (>= R/2, % 16)  output: packed codes of X^T
- *   FT   [C, R/16] bytes, dense                          output: FT[c, j] factor of X[16j..16j+15, c]
+ *   FT   [ceil(R/256), C, 16] bytes                       output: factors of X^T's rows, by K block
  *   amax one float                                       output: max |X|
  *   Requires R % 64 == 0 (R >= 64), C % 8 == 0; alignment as above.
  * Status: PURO_ERR_NULL, PURO_ERR_SHAPE, PURO_ERR_ALIGN, PURO_ERR_DEVICE, PURO_ERR_CUDA or
@@ -237,8 +241,8 @@ PURO_API int puro_nvfp4_quantize_1x16_transposed(const uint16_t *X, int64_t R, i
  * with s_t = amax / 2688 of each operand's tensor, rounded to BF16 (nearest even) once.
  * Both operands are quantised along K (the 1x16 quantisers above): fprop takes X and W
  * row-wise, dgrad dY row-wise and W transposed, wgrad dY and X transposed.
- *   Aq [M, K/2] packed codes, dense     As [M, K/16] factors, dense     a_amax: A's tensor amax
- *   Bq [N, K/2] packed codes, dense     Bs [N, K/16] factors, dense     b_amax: B's tensor amax
+ *   Aq [M, K/2] packed codes, dense   As [ceil(K/256), M, 16] factors   a_amax: A's tensor amax
+ *   Bq [N, K/2] packed codes, dense   Bs [ceil(K/256), N, 16] factors   b_amax: B's tensor amax
  *   C  [M, N] BF16, dense               output
  * Requires M >= 1, N >= 8, N % 8 == 0, K >= 128, K % 128 == 0; Aq, As, Bq, Bs, C 16-byte
  * aligned, the amax pointers 4-byte aligned (device memory). Status codes as for

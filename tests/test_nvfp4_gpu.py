@@ -43,19 +43,25 @@ def rand_bf16(shape, seed, scale=1.0, tails=True):
     return x.to(torch.bfloat16)
 
 
+def unblocked(f_blocked, groups):
+    """[ceil(K/256), R, 16] -> [R, K/16] (the defined bytes)."""
+    nb, r, _ = f_blocked.shape
+    return f_blocked.transpose(1, 0, 2).reshape(r, nb * 16)[:, :groups]
+
+
 def check_rows(pf, x, ldq_pad=0, ldx_pad=0):
     R, C = x.shape
     xs = torch.zeros((R, C + ldx_pad), dtype=torch.bfloat16, device="cuda")
     xs[:, :C] = x.cuda()
     X = xs[:, :C]
     q_full = torch.zeros((R, C // 2 + ldq_pad), dtype=torch.uint8, device="cuda")
-    f = torch.zeros((R, C // 16), dtype=torch.uint8, device="cuda")
+    f = torch.zeros(((C + 255) // 256, R, 16), dtype=torch.uint8, device="cuda")
     amax = torch.full((1,), -1.0, device="cuda")
     pf.puro_nvfp4_quantize_1x16(X, q_full[:, :C // 2], f, amax)
     sync(pf)
     wq, wf, wa = onv.quant_1x16(bits_of(x))
     assert amax.item() == float(wa) or (amax.item() == 0 and wa == 0)
-    assert np.array_equal(f.cpu().numpy(), wf)
+    assert np.array_equal(unblocked(f.cpu().numpy(), C // 16), wf)
     assert np.array_equal(q_full[:, :C // 2].cpu().numpy(), wq)
     if ldq_pad:
         assert not q_full[:, C // 2:].any(), "nothing written past a row's codes"
@@ -65,12 +71,12 @@ def check_cols(pf, x):
     R, C = x.shape
     X = x.cuda()
     q = torch.zeros((C, R // 2), dtype=torch.uint8, device="cuda")
-    f = torch.zeros((C, R // 16), dtype=torch.uint8, device="cuda")
+    f = torch.zeros(((R + 255) // 256, C, 16), dtype=torch.uint8, device="cuda")
     amax = torch.zeros(1, device="cuda")
     pf.puro_nvfp4_quantize_1x16_transposed(X, q, f, amax)
     wq, wf, wa = onv.quant_1x16_transposed(bits_of(x))
     assert amax.item() == float(wa)
-    assert np.array_equal(f.cpu().numpy(), wf)
+    assert np.array_equal(unblocked(f.cpu().numpy(), R // 16), wf)
     assert np.array_equal(q.cpu().numpy(), wq)
 
 
@@ -106,7 +112,7 @@ def test_quant_rows_worked_row(pf):
     q, f, a = pf.nvfp4_quantize(x.cuda())
     sync(pf)
     assert a.item() == g["tensor_amax"]
-    assert f.cpu().numpy().reshape(-1).tolist() == g["factors"]
+    assert unblocked(f.cpu().numpy(), 4).reshape(-1).tolist() == g["factors"]
     assert onv.unpack(q.cpu().numpy()).reshape(4, 16).tolist() == g["codes"]
 
 
@@ -140,6 +146,7 @@ def test_gemm_within_tolerance(pf, m, n, k, seed):
     sync(pf)
     host = [t.cpu().numpy() for t in ops]
     aq, af, aa, bq, bf, ba = host
+    af, bf = unblocked(af, k // 16), unblocked(bf, k // 16)
     want = onv.gemm_ref(aq, af, aa[0], bq, bf, ba[0])
     na, nb = onv.row_col_norms(aq, af, aa[0], bq, bf, ba[0])
     _tolerance_check(c.float().cpu().numpy().astype(np.float64), want, na, nb)
@@ -165,11 +172,12 @@ def test_gemm_exact_integers(pf):
     c = pf.nvfp4_gemm(aq, af, aa, bq, bf, ba)
     sync(pf)
     assert aa.item() == 2688.0 and ba.item() == 2688.0
-    fa, fb = af.cpu().numpy(), bf.cpu().numpy()
+    fa, fb = unblocked(af.cpu().numpy(), k // 16), unblocked(bf.cpu().numpy(), k // 16)
+    want = onv.gemm_ref(aq.cpu().numpy(), fa, 2688.0, bq.cpu().numpy(), fb, 2688.0)
     assert fa[0, 0] == 0x7E and fb[3, 6] == 0x7E
+    fa, fb = fa.copy(), fb.copy()
     fa[0, 0] = fb[3, 6] = 0x38
     assert (fa == 0x38).all() and (fb == 0x38).all()
-    want = onv.gemm_ref(aq.cpu().numpy(), af.cpu().numpy(), 2688.0, bq.cpu().numpy(), bf.cpu().numpy(), 2688.0)
     assert np.array_equal(want, np.round(want)), "the oracle's result is integral"
     want_bf16 = torch.from_numpy(want.astype(np.float32)).to(torch.bfloat16)
     assert torch.equal(c.cpu(), want_bf16)
@@ -185,10 +193,10 @@ def test_full_size_quantiser_and_sampled_gemm_rows(pf, m, n, k):
     sync(pf)
     wq, wf, wa = onv.quant_1x16(bits_of(a))
     assert aa.item() == float(wa)
-    assert np.array_equal(af.cpu().numpy(), wf) and np.array_equal(aq.cpu().numpy(), wq)
+    assert np.array_equal(unblocked(af.cpu().numpy(), k // 16), wf) and np.array_equal(aq.cpu().numpy(), wq)
     rows = np.sort(np.random.default_rng(42).choice(m, size=48, replace=False))
     aqh, afh = wq[rows], wf[rows]
-    bqh, bfh = bq.cpu().numpy(), bf.cpu().numpy()
+    bqh, bfh = bq.cpu().numpy(), unblocked(bf.cpu().numpy(), k // 16)
     want = onv.gemm_ref(aqh, afh, wa, bqh, bfh, ba.item())
     na, nb = onv.row_col_norms(aqh, afh, wa, bqh, bfh, ba.item())
     _tolerance_check(c.float().cpu().numpy()[rows].astype(np.float64), want, na, nb)
