@@ -79,7 +79,8 @@ def _args():
                         "'scales' for the full step with FP32 scales against power-of-two scales, "
                         "'vendor' for the library FP8 and BF16 GEMMs on the step's shapes (roofline context), "
                         "'kernels' for single GEMMs with FP32 against power-of-two scales, "
-                        "'nvfp4' for the NVFP4 quantisers and GEMMs on the step's shapes")
+                        "'nvfp4' for the NVFP4 quantisers and GEMMs on the step's shapes, "
+                        "'nvfp4-step' for the whole step in NVFP4 against FP32 scales")
     p.add_argument("--reps", type=int, default=10, help="timed repetitions of configs 1-4")
     return p.parse_args()
 
@@ -706,11 +707,12 @@ def main():
     if args.impl == "reference":
         run_reference(args)
         return
-    if args.config in ("fused", "grouped", "scales", "vendor", "kernels", "nvfp4"):
+    if args.config in ("fused", "grouped", "scales", "vendor", "kernels", "nvfp4", "nvfp4-step"):
         import bench_configs
         {"fused": bench_configs.run_fused_comparison, "grouped": bench_configs.run_grouped_comparison,
          "scales": bench_configs.run_scales_comparison, "vendor": bench_configs.run_vendor_reference,
-         "kernels": bench_configs.run_kernel_comparison, "nvfp4": bench_configs.run_nvfp4}[args.config](args)
+         "kernels": bench_configs.run_kernel_comparison, "nvfp4": bench_configs.run_nvfp4,
+         "nvfp4-step": bench_configs.run_nvfp4_step}[args.config](args)
         return
     if args.config in ("1", "2", "3", "4", "all"):
         from bench_configs import run_config

@@ -521,15 +521,17 @@ def run_kernel_comparison(args):
 
 
 NVFP4_BYTES_PER_ELEMENT = 2 + 2 + 0.5 + 1 / 16  # amax read, quantise read, codes, factors
+NVFP4_DUAL_BYTES_PER_ELEMENT = 2 + 2 + 2 * (0.5 + 1 / 16)  # the same, both layouts from one read
 
 
 def run_nvfp4(args):
     """The NVFP4 mode on the step's shapes (8192 tokens), CUDA events, L2 flushed before every
     timed call (512 MB written and read back), median over repetitions:
-    - the 1x16 quantisers (row-wise, and along the tokens written transposed) on the step's
-      activation, gradient and weight shapes, in GB/s of algorithmic bytes: the tensor-amax
-      pass reads X once, the quantising pass reads it again and writes the packed codes and
-      one factor byte per 16 elements (4.5625 bytes per element);
+    - the 1x16 quantisers (row-wise, along the tokens written transposed, and both from one
+      call) on the step's activation, gradient and weight shapes, in GB/s of algorithmic bytes:
+      the tensor-amax pass reads X once, the quantising pass reads it again and writes the
+      packed codes and one factor byte per 16 elements (4.5625 bytes per element; 5.125 for
+      both layouts);
     - the GEMMs of the kernel comparison (fprop, dgrad, wgrad and LM-head shapes), each on
       operands the NVFP4 quantisers made from seeded random BF16 tensors, in TFLOP/s and as
       a fraction of the dense FP4 tensor peak, taken as 4 x the BF16 peak (the nominal ratio
@@ -562,24 +564,27 @@ def run_nvfp4(args):
         return torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
 
     quant = []
-    for name, r, c, transposed in (("X 1x16", T, 2048, False), ("X along tokens", T, 2048, True),
-                                   ("X 1x16", T, 6144, False), ("dY 1x16", T, 12288, False),
-                                   ("dY along tokens", T, 12288, True), ("W gate/up 1x16", 12288, 2048, False),
-                                   ("W gate/up along N_out", 12288, 2048, True)):
+    for name, r, c, mode in (("X 1x16", T, 2048, "rows"), ("X along tokens", T, 2048, "cols"),
+                             ("X both (dual)", T, 2048, "dual"), ("X 1x16", T, 6144, "rows"),
+                             ("X both (dual)", T, 6144, "dual"), ("dY 1x16", T, 12288, "rows"),
+                             ("dY along tokens", T, 12288, "cols"), ("dY both (dual)", T, 12288, "dual"),
+                             ("W gate/up 1x16", 12288, 2048, "rows"), ("W gate/up along N_out", 12288, 2048, "cols"),
+                             ("W gate/up both (dual)", 12288, 2048, "dual"),
+                             ("LM-head dY both (dual)", T, 151936, "dual")):
         x = rand((r, c), 7 + len(quant))
         amax = torch.empty(1, dtype=torch.float32, device=dev)
-        if transposed:
-            q = torch.empty((c, r // 2), dtype=torch.uint8, device=dev)
-            f = torch.empty(((r + 255) // 256, c, 16), dtype=torch.uint8, device=dev)
-            fn = lambda: pf.puro_nvfp4_quantize_1x16_transposed(x, q, f, amax)
-        else:
-            q = torch.empty((r, c // 2), dtype=torch.uint8, device=dev)
-            f = torch.empty(((c + 255) // 256, r, 16), dtype=torch.uint8, device=dev)
-            fn = lambda: pf.puro_nvfp4_quantize_1x16(x, q, f, amax)
+        q = torch.empty((r, c // 2), dtype=torch.uint8, device=dev)
+        f = torch.empty(((c + 255) // 256, r, 16), dtype=torch.uint8, device=dev)
+        qt = torch.empty((c, r // 2), dtype=torch.uint8, device=dev)
+        ft = torch.empty(((r + 255) // 256, c, 16), dtype=torch.uint8, device=dev)
+        fn = {"rows": lambda: pf.puro_nvfp4_quantize_1x16(x, q, f, amax),
+              "cols": lambda: pf.puro_nvfp4_quantize_1x16_transposed(x, qt, ft, amax),
+              "dual": lambda: pf.puro_nvfp4_quantize_1x16_dual(x, q, f, qt, ft, amax)}[mode]
         ms = timed(fn)
-        gb = r * c * NVFP4_BYTES_PER_ELEMENT / 1e9
+        gb = r * c * (NVFP4_DUAL_BYTES_PER_ELEMENT if mode == "dual" else NVFP4_BYTES_PER_ELEMENT) / 1e9
         quant.append({"tensor": name, "R": r, "C": c, "us": round(ms * 1e3, 1), "GB_per_s": round(gb / (ms * 1e-3), 1)})
-        del x, q, f
+        del x, q, f, qt, ft
+        torch.cuda.empty_cache()
 
     shapes = [("fprop", T, 4096, 2048), ("fprop", T, 12288, 2048), ("fprop", T, 2048, 6144),
               ("dgrad", T, 2048, 12288), ("dgrad", T, 2048, 4096), ("wgrad", 12288, 2048, T),
@@ -602,5 +607,109 @@ def run_nvfp4(args):
                       "l2": "flushed before every timed call (512 MB written, then read back)",
                       "fp4_peak_tflops": round(fp4_peak, 1),
                       "fp4_peak_note": f"4 x {peak_src} BF16 burst ({bf16_tf}) (dense FP4 / BF16 nominal ratio)",
-                      "quant_bytes_per_element": NVFP4_BYTES_PER_ELEMENT, "quantisers": quant, "gemms": gemms}),
+                      "quant_bytes_per_element": NVFP4_BYTES_PER_ELEMENT,
+                      "dual_bytes_per_element": NVFP4_DUAL_BYTES_PER_ELEMENT, "quantisers": quant, "gemms": gemms}),
           flush=True)
+
+
+def run_nvfp4_step(args):
+    """The full micro-step (28 Qwen3-1.7B-shaped layers and the LM head at 8192 tokens, fprop +
+    dgrad + wgrad) in NVFP4 against the method's FP32-scale step, on the same seeded inputs in
+    one process. NVFP4 needs each of W, X and dY in two layouts: W row-wise (fprop) and along
+    N_out (dgrad), X row-wise and along the tokens, dY row-wise and along the tokens. Timed two
+    ways: with the single-layout quantisers (two calls per tensor, each an amax launch and a
+    codes launch: 15 launches per linear with the three GEMMs), and with the dual quantiser
+    (one call per tensor: 9 launches per linear). Every variant runs on one stream, captured
+    once into a CUDA graph and replayed; args.warmup replays, then `steps` replays between two
+    CUDA events (inputs larger than L2). The FP32-scale step is also timed as bench.py's
+    default runs it (weight quantisers and wgrads on a second stream)."""
+    from bench import Step
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    steps = max(1, min(args.steps, 10))
+    step = Step(pf, wl, args.tokens, args.layers, dev, seed=4, lm_head=not args.no_lm_head)
+    T = args.tokens
+    u8 = torch.uint8
+
+    def both(r, c):
+        """(row-wise codes, factors, amax), (transposed codes, factors, amax) buffers of [r, c]."""
+        return ((torch.empty((r, c // 2), dtype=u8, device=dev), torch.empty(((c + 255) // 256, r, 16), dtype=u8, device=dev),
+                 torch.empty(1, dtype=torch.float32, device=dev)),
+                (torch.empty((c, r // 2), dtype=u8, device=dev), torch.empty(((r + 255) // 256, c, 16), dtype=u8, device=dev),
+                 torch.empty(1, dtype=torch.float32, device=dev)))
+
+    lin_bufs, shape_bufs = [], {}
+    for _, x, w, dy, *_ in step.linears:
+        n, k = w.shape
+        wr, wt = both(n, k)
+        lin_bufs.append({"w": wr, "wt": wt, "xt": both(T, k)[1]})
+        if (n, k) not in shape_bufs:
+            dyr, dyt = both(T, n)
+            shape_bufs[(n, k)] = {"x": both(T, k)[0], "dy": dyr, "dyt": dyt,
+                                  "y": torch.empty((T, n), dtype=torch.bfloat16, device=dev),
+                                  "dx": torch.empty((T, k), dtype=torch.bfloat16, device=dev),
+                                  "dw": torch.empty((n, k), dtype=torch.bfloat16, device=dev)}
+
+    def quantise_both(t, rows, cols, dual):
+        """rows = (q, f, amax), cols = (qt, ft, amax'); with `dual` one call fills both and writes
+        the tensor's amax into cols (X's row-wise buffers are shared by the linears of one shape
+        while its transposed ones are kept per linear until its wgrad)."""
+        if dual:
+            pf.puro_nvfp4_quantize_1x16_dual(t, rows[0], rows[1], cols[0], cols[1], cols[2])
+        else:
+            pf.puro_nvfp4_quantize_1x16(t, *rows)
+            pf.puro_nvfp4_quantize_1x16_transposed(t, *cols)
+
+    def nv_step(dual):
+        g = pf.puro_nvfp4_gemm
+        ar = (lambda rows, cols: cols[2]) if dual else (lambda rows, cols: rows[2])  # row-wise side's amax
+        for (_, x, w, dy, *_), lb in zip(step.linears, lin_bufs):
+            quantise_both(w, lb["w"], lb["wt"], dual)
+        for (_, x, w, dy, *_), lb in zip(step.linears, lin_bufs):
+            sb = shape_bufs[tuple(w.shape)]
+            quantise_both(x, sb["x"], lb["xt"], dual)
+            g(*sb["x"][:2], ar(sb["x"], lb["xt"]), *lb["w"][:2], ar(lb["w"], lb["wt"]), sb["y"])
+        for i in range(len(step.linears) - 1, -1, -1):
+            _, x, w, dy, *_ = step.linears[i]
+            lb, sb = lin_bufs[i], shape_bufs[tuple(w.shape)]
+            quantise_both(dy, sb["dy"], sb["dyt"], dual)
+            g(*sb["dy"][:2], ar(sb["dy"], sb["dyt"]), *lb["wt"], sb["dx"])
+            g(*sb["dyt"], *lb["xt"], sb["dw"])
+
+    def timed_graph(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        pf.puro_fp8_sync_status()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            fn()
+        for _ in range(max(1, args.warmup)):
+            graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+        pf.puro_fp8_sync_status()
+        del graph
+        return e0.elapsed_time(e1) / steps
+
+    out = {}
+    for name, fn in (("fp32_scales_one_stream", lambda: step.run(stream=stream, overlap=False)),
+                     ("fp32_scales_two_streams", lambda: step.run(stream=stream, overlap=True)),
+                     ("nvfp4_single_layout_quantisers", lambda: nv_step(False)),
+                     ("nvfp4_dual_quantiser", lambda: nv_step(True))):
+        ms = timed_graph(fn)
+        out[name] = {"ms_per_step": round(ms, 3), "tflops": round(step.gemm_flops / (ms * 1e-3) / 1e12, 1)}
+    n_lin = len(step.linears)
+    out["launches"] = {"nvfp4_single_layout_quantisers": 15 * n_lin, "nvfp4_dual_quantiser": 9 * n_lin}
+    out["nvfp4_dual_speedup_vs_fp32_scales_one_stream"] = round(
+        out["fp32_scales_one_stream"]["ms_per_step"] / out["nvfp4_dual_quantiser"]["ms_per_step"], 3)
+    print(json.dumps({"comparison": "full step: FP32 scales + blockwise FP8 GEMM vs NVFP4 quantisers + FP4 GEMM",
+                      "workload": f"qwen3-1.7b-linear-stack-{args.layers}L{'' if args.no_lm_head else '+lm_head'} "
+                                  f"fwd+dgrad+wgrad, {T} tokens, seed 4",
+                      "steps": steps, "warmup": args.warmup, **out}), flush=True)

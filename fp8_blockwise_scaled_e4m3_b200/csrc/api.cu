@@ -192,6 +192,22 @@ int puro_nvfp4_quantize_1x16_transposed(const uint16_t *X, int64_t R, int64_t C,
   return puro::launch_nvfp4_quant_cols(X, R, C, ldx, XqT, ldq, FT, amax, stream);
 }
 
+int puro_nvfp4_quantize_1x16_dual(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                                  int64_t ldq, uint8_t *F, uint8_t *XqT, int64_t ldqt, uint8_t *FT, float *amax,
+                                  puro_stream_t stream) {
+  if (X == nullptr || Xq == nullptr || F == nullptr || XqT == nullptr || FT == nullptr || amax == nullptr)
+    return PURO_ERR_NULL;
+  if (R < 64 || R % 64 != 0 || C < 16 || C % 16 != 0 || ldx < C || ldq < C / 2 || ldqt < R / 2)
+    return PURO_ERR_SHAPE;
+  if (R > (1ll << 31) - 1 || C > (1ll << 31) - 1 || (R / 64) * ((C + 255) / 256) > (1ll << 31) - 1)
+    return PURO_ERR_SHAPE;
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(F, 16) || !aligned(XqT, 16) || !aligned(FT, 16) ||
+      !aligned(amax, 4) || ldx % 8 != 0 || ldq % 8 != 0 || ldqt % 16 != 0)
+    return PURO_ERR_ALIGN;
+  if (int d = check_device()) return d;
+  return puro::launch_nvfp4_quant_dual(X, R, C, ldx, Xq, ldq, F, XqT, ldqt, FT, amax, stream);
+}
+
 int puro_nvfp4_gemm(const uint8_t *Aq, const uint8_t *As, const float *a_amax, const uint8_t *Bq,
                     const uint8_t *Bs, const float *b_amax, uint16_t *C, int64_t M, int64_t N, int64_t K,
                     puro_stream_t stream) {

@@ -633,6 +633,30 @@ int launch_gemm_nvfp4(const uint8_t *Aq, const uint8_t *As, const float *a_amax,
                 : launch_nv<false>(Aq, As, a_amax, Bq, Bs, b_amax, C, M, N, K, stream);
 }
 
+int *nv_status_word() {
+  static PerDevice<int *> status_addr;
+  int *st = nullptr;
+  if (!status_addr.get(st, [](int, int *&v) {
+        return cudaGetSymbolAddress(reinterpret_cast<void **>(&v), g_nv_status) == cudaSuccess;
+      }))
+    return nullptr;
+  return st;
+}
+
+unsigned long long nv_wait_timeout_ns() { return nv_timeout_ns(); }
+
+bool nv_bf16_map(CUtensorMap *map, const uint16_t *X, int64_t rows, int64_t cols, int64_t ld, uint32_t box_rows) {
+  EncodeTiledFn fn = nv_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(X), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int read_and_clear_nv_status(cudaStream_t stream, int *status_out) {
   int host = 0;
   const int zero = 0;

@@ -2,6 +2,7 @@
 // validated by the C-ABI layer before these are called.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -31,10 +32,20 @@ int launch_nvfp4_quant_rows(const uint16_t *X, int64_t R, int64_t C, int64_t ldx
                             uint8_t *F, float *amax, cudaStream_t stream);
 int launch_nvfp4_quant_cols(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *XqT, int64_t ldq,
                             uint8_t *FT, float *amax, cudaStream_t stream);
+int launch_nvfp4_quant_dual(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq, int64_t ldq,
+                            uint8_t *F, uint8_t *XqT, int64_t ldqt, uint8_t *FT, float *amax,
+                            cudaStream_t stream);
 int launch_gemm_nvfp4(const uint8_t *Aq, const uint8_t *As, const float *a_amax, const uint8_t *Bq,
                       const uint8_t *Bs, const float *b_amax, uint16_t *C, int64_t M, int64_t N, int64_t K,
                       cudaStream_t stream);
 int read_and_clear_nv_status(cudaStream_t stream, int *status_out);
+// NVFP4 host helpers shared by its quantisers and GEMM: the device status word its kernels
+// raise when a bounded wait gives up (address cached per device), the wait limit, and a
+// tensor map of a BF16 matrix [rows, cols] with row stride `ld` elements, box [box_rows x 64]
+// (128 bytes per row, 128-byte swizzle), reads past the edge returning zeros.
+int *nv_status_word();
+unsigned long long nv_wait_timeout_ns();
+bool nv_bf16_map(CUtensorMap *map, const uint16_t *X, int64_t rows, int64_t cols, int64_t ld, uint32_t box_rows);
 
 // Reads and clears the quantisers' device status word (after a stream sync).
 int read_and_clear_quant_status(cudaStream_t stream, int *status_out);

@@ -65,6 +65,7 @@ def _load():
         "puro_fp8_quantize_128x128_pow2": [_p, _i64, _i64, _i64, _p, _p, _p, _p],
         "puro_nvfp4_quantize_1x16": [_p, _i64, _i64, _i64, _p, _i64, _p, _p, _p],
         "puro_nvfp4_quantize_1x16_transposed": [_p, _i64, _i64, _i64, _p, _i64, _p, _p, _p],
+        "puro_nvfp4_quantize_1x16_dual": [_p, _i64, _i64, _i64, _p, _i64, _p, _p, _i64, _p, _p, _p],
         "puro_nvfp4_gemm": [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p],
         "puro_fp8_sync_status": [_p],
     }
@@ -336,6 +337,25 @@ def puro_nvfp4_quantize_1x16_transposed(X, XqT, FT, amax, stream=None):
                "puro_nvfp4_quantize_1x16_transposed", st)
 
 
+def puro_nvfp4_quantize_1x16_dual(X, Xq, F, XqT, FT, amax, stream=None):
+    """Both NVFP4 layouts of X [R, C] bf16 from one read (see the C declaration): Xq [R, C/2] and
+    F [ceil(C/256), R, 16] along the columns, XqT [C, R/2] and FT [ceil(R/256), C, 16] along the
+    rows, amax float32 [1]."""
+    _need(X, torch.bfloat16, "X"); _need(Xq, torch.uint8, "Xq"); _need(F, torch.uint8, "F")
+    _need(XqT, torch.uint8, "XqT"); _need(FT, torch.uint8, "FT"); _need(amax, torch.float32, "amax")
+    R, C = X.shape
+    if (tuple(Xq.shape) != (R, C // 2) or tuple(F.shape) != ((C + 255) // 256, R, 16)
+            or tuple(XqT.shape) != (C, R // 2) or tuple(FT.shape) != ((R + 255) // 256, C, 16) or amax.numel() != 1):
+        raise ValueError("Xq must be [R, C/2], F [ceil(C/256), R, 16], XqT [C, R/2], FT [ceil(R/256), C, 16] "
+                         "and amax one float")
+    _dense(F, "F"); _dense(FT, "FT")
+    with torch.cuda.device(X.device):
+        st = _stream(stream)
+        _check(_lib.puro_nvfp4_quantize_1x16_dual(_ptr(X), R, C, X.stride(0), _ptr(Xq), Xq.stride(0), _ptr(F),
+                                                  _ptr(XqT), XqT.stride(0), _ptr(FT), _ptr(amax), st),
+               "puro_nvfp4_quantize_1x16_dual", st)
+
+
 def puro_nvfp4_gemm(Aq, As, a_amax, Bq, Bs, b_amax, C, stream=None):
     """NVFP4 GEMM C [M, N] bf16 = A . B^T of two operands quantised along K (see the C
     declaration): Aq [M, K/2], Bq [N, K/2] packed codes, As [ceil(K/256), M, 16], Bs
@@ -372,6 +392,18 @@ def nvfp4_quantize(X, transposed=False, stream=None):
         f = torch.zeros(((C + 255) // 256, R, 16), dtype=torch.uint8, device=X.device)
         puro_nvfp4_quantize_1x16(X, q, f, amax, stream)
     return q, f, amax
+
+
+def nvfp4_quantize_dual(X, stream=None):
+    """((Xq, F), (XqT, FT), amax): both NVFP4 layouts of X from one call (allocating helper)."""
+    R, C = X.shape
+    amax = torch.empty(1, dtype=torch.float32, device=X.device)
+    q = torch.empty((R, C // 2), dtype=torch.uint8, device=X.device)
+    f = torch.zeros(((C + 255) // 256, R, 16), dtype=torch.uint8, device=X.device)
+    qt = torch.empty((C, R // 2), dtype=torch.uint8, device=X.device)
+    ft = torch.zeros(((R + 255) // 256, C, 16), dtype=torch.uint8, device=X.device)
+    puro_nvfp4_quantize_1x16_dual(X, q, f, qt, ft, amax, stream)
+    return (q, f), (qt, ft), amax
 
 
 def nvfp4_gemm(Aq, As, a_amax, Bq, Bs, b_amax, stream=None):

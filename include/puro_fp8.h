@@ -225,6 +225,13 @@ PURO_API int puro_fp8_mx_gemm(const uint8_t *Aq, const uint8_t *As, const uint8_
  *   FT   [ceil(R/256), C, 16] bytes                       output: factors of X^T's rows, by K block
  *   amax one float                                       output: max |X|
  *   Requires R % 64 == 0 (R >= 64), C % 8 == 0; alignment as above.
+ * puro_nvfp4_quantize_1x16_dual: both of the above from one read of X (plus the amax pass):
+ * the outputs are byte for byte those of the two calls, with one amax shared by both.
+ *   X, Xq, ldq, F    as for puro_nvfp4_quantize_1x16
+ *   XqT, ldqt, FT    as XqT, ldq, FT of puro_nvfp4_quantize_1x16_transposed
+ *   amax             one float, output: max |X|
+ *   Requires R % 64 == 0 (R >= 64), C % 16 == 0 (C >= 16), ldq % 8 == 0, ldqt % 16 == 0;
+ *   alignment as above.
  * Status: PURO_ERR_NULL, PURO_ERR_SHAPE, PURO_ERR_ALIGN, PURO_ERR_DEVICE, PURO_ERR_CUDA or
  * PURO_ERR_LAUNCH, checked on the host before any launch.
  */
@@ -233,6 +240,9 @@ PURO_API int puro_nvfp4_quantize_1x16(const uint16_t *X, int64_t R, int64_t C, i
 PURO_API int puro_nvfp4_quantize_1x16_transposed(const uint16_t *X, int64_t R, int64_t C, int64_t ldx,
                                                  uint8_t *XqT, int64_t ldq, uint8_t *FT, float *amax,
                                                  puro_stream_t stream);
+PURO_API int puro_nvfp4_quantize_1x16_dual(const uint16_t *X, int64_t R, int64_t C, int64_t ldx, uint8_t *Xq,
+                                           int64_t ldq, uint8_t *F, uint8_t *XqT, int64_t ldqt, uint8_t *FT,
+                                           float *amax, puro_stream_t stream);
 
 /*
  * NVFP4 GEMM on the tensor cores' block-scaled FP4 MMA, which applies the UE4M3 factors

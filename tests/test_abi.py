@@ -47,8 +47,8 @@ def test_header_declares_the_entry_points():
         "puro_fp8_gemm_blockwise_grouped", "puro_fp8_quantize_1x128_pow2",
         "puro_fp8_quantize_1x128_transposed_pow2", "puro_fp8_quantize_128x128_pow2", "puro_fp8_mx_gemm",
         "puro_fp8_quantize_128x128_grouped",
-        "puro_nvfp4_quantize_1x16", "puro_nvfp4_quantize_1x16_transposed", "puro_nvfp4_gemm",
-        "puro_fp8_sync_status", "puro_strerror"])
+        "puro_nvfp4_quantize_1x16", "puro_nvfp4_quantize_1x16_transposed", "puro_nvfp4_quantize_1x16_dual",
+        "puro_nvfp4_gemm", "puro_fp8_sync_status", "puro_strerror"])
 
 
 def test_library_exports_exactly_the_declared_symbols(lib):
@@ -300,6 +300,14 @@ def test_nvfp4_entry_points_reject_bad_arguments(lib):
     assert qt(A16, 128, 60, 64, A16, 64, A16, A16, None) == ESHAPE           # C % 8
     assert qt(A16, 128, 64, 64, A16, 32, A16, A16, None) == ESHAPE           # ldq < R / 2
     assert qt(A16, 128, 64, 64, A16, 72, A16, A16, None) == EALIGN           # ldq % 16
+    d = lib.puro_nvfp4_quantize_1x16_dual
+    assert d(A16, 128, 64, 64, A16, 32, A16, None, 64, A16, A16, None) == ENULL      # XqT
+    assert d(A16, 100, 64, 64, A16, 32, A16, A16, 64, A16, A16, None) == ESHAPE      # R % 64
+    assert d(A16, 128, 56, 64, A16, 32, A16, A16, 64, A16, A16, None) == ESHAPE      # C % 16
+    assert d(A16, 128, 64, 64, A16, 32, A16, A16, 48, A16, A16, None) == ESHAPE      # ldqt < R / 2
+    assert d(A16, 128, 64, 64, A16, 32, A16, A16, 72, A16, A16, None) == EALIGN      # ldqt % 16
+    assert d(A16, 128, 64, 64, A16, 36, A16, A16, 64, A16, A16, None) == EALIGN      # ldq % 8
+    assert d(A16, 128, 64, 64, A16, 32, A16, A16, 64, A16 + 4, A16, None) == EALIGN  # FT 16-byte aligned
     g = lib.puro_nvfp4_gemm
     ops = [A16, A16, A16, A16, A16, A16, A16]
     assert g(None, *ops[1:], 128, 256, 256, None) == ENULL

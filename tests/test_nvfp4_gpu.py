@@ -1,7 +1,7 @@
 """NVFP4 mode on the GPU against the oracle (oracle/nvfp4.py), through the C ABI.
 
-- quantisers: packed codes, UE4M3 factors and the tensor amax bit-exact, row-wise and
-  transposed, on ragged and strided shapes, all-zero groups, negative zeros, a tiny tensor
+- quantisers: packed codes, UE4M3 factors and the tensor amax bit-exact, row-wise,
+  transposed and both from one call (dual), on ragged and strided shapes, all-zero groups, negative zeros, a tiny tensor
   (subnormal factors) and the hand-worked row of tests/golden/nvfp4_blocks_worked.json;
 - GEMM: the benchmark spec's tolerance (relative Frobenius <= 2e-3, elementwise <= 1e-2 ||a_m|| ||b_n||)
   against the FP64 oracle, including a half K block (K % 256 == 128), single CTAs and CTA
@@ -17,6 +17,7 @@ import pytest
 import torch
 
 from oracle import nvfp4 as onv
+from oracle.quant import bf16_bits_to_f32
 
 pytestmark = pytest.mark.gpu
 
@@ -202,6 +203,82 @@ def test_full_size_quantiser_and_sampled_gemm_rows(pf, m, n, k):
     _tolerance_check(c.float().cpu().numpy()[rows].astype(np.float64), want, na, nb)
 
 
+def run_dual(pf, X, pads=(0, 0)):
+    R, C = X.shape
+    q = torch.zeros((R, C // 2 + pads[0]), dtype=torch.uint8, device="cuda")
+    qt = torch.zeros((C, R // 2 + pads[1]), dtype=torch.uint8, device="cuda")
+    f = torch.zeros(((C + 255) // 256, R, 16), dtype=torch.uint8, device="cuda")
+    ft = torch.zeros(((R + 255) // 256, C, 16), dtype=torch.uint8, device="cuda")
+    amax = torch.full((1,), -1.0, device="cuda")
+    pf.puro_nvfp4_quantize_1x16_dual(X, q[:, :C // 2], f, qt[:, :R // 2], ft, amax)
+    sync(pf)
+    if pads[0]:
+        assert not q[:, C // 2:].any()
+    if pads[1]:
+        assert not qt[:, R // 2:].any()
+    return q[:, :C // 2], f, qt[:, :R // 2], ft, amax
+
+
+@pytest.mark.parametrize("shape,seed,pads", [((64, 16), 20, (0, 0)), ((128, 272), 21, (8, 16)),
+                                             ((192, 512), 22, (0, 0)), ((256, 2064), 23, (24, 32)),
+                                             ((640, 768), 24, (0, 0))])
+def test_quant_dual_bit_exact(pf, shape, seed, pads):
+    """One call, both layouts: each equal to its oracle routine byte for byte, with tiles that end
+    inside a 256-column block (272, 2064) and padded output rows."""
+    R, C = shape
+    x = rand_bf16(shape, seed)
+    xs = torch.zeros((R, C + 8), dtype=torch.bfloat16, device="cuda")
+    xs[:, :C] = x.cuda()
+    q, f, qt, ft, amax = run_dual(pf, xs[:, :C], pads)
+    wq, wf, wa = onv.quant_1x16(bits_of(x))
+    tq, tf, ta = onv.quant_1x16_transposed(bits_of(x))
+    assert amax.item() == float(wa) == float(ta)
+    assert np.array_equal(q.cpu().numpy(), wq) and np.array_equal(unblocked(f.cpu().numpy(), C // 16), wf)
+    assert np.array_equal(qt.cpu().numpy(), tq) and np.array_equal(unblocked(ft.cpu().numpy(), R // 16), tf)
+
+
+def test_quant_dual_special_groups(pf):
+    x = rand_bf16((64, 256), 25)
+    x[1, :16] = 0.0
+    x[:16, 3] = -0.0
+    x[2, 32:48] = 1e-30
+    x[16:32, 40] = 1e-30
+    x[5, 7] = -3000.0  # the tensor amax
+    for t in (x, torch.zeros((64, 32), dtype=torch.bfloat16), (torch.randn((64, 48)) * 1e-38).to(torch.bfloat16)):
+        q, f, qt, ft, amax = run_dual(pf, t.cuda())
+        wq, wf, wa = onv.quant_1x16(bits_of(t))
+        tq, tf, _ = onv.quant_1x16_transposed(bits_of(t))
+        assert amax.item() == float(wa)
+        assert np.array_equal(q.cpu().numpy(), wq) and np.array_equal(unblocked(f.cpu().numpy(), t.shape[1] // 16), wf)
+        assert np.array_equal(qt.cpu().numpy(), tq) and np.array_equal(unblocked(ft.cpu().numpy(), t.shape[0] // 16), tf)
+
+
+@pytest.mark.parametrize("R,C", [(8192, 2048), (8192, 151936)])
+def test_quant_dual_full_size(pf, R, C):
+    """The step's activation (8192 x 2048) and LM-head dlogits (8192 x 151936) shapes: the dual
+    call equals the two single calls byte for byte; sampled rows and columns equal the oracle's
+    groups under the tensor's exact amax."""
+    x = rand_bf16((R, C), 26, tails=C < 100000).cuda()
+    q, f, qt, ft, amax = run_dual(pf, x)
+    q1, f1, a1 = pf.nvfp4_quantize(x)
+    q2, f2, a2 = pf.nvfp4_quantize(x, transposed=True)
+    sync(pf)
+    assert amax.item() == a1.item() == a2.item()
+    assert torch.equal(q, q1) and torch.equal(f, f1) and torch.equal(qt, q2) and torch.equal(ft, f2)
+    xb = bits_of(x)
+    wa = onv.tensor_amax(xb)
+    assert amax.item() == float(wa)
+    rng = np.random.default_rng(27)
+    rows = np.sort(rng.choice(R, size=16, replace=False))
+    codes, fac = onv.quantize_groups(bf16_bits_to_f32(xb[rows]).reshape(16, C // 16, 16), wa)
+    assert np.array_equal(q[rows].cpu().numpy(), onv.pack(codes.reshape(16, C)))
+    assert np.array_equal(unblocked(f.cpu().numpy(), C // 16)[rows], fac)
+    cols = np.sort(rng.choice(C, size=16, replace=False))
+    codes, fac = onv.quantize_groups(bf16_bits_to_f32(np.ascontiguousarray(xb[:, cols].T)).reshape(16, R // 16, 16), wa)
+    assert np.array_equal(qt[cols].cpu().numpy(), onv.pack(codes.reshape(16, R)))
+    assert np.array_equal(unblocked(ft.cpu().numpy(), R // 16)[cols], fac)
+
+
 def test_argument_errors(pf):
     lib = pf.library()
     st = pf._stream(None)
@@ -215,6 +292,13 @@ def test_argument_errors(pf):
     assert lib.puro_nvfp4_quantize_1x16(p(x), 4, 32, 32, p(q), 8, p(f), p(a), st) == -2    # ldq < C/2
     assert lib.puro_nvfp4_quantize_1x16(p(x), 4, 32, 32, p(q) + 1, 16, p(f), p(a), st) == -3  # alignment
     assert lib.puro_nvfp4_quantize_1x16_transposed(p(x), 4, 32, 32, p(q), 16, p(f), p(a), st) == -2  # R % 64
+    assert lib.puro_nvfp4_quantize_1x16_dual(p(x), 4, 32, 32, p(q), 16, p(f), p(q), 16, p(f), p(a), st) == -2
+    x64 = torch.zeros((64, 32), dtype=torch.bfloat16, device="cuda")
+    q64, qt64 = torch.zeros((64, 16), dtype=torch.uint8, device="cuda"), torch.zeros((32, 32), dtype=torch.uint8, device="cuda")
+    f64 = torch.zeros((1, 64, 16), dtype=torch.uint8, device="cuda")
+    assert lib.puro_nvfp4_quantize_1x16_dual(p(x64), 64, 32, 32, p(q64), 16, p(f64), p(qt64), 32, p(f64), p(a), st) == 0
+    assert lib.puro_nvfp4_quantize_1x16_dual(p(x64), 64, 32, 32, p(q64), 16, p(f64), p(qt64), 40, p(f64), p(a), st) == -3
+    assert lib.puro_nvfp4_quantize_1x16_dual(p(x64), 64, 32, 32, p(q64), 16, None, p(qt64), 32, p(f64), p(a), st) == -1
     c = torch.zeros((128, 8), dtype=torch.bfloat16, device="cuda")
     ops = torch.zeros((128, 64), dtype=torch.uint8, device="cuda")
     fs = torch.zeros((128, 8), dtype=torch.uint8, device="cuda")
