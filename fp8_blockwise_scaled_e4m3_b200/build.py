@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libpuro_fp8.so")
 SOURCES = ["quant.cu", "gemm.cu", "gemm_mx.cu", "nvfp4_quant.cu", "gemm_nvfp4.cu", "api.cu"]
-HEADERS = ["ptx.cuh", "quant.h", "quant_math.cuh", "host_cache.h"]
+HEADERS = ["ptx.cuh", "quant.h", "quant_math.cuh", "nvfp4_math.cuh", "host_cache.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

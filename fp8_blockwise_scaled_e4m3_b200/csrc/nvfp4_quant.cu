@@ -29,7 +29,8 @@
 //   k_nv_quant_dual  both of the above from one read of X: persistent CTAs take 128 x 128 tiles
 //                    through a two-stage TMA ring (two 128-byte-swizzled boxes of 64 columns per
 //                    tile); a thread quantises 64 elements of one row, then two columns over 32
-//                    rows, both from shared memory without bank conflicts
+//                    rows, both from shared memory without bank conflicts; the transposed codes
+//                    leave through a staging buffer as whole 64-byte rows
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -156,7 +157,8 @@ constexpr int kDualBox = kDualTile * 128;       // one TMA box: 128 rows x 64 BF
 constexpr int kDualStage = 2 * kDualBox;        // one tile, 32 KB
 constexpr int kDualStages = 2;
 constexpr int kDualCtas = 3;                    // CTAs per SM
-constexpr int kDualSmem = kDualStages * kDualStage + 1024 + 64;  // + alignment, barriers, flag
+constexpr int kDualStg = 8192 + 1024;           // staging of a tile's transposed codes and factors
+constexpr int kDualSmem = kDualStages * kDualStage + kDualStg + 1024 + 64;  // + alignment, barriers, flag
 
 struct NvDualArgs {
   int64_t R, C, ldq, ldqt;
@@ -175,17 +177,20 @@ struct NvDualArgs {
 //    factor bytes (one K block's bytes 4 m .. 4 m + 3) per thread;
 //  - columns: thread (pair p = tid % 64, quarter = tid / 64) reads the 4-byte word of columns
 //    2p, 2p + 1 from the 32 rows of its quarter (a warp reads the 32 words of one row), takes
-//    both columns' group maxima with packed BF16 maxima, and writes 16 bytes of codes and 2
-//    factor bytes per column;
-// then the CTA syncs and thread 0 refills the stage.
+//    both columns' group maxima with packed BF16 maxima, and forms 16 bytes of codes and 2
+//    factor bytes per column, written into a staging buffer (8 KB of codes, 1 KB of factors);
+//    after a CTA sync they leave it as whole 64-byte rows of XqT and 8-byte runs of FT, instead
+//    of one partial sector per thread and column;
+// then the CTA syncs (the stage and the staging buffer are free) and thread 0 refills the stage.
 __global__ void __launch_bounds__(kThreads, kDualCtas)
     k_nv_quant_dual(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ NvDualArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + kDualStages * kDualStage;
-  volatile int *fail = reinterpret_cast<volatile int *>(smem + kDualStages * kDualStage + 8 * kDualStages);
+  uint8_t *stg = smem + kDualStages * kDualStage;
+  const uint32_t bar0 = sbase + kDualStages * kDualStage + kDualStg;
+  volatile int *fail = reinterpret_cast<volatile int *>(smem + kDualStages * kDualStage + kDualStg + 8 * kDualStages);
   const int tid = threadIdx.x;
   if (tid == 0) {
     for (int s = 0; s < kDualStages; ++s) mbar_init(bar0 + 8 * s, 1);
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, kDualCtas)
       }
     }
 
-    // ---- down the columns
+    // ---- down the columns, staged
     {
       const int64_t c = c0 + 2 * p, rq = r0 + 32 * quarter;
       if (c < a.C && rq < a.R) {
@@ -273,12 +278,34 @@ __global__ void __launch_bounds__(kThreads, kDualCtas)
           const uint32_t e0 = col ? nv_col_group<true>(w, m0, t, o[0], o[1]) : nv_col_group<false>(w, m0, t, o[0], o[1]);
           const uint32_t e1 = col ? nv_col_group<true>(w + 16, m1, t, o[2], o[3])
                                   : nv_col_group<false>(w + 16, m1, t, o[2], o[3]);
-          *reinterpret_cast<uint4 *>(a.XqT + (c + col) * a.ldqt + rq / 2) = make_uint4(o[0], o[1], o[2], o[3]);
-          // groups rq/16 and rq/16 + 1 of column c + col: K block rq / 256, bytes (rq / 16) % 16 ..
-          *reinterpret_cast<uint16_t *>(a.FT + ((rq >> 8) * a.C + c + col) * 16 + ((rq >> 4) & 15)) =
+          // codes of column 2p + col, rows 32 quarter .. + 31: 16-byte chunk 4 col + quarter of
+          // staging pair-row p (columns 2p, 2p + 1), XOR-swizzled by p so that the eight
+          // threads of a quarter warp write eight different bank groups
+          *reinterpret_cast<uint4 *>(stg + p * 128 + (((4 * col + quarter) ^ (p & 7)) << 4)) =
+              make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint16_t *>(stg + 8192 + (2 * p + col) * 8 + 2 * quarter) =
               static_cast<uint16_t>(e0 | (e1 << 8));
         }
       }
+    }
+    __syncthreads();
+    // copy-out: each column's 64 bytes of codes as four 16-byte stores (a warp writes 8 full
+    // 64-byte row segments of XqT), its 8 factor bytes as one 8-byte store
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int u = tid + kThreads * h, r = u >> 2, j = u & 3;
+      if (c0 + r < a.C && r0 + 32 * j < a.R)
+        *reinterpret_cast<uint4 *>(a.XqT + (c0 + r) * a.ldqt + r0 / 2 + 16 * j) =
+            *reinterpret_cast<const uint4 *>(stg + (r >> 1) * 128 + (((4 * (r & 1) + j) ^ ((r >> 1) & 7)) << 4));
+    }
+    if (tid < kDualTile && c0 + tid < a.C) {
+      // groups r0/16 .. r0/16 + 7 of column c0 + tid: K block r0 / 256, bytes 8 (tr % 2) ..
+      uint8_t *df = a.FT + ((r0 >> 8) * a.C + c0 + tid) * 16 + ((r0 >> 4) & 15);
+      const uint2 f = *reinterpret_cast<const uint2 *>(stg + 8192 + tid * 8);
+      if (r0 + kDualTile <= a.R)
+        *reinterpret_cast<uint2 *>(df) = f;
+      else  // 64 rows left: their four groups only
+        *reinterpret_cast<uint32_t *>(df) = f.x;
     }
     __syncthreads();  // the stage is consumed
     if (tid == 0) issue(i + kDualStages);
