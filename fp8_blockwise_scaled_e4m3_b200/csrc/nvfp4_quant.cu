@@ -9,11 +9,12 @@
 //   e   = E4M3_RNE_sat(RN(RN(amax_g / 6) / s_t))      the group's UE4M3 factor
 //   S   = RN(dec(e) * s_t)
 //   q   = E2M1_RNE_sat(RN(x / S)), or a signed zero when S == 0
-// Two codes per byte (element 2i in the low nibble). Factors are stored by 256-element K
-// block: F[b][r][j] (16 bytes per row and block) is the factor of X[r, 256 b + 16 j ..], so the
-// GEMM reads a K block's factors of consecutive rows as one contiguous run. The tensor amax is
-// an output of its own kernel, read by the quantising kernel from device memory, so the two launches need no host
-// round trip. Inputs must be finite.
+// (the arithmetic, and how it stays correctly rounded, is in nvfp4_math.cuh). Two codes per
+// byte (element 2i in the low nibble). Factors are stored by 256-element K block: F[b][r][j]
+// (16 bytes per row and block) is the factor of X[r, 256 b + 16 j ..], so the GEMM reads a K
+// block's factors of consecutive rows as one contiguous run. The tensor amax is an output of
+// its own kernel, read by the quantising kernel from device memory, so the two launches need no
+// host round trip. Inputs must be finite.
 //
 //   k_nv_amax        max |x| over X [R, C]: a warp per row (or row segment, when rows are too few
 //                    to fill the GPU), four 16-byte loads in flight per lane, a block maximum,
