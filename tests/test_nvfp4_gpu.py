@@ -221,10 +221,11 @@ def run_dual(pf, X, pads=(0, 0)):
 
 @pytest.mark.parametrize("shape,seed,pads", [((64, 16), 20, (0, 0)), ((128, 272), 21, (8, 16)),
                                              ((192, 512), 22, (0, 0)), ((256, 2064), 23, (24, 32)),
-                                             ((640, 768), 24, (0, 0))])
+                                             ((640, 768), 24, (0, 0)), ((128, 80), 28, (0, 0))])
 def test_quant_dual_bit_exact(pf, shape, seed, pads):
     """One call, both layouts: each equal to its oracle routine byte for byte, with tiles that end
-    inside a 256-column block (272, 2064) and padded output rows."""
+    inside a 256-column block (272, 2064, 80), padded output rows, and code rows that are only
+    8-byte aligned (C = 80: a row stride of 40 bytes)."""
     R, C = shape
     x = rand_bf16(shape, seed)
     xs = torch.zeros((R, C + 8), dtype=torch.bfloat16, device="cuda")
