@@ -39,17 +39,22 @@ __device__ __forceinline__ float ue4m3_value(uint32_t b) {
                  : __uint_as_float(((ex + 120u) << 23) | (m << 20));
 }
 
-// The tensor's constants: s_t, and RN(1 / s_t) when the fast path applies.
+// The tensor's constants: s_t, and RN(1 / s_t) when the fast path applies. `all_fast`: s_t >=
+// 2^-81, so that every group of the tensor takes the fast path: a group maximum below 2^-100
+// gives a quotient by s_t below 2^-21 (factor 0, whatever its last bits), and every non-zero
+// factor's S = dec(e) * s_t is at least 2^-9 * 2^-81 = 2^-90.
 struct NvTensor {
   float s_t;
   float r_t;
   bool fast;
+  bool all_fast;
 };
 
 __device__ __forceinline__ NvTensor nv_tensor(float amax_t) {
   NvTensor t;
   t.s_t = __fdiv_rn(amax_t, kNvTensorDiv);
   t.fast = t.s_t >= 0x1p-90f;  // s_t <= 2^128 / 2688 < 2^120 always
+  t.all_fast = t.s_t >= 0x1p-81f;
   t.r_t = t.fast ? rcp_rn_fast(t.s_t) : 0.0f;
   return t;
 }
@@ -67,8 +72,10 @@ __device__ __noinline__ uint2 nv_factor_exact(float amax_g, float s_t) {
 // The same, by Markstein's correction when the tensor and the group allow it (amax_g = 0, or
 // amax_g >= 2^-100 so that amax_g / 6 is a normal number; the quotient by s_t is at most
 // about 448, and where it is below the normal range its factor is zero either way).
+// ALL_FAST: the caller has checked t.all_fast, and no group needs the exact path.
+template <bool ALL_FAST = false>
 __device__ __forceinline__ uint32_t nv_factor(float amax_g, const NvTensor &t, float &S) {
-  if (t.fast && (amax_g == 0.0f || amax_g >= 0x1p-100f)) {
+  if (ALL_FAST || (t.fast && (amax_g == 0.0f || amax_g >= 0x1p-100f))) {
     const float q = __fmul_rn(amax_g, kNvInv6);
     const float d = __fmaf_rn(__fmaf_rn(-q, 6.0f, amax_g), kNvInv6, q);
     const float q2 = __fmul_rn(d, t.r_t);
@@ -90,9 +97,10 @@ struct NvDivider {
   bool fast;
 };
 
+template <bool ALL_FAST = false>
 __device__ __forceinline__ NvDivider nv_divider(float S) {
   NvDivider d;
-  d.fast = S == 0.0f || S >= 0x1p-90f;
+  d.fast = ALL_FAST || S == 0.0f || S >= 0x1p-90f;
   const float s = S == 0.0f ? 1.0f : S;
   const float r = S == 0.0f ? 0.0f : (d.fast ? rcp_rn_fast(S) : 0.0f);
   d.nr2 = pack2(-r, -r);
@@ -151,6 +159,7 @@ __device__ __noinline__ uint32_t nv_codes8_exact(uint4 a, uint4 b, bool pairs, b
 
 // A 16-element group held in two 16-byte words (element 2i in the low half of word i): its
 // factor byte, and its eight bytes of codes in out0 (elements 0..7) and out1.
+template <bool ALL_FAST = false>
 __device__ __forceinline__ uint32_t nv_row_group(const uint4 &v0, const uint4 &v1, const NvTensor &t, uint32_t &out0,
                                                  uint32_t &out1) {
   uint32_t m = bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(v0.x, v0.y), bf16x2_absmax(v0.z, v0.w)),
@@ -158,9 +167,9 @@ __device__ __forceinline__ uint32_t nv_row_group(const uint4 &v0, const uint4 &v
   m &= 0x7FFF7FFFu;
   m = max(m & 0xFFFFu, m >> 16);
   float S;
-  const uint32_t e = nv_factor(__uint_as_float(m << 16), t, S);
-  const NvDivider d = nv_divider(S);
-  if (d.fast) {
+  const uint32_t e = nv_factor<ALL_FAST>(__uint_as_float(m << 16), t, S);
+  const NvDivider d = nv_divider<ALL_FAST>(S);
+  if (ALL_FAST || d.fast) {
     out0 = nv_codes8_fast(pack2(neg_bf16_lo(v0.x), neg_bf16_hi(v0.x)), pack2(neg_bf16_lo(v0.y), neg_bf16_hi(v0.y)),
                           pack2(neg_bf16_lo(v0.z), neg_bf16_hi(v0.z)), pack2(neg_bf16_lo(v0.w), neg_bf16_hi(v0.w)), d);
     out1 = nv_codes8_fast(pack2(neg_bf16_lo(v1.x), neg_bf16_hi(v1.x)), pack2(neg_bf16_lo(v1.y), neg_bf16_hi(v1.y)),
@@ -185,14 +194,14 @@ __device__ __forceinline__ uint32_t nv_absmax16(const uint32_t *w) {
 // A 16-element group down one column: w[i] holds row i of two adjacent columns (the left one
 // in the low half), HI picks the right one; `m2` is nv_absmax16(w). Returns the factor byte;
 // codes in out0/out1.
-template <bool HI>
+template <bool HI, bool ALL_FAST = false>
 __device__ __forceinline__ uint32_t nv_col_group(const uint32_t *w, uint32_t m2, const NvTensor &t, uint32_t &out0,
                                                  uint32_t &out1) {
   const uint32_t m = HI ? (m2 >> 16) : (m2 & 0xFFFFu);
   float S;
-  const uint32_t e = nv_factor(__uint_as_float(m << 16), t, S);
-  const NvDivider d = nv_divider(S);
-  if (d.fast) {
+  const uint32_t e = nv_factor<ALL_FAST>(__uint_as_float(m << 16), t, S);
+  const NvDivider d = nv_divider<ALL_FAST>(S);
+  if (ALL_FAST || d.fast) {
     uint64_t n[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)

@@ -161,6 +161,25 @@ constexpr int kDualCtas = 3;                    // CTAs per SM
 constexpr int kDualStg = 8192 + 1024;           // staging of a tile's transposed codes and factors
 constexpr int kDualSmem = kDualStages * kDualStage + kDualStg + 1024 + 64;  // + alignment, barriers, flag
 
+// The four groups of 64 elements of a row held in v[0..7]: their codes in o, their factors as
+// the bytes of the result.
+template <bool ALL_FAST>
+__device__ __forceinline__ uint32_t dual_row_codes(const uint4 (&v)[8], const NvTensor &t, uint32_t (&o)[8]) {
+  uint32_t fac = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) fac |= nv_row_group<ALL_FAST>(v[2 * j], v[2 * j + 1], t, o[2 * j], o[2 * j + 1]) << (8 * j);
+  return fac;
+}
+
+// The two 16-row groups of column `col` of a column pair held in w[0..31] (m0, m1: their
+// per-half maxima): codes in o, factors e0, e1.
+template <bool ALL_FAST, bool HI>
+__device__ __forceinline__ void dual_col_codes(const uint32_t (&w)[32], uint32_t m0, uint32_t m1, const NvTensor &t,
+                                               uint32_t (&o)[4], uint32_t &e0, uint32_t &e1) {
+  e0 = nv_col_group<HI, ALL_FAST>(w, m0, t, o[0], o[1]);
+  e1 = nv_col_group<HI, ALL_FAST>(w + 16, m1, t, o[2], o[3]);
+}
+
 struct NvDualArgs {
   int64_t R, C, ldq, ldqt;
   uint8_t *Xq, *F, *XqT, *FT;
@@ -238,9 +257,9 @@ __global__ void __launch_bounds__(kThreads, kDualCtas)
         uint4 v[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = *reinterpret_cast<const uint4 *>(rp + ((k ^ (row & 7)) << 4));
-        uint32_t o[8], fac = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) fac |= nv_row_group(v[2 * j], v[2 * j + 1], t, o[2 * j], o[2 * j + 1]) << (8 * j);
+        uint32_t o[8];
+        // one branch per tile phase, uniform over the grid: the tensor decides the path
+        const uint32_t fac = t.all_fast ? dual_row_codes<true>(v, t, o) : dual_row_codes<false>(v, t, o);
         uint8_t *dq = a.Xq + gr * a.ldq + cb / 2;
         uint8_t *df = a.F + ((cb >> 8) * a.R + gr) * 16 + ((cb >> 4) & 15);
         if (cb + 64 <= a.C) {
@@ -275,10 +294,14 @@ __global__ void __launch_bounds__(kThreads, kDualCtas)
         const uint32_t m0 = nv_absmax16(w), m1 = nv_absmax16(w + 16);
 #pragma unroll
         for (int col = 0; col < 2; ++col) {
-          uint32_t o[4];
-          const uint32_t e0 = col ? nv_col_group<true>(w, m0, t, o[0], o[1]) : nv_col_group<false>(w, m0, t, o[0], o[1]);
-          const uint32_t e1 = col ? nv_col_group<true>(w + 16, m1, t, o[2], o[3])
-                                  : nv_col_group<false>(w + 16, m1, t, o[2], o[3]);
+          uint32_t o[4], e0, e1;
+          if (t.all_fast) {
+            if (col) dual_col_codes<true, true>(w, m0, m1, t, o, e0, e1);
+            else dual_col_codes<true, false>(w, m0, m1, t, o, e0, e1);
+          } else {
+            if (col) dual_col_codes<false, true>(w, m0, m1, t, o, e0, e1);
+            else dual_col_codes<false, false>(w, m0, m1, t, o, e0, e1);
+          }
           // codes of column 2p + col, rows 32 quarter .. + 31: 16-byte chunk 4 col + quarter of
           // staging pair-row p (columns 2p, 2p + 1), XOR-swizzled by p so that the eight
           // threads of a quarter warp write eight different bank groups

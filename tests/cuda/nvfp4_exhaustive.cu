@@ -4,7 +4,8 @@
 // Factors: for every positive finite BF16 tensor amax a_t (s_t = RN(a_t / 2688)) and every BF16
 // group amax a_g <= a_t, the factor byte E4M3_RNE_sat(RN(RN(a_g / 6) / s_t)) and its decoded
 // scale S = RN(dec(e) * s_t), with the divisions done by __fdiv_rn and the decode by CUDA's
-// E4M3 conversion. counts: [0] mismatches, [1] pairs checked.
+// E4M3 conversion; where the tensor takes the all-fast path (s_t >= 2^-81), that path's factor too.
+// counts: [0] mismatches, [1] pairs checked, [2] pairs checked on the all-fast path.
 //
 // Codes: for every positive finite BF16 a_t and every factor byte e (0 .. 0x7E), the scale
 // S = RN(dec(e) * s_t), and every BF16 x of either sign with S / 32 <= |x| <= 16 S (every value
@@ -32,14 +33,17 @@ __device__ __forceinline__ uint32_t e4m3_of(float v) {
   return __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
 }
 
-__device__ __forceinline__ void flush(unsigned long long *counts, unsigned long long bad, unsigned long long n) {
+__device__ __forceinline__ void flush(unsigned long long *counts, unsigned long long bad, unsigned long long n,
+                                      unsigned long long n2 = 0) {
   for (int o = 16; o > 0; o >>= 1) {
     bad += __shfl_xor_sync(0xffffffffu, bad, o);
     n += __shfl_xor_sync(0xffffffffu, n, o);
+    n2 += __shfl_xor_sync(0xffffffffu, n2, o);
   }
   if ((threadIdx.x & 31) == 0) {
     atomicAdd(counts + 0, bad);
     atomicAdd(counts + 1, n);
+    atomicAdd(counts + 2, n2);
   }
 }
 
@@ -48,7 +52,7 @@ __global__ void k_factor_check(unsigned long long *counts, unsigned int *first_b
   const float amax_t = __uint_as_float(tb << 16);
   const float s_t = __fdiv_rn(amax_t, 2688.0f);
   const puro::NvTensor t = puro::nv_tensor(amax_t);
-  unsigned long long bad = 0, n = 0;
+  unsigned long long bad = 0, n = 0, n2 = 0;
   if (threadIdx.x == 0 && __float_as_uint(t.s_t) != __float_as_uint(s_t)) {
     ++bad;
     atomicCAS(first_bad, 0u, tb << 16);
@@ -65,12 +69,19 @@ __global__ void k_factor_check(unsigned long long *counts, unsigned int *first_b
     const float S_ref = __fmul_rn(dec_e4m3(e_ref), s_t);
     float S;
     const uint32_t e = puro::nv_factor(amax_g, t, S);
-    if (e != e_ref || __float_as_uint(S) != __float_as_uint(S_ref)) {
+    bool good = e == e_ref && __float_as_uint(S) == __float_as_uint(S_ref);
+    if (t.all_fast) {
+      ++n2;
+      float S2;
+      const uint32_t e2 = puro::nv_factor<true>(amax_g, t, S2);
+      good = good && e2 == e_ref && __float_as_uint(S2) == __float_as_uint(S_ref);
+    }
+    if (!good) {
       ++bad;
       atomicCAS(first_bad, 0u, (tb << 16) | gb);
     }
   }
-  flush(counts, bad, n);
+  flush(counts, bad, n, n2);
 }
 
 // one value x (bits xb): its code by IEEE division, and by the kernels' helpers for eight
@@ -136,13 +147,13 @@ int run(void (*launch)(unsigned long long *, unsigned int *), unsigned long long
         unsigned int *host_first_bad) {
   unsigned long long *counts = nullptr;
   unsigned int *first = nullptr;
-  if (cudaMalloc(&counts, 2 * sizeof(unsigned long long)) != cudaSuccess) return 1;
+  if (cudaMalloc(&counts, 3 * sizeof(unsigned long long)) != cudaSuccess) return 1;
   if (cudaMalloc(&first, sizeof(unsigned int)) != cudaSuccess) return 2;
-  cudaMemset(counts, 0, 2 * sizeof(unsigned long long));
+  cudaMemset(counts, 0, 3 * sizeof(unsigned long long));
   cudaMemset(first, 0, sizeof(unsigned int));
   launch(counts, first);
   if (cudaGetLastError() != cudaSuccess) return 3;
-  if (cudaMemcpy(host_counts, counts, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpy(host_counts, counts, 3 * sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess)
     return 4;
   cudaMemcpy(host_first_bad, first, sizeof(unsigned int), cudaMemcpyDeviceToHost);
   cudaFree(counts);

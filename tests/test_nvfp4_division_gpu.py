@@ -15,6 +15,7 @@ import ctypes
 import os
 import subprocess
 
+import numpy as np
 import pytest
 
 from tests.conftest import ROOT
@@ -37,24 +38,28 @@ def _build():
 
 
 def test_group_factor_matches_ieee_division_exhaustively():
+    """Both the general path and, for tensors with s_t >= 2^-81, the all-fast path."""
     _build()
     lib = ctypes.CDLL(LIB)
-    counts = (ctypes.c_ulonglong * 2)()
+    counts = (ctypes.c_ulonglong * 3)()
     first = ctypes.c_uint(0)
     assert lib.run_nvfp4_factor_check(counts, ctypes.byref(first)) == 0
-    bad, checked = list(counts)
+    bad, checked, checked_all_fast = list(counts)
     n_t = 0x7F7F
     assert checked == n_t * (n_t + 1) // 2 + n_t  # group amax 0 .. tensor amax, per tensor amax
+    tb = np.arange(1, n_t + 1, dtype=np.uint32)
+    s_t = (tb << 16).view(np.float32) / np.float32(2688.0)  # IEEE float32 division
+    assert checked_all_fast == int((tb[s_t >= np.float32(2.0 ** -81)].astype(np.int64) + 1).sum())
     assert bad == 0, f"{bad} factor mismatches, first (tensor amax << 16 | group amax) = {first.value:#010x}"
 
 
 def test_codes_match_ieee_division_exhaustively():
     _build()
     lib = ctypes.CDLL(LIB)
-    counts = (ctypes.c_ulonglong * 2)()
+    counts = (ctypes.c_ulonglong * 3)()
     first = ctypes.c_uint(0)
     assert lib.run_nvfp4_codes_check(counts, ctypes.byref(first)) == 0
-    bad, checked = list(counts)
+    bad, checked, _ = list(counts)
     print(f"values checked: {checked}")
     # 0x7F7F tensor amaxes x 126 non-zero factors x (about 9 binades of 128 values, 2 signs)
     assert checked > 0x7F7F * 126 * 1500
