@@ -245,7 +245,14 @@ def test_quant_dual_special_groups(pf):
     x[2, 32:48] = 1e-30
     x[16:32, 40] = 1e-30
     x[5, 7] = -3000.0  # the tensor amax
-    for t in (x, torch.zeros((64, 32), dtype=torch.bfloat16), (torch.randn((64, 48)) * 1e-38).to(torch.bfloat16)):
+    # s_t >= 2^-81 with groups below 2^-100 (the all-fast path); s_t between 2^-90 and 2^-81 (the
+    # per-group path); s_t below 2^-90 (IEEE division)
+    small = (torch.randn((64, 64)) * 1e-20).to(torch.bfloat16)
+    small[3, :16] = 1e-32
+    small[:16, 40] = -1e-33
+    mid = (torch.randn((64, 32)) * 1e-24).to(torch.bfloat16)
+    for t in (x, torch.zeros((64, 32), dtype=torch.bfloat16), (torch.randn((64, 48)) * 1e-38).to(torch.bfloat16),
+              small, mid):
         q, f, qt, ft, amax = run_dual(pf, t.cuda())
         wq, wf, wa = onv.quant_1x16(bits_of(t))
         tq, tf, _ = onv.quant_1x16_transposed(bits_of(t))
