@@ -153,6 +153,17 @@ __global__ void __launch_bounds__(kThreads) k_nv_quant_cols(const uint16_t *__re
 
 // ---------------------------------------------------------------- both layouts, one read
 
+#ifdef PURO_TEST_HOOKS
+// Test builds only, never libpuro_fp8.so: while set, each CTA of the dual kernel skips the load
+// of its first tile, so the bounded wait for it runs out. The failure-detection test uses this
+// to check that the give-up reaches the status word and that the kernel drains and exits with
+// the context intact.
+__device__ int g_test_nv_skip_load;
+#define PURO_NV_SKIP_LOAD(i) (g_test_nv_skip_load != 0 && (i) == 0)
+#else
+#define PURO_NV_SKIP_LOAD(i) false
+#endif
+
 constexpr int kDualTile = 128;                  // rows and columns of a tile
 constexpr int kDualBox = kDualTile * 128;       // one TMA box: 128 rows x 64 BF16 (128 bytes)
 constexpr int kDualStage = 2 * kDualBox;        // one tile, 32 KB
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, kDualCtas)
   __syncthreads();
   auto issue = [&](int i) {
     const int tile = blockIdx.x + i * gridDim.x;
-    if (tile >= a.tiles) return;
+    if (tile >= a.tiles || PURO_NV_SKIP_LOAD(i)) return;
     const int tr = tile / a.tiles_c, tc = tile - tr * a.tiles_c;
     const uint32_t bar = bar0 + 8 * (i % kDualStages), dst = sbase + (i % kDualStages) * kDualStage;
     mbar_arrive_expect_tx(bar, kDualStage);
@@ -431,3 +442,9 @@ int launch_nvfp4_quant_dual(const uint16_t *X, int64_t R, int64_t C, int64_t ldx
 }
 
 }  // namespace puro
+
+#ifdef PURO_TEST_HOOKS
+extern "C" __attribute__((visibility("default"))) int puro_test_set_nv_skip_load(int on) {
+  return cudaMemcpyToSymbol(puro::g_test_nv_skip_load, &on, sizeof(int)) == cudaSuccess ? 0 : -1;
+}
+#endif

@@ -7,7 +7,7 @@ PURO_TEST_HOOKS, a flag libpuro_fp8.so never sets) has two more hooks:
   the MMA issuer's bounded wait for the scale factors runs out (single CTA and CTA pair,
   fprop and wgrad);
 * the quantiser skips the load of each CTA's first tile, so the bounded wait for it runs
-  out (row-wise, dual and grouped weight launches).
+  out (row-wise, dual and grouped weight launches), and so does the NVFP4 dual quantiser.
 
 In a child process whose wait limit is 20 ms, each call is accepted (the give-up happens on
 the device), puro_fp8_sync_status() reports PURO_ERR_TIMEOUT and clears the status word,
@@ -112,6 +112,39 @@ print("RESULT", *out, flush=True)
 """
 
 
+CHILD_NV = r"""
+import ctypes, sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[2])
+from oracle import nvfp4 as onv
+lib = ctypes.CDLL(sys.argv[1])
+p, i64 = ctypes.c_void_p, ctypes.c_int64
+lib.puro_nvfp4_quantize_1x16_dual.argtypes = [p, i64, i64, i64, p, i64, p, p, i64, p, p, p]
+lib.puro_fp8_sync_status.argtypes = [p]
+R, Cn = 512, 384
+x = (torch.randn((R, Cn), generator=torch.Generator().manual_seed(4)) * 2.0).to(torch.bfloat16)
+bits = x.view(torch.int16).numpy().view(np.uint16)
+xd = x.cuda()
+st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+u8 = torch.uint8
+q = torch.zeros((R, Cn // 2), dtype=u8, device="cuda"); f = torch.zeros(((Cn + 255) // 256, R, 16), dtype=u8, device="cuda")
+qt = torch.zeros((Cn, R // 2), dtype=u8, device="cuda"); ft = torch.zeros(((R + 255) // 256, Cn, 16), dtype=u8, device="cuda")
+amax = torch.zeros(1, device="cuda")
+call = lambda: lib.puro_nvfp4_quantize_1x16_dual(xd.data_ptr(), R, Cn, Cn, q.data_ptr(), Cn // 2, f.data_ptr(),
+                                                  qt.data_ptr(), R // 2, ft.data_ptr(), amax.data_ptr(), st)
+out = [lib.puro_test_set_nv_skip_load(1), call(), lib.puro_fp8_sync_status(st), lib.puro_fp8_sync_status(st),
+       lib.puro_test_set_nv_skip_load(0), call(), lib.puro_fp8_sync_status(st)]
+by_row = lambda fb, groups: fb.transpose(1, 0, 2).reshape(fb.shape[1], -1)[:, :groups]  # [K blocks, rows, 16]
+wq, wf, _ = onv.quant_1x16(bits)
+tq, tf, _ = onv.quant_1x16_transposed(bits)
+exact = (np.array_equal(q.cpu().numpy(), wq) and np.array_equal(by_row(f.cpu().numpy(), Cn // 16), wf)
+         and np.array_equal(qt.cpu().numpy(), tq) and np.array_equal(by_row(ft.cpu().numpy(), R // 16), tf))
+out.append(int(exact))
+print("RESULT", *out, flush=True)
+"""
+
+
 def _run(child, *args):
     env = dict(os.environ, PURO_WAIT_TIMEOUT_MS="20")
     r = subprocess.run([sys.executable, "-c", child, LIB, *map(str, args)], capture_output=True, text=True,
@@ -138,3 +171,8 @@ def test_mx_gemm_wait_gives_up_reports_timeout_and_context_survives(layout, m):
 def test_quantiser_wait_gives_up_reports_timeout_and_context_survives(mode):
     _build()
     _run(CHILD_QUANT, mode, ROOT)
+
+
+def test_nvfp4_dual_quantiser_wait_gives_up_reports_timeout_and_context_survives():
+    _build()
+    _run(CHILD_NV, ROOT)
