@@ -287,6 +287,34 @@ def test_quant_dual_full_size(pf, R, C):
     assert np.array_equal(unblocked(ft.cpu().numpy(), R // 16)[cols], fac)
 
 
+def test_linear_pass_on_dual_operands(pf):
+    """One linear's three GEMMs as the NVFP4 step runs them, every operand from the dual
+    quantiser: fprop X . W^T, dgrad dY . W (W quantised along N_out), wgrad dY^T . X (both along
+    the tokens), each within the tolerance of the oracle's contraction of the oracle's own
+    quantisation of the same BF16 tensors."""
+    T, K, N = 256, 512, 384
+    x = rand_bf16((T, K), 50)
+    w = rand_bf16((N, K), 51, scale=0.02, tails=False)
+    dy = rand_bf16((T, N), 52, scale=1e-3)
+    (xq, xf), (xqt, xft), xa = pf.nvfp4_quantize_dual(x.cuda())
+    (wq, wf), (wqt, wft), wa = pf.nvfp4_quantize_dual(w.cuda())
+    (dq, df), (dqt, dft), da = pf.nvfp4_quantize_dual(dy.cuda())
+    got = {"fprop": pf.nvfp4_gemm(xq, xf, xa, wq, wf, wa),
+           "dgrad": pf.nvfp4_gemm(dq, df, da, wqt, wft, wa),
+           "wgrad": pf.nvfp4_gemm(dqt, dft, da, xqt, xft, xa)}
+    sync(pf)
+    rows, cols = onv.quant_1x16, onv.quant_1x16_transposed
+    ops = {"fprop": (rows(bits_of(x)), rows(bits_of(w))),
+           "dgrad": (rows(bits_of(dy)), cols(bits_of(w))),
+           "wgrad": (cols(bits_of(dy)), cols(bits_of(x)))}
+    for name, ((aq, af, aa), (bq, bf, ba)) in ops.items():
+        want = onv.gemm_ref(aq, af, aa, bq, bf, ba)
+        na, nb = onv.row_col_norms(aq, af, aa, bq, bf, ba)
+        c = got[name].float().cpu().numpy().astype(np.float64)
+        assert c.shape == want.shape, name
+        _tolerance_check(c, want, na, nb)
+
+
 def test_argument_errors(pf):
     lib = pf.library()
     st = pf._stream(None)
