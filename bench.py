@@ -85,13 +85,31 @@ def _args():
     return p.parse_args()
 
 
-def _peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = (6650.0, 1590.0, 1400.0)  # HBM GB/s, BF16 TFLOP/s burst, BF16 TFLOP/s sustained
+
+
+def _peaks(path=None):
+    """(HBM GB/s, BF16 TFLOP/s burst, BF16 TFLOP/s sustained, source) from the measured-peaks file
+    when it is there and readable (a value may also be an object holding "value"), else the
+    fallback figures."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
-        with open(path) as f:
-            d = json.load(f)
-        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
-    return 6650.0, 1590.0, 1400.0, "fallback"
+        try:
+            with open(path) as f:
+                d = json.load(f)
+            vals = []
+            for key in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained"):
+                v = d[key]
+                if isinstance(v, dict):
+                    v = v["value"]
+                v = float(v)
+                if not v > 0:
+                    raise ValueError(f"{key} = {v}")
+                vals.append(v)
+            return vals[0], vals[1], vals[2], "measured"
+        except (OSError, ValueError, TypeError, KeyError) as e:
+            print(f"bench: {path} not usable ({e!r}); using the fallback peaks", file=sys.stderr)
+    return (*FALLBACK_PEAKS, "fallback")
 
 
 # ------------------------------------------------------------------ DRAM traffic (ncu)
